@@ -1,0 +1,210 @@
+"""ctypes binding of the CPU oracle (TEST INFRASTRUCTURE ONLY).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg import this package.  It restates, slowly and plainly, what the GPU path
+computes; it never imports the product package and the product never imports
+it.  Every function takes and returns numpy arrays.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+UNIFORM, EXP = 0, 1
+SCALE_L2, SCALE_MAXABS = 0, 1
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64, i32, u32, u64, f32 = (ctypes.c_int64, ctypes.c_int, ctypes.c_uint32,
+                                   ctypes.c_uint64, ctypes.c_float)
+        L.gqo_philox4x32.argtypes = [P, u32, u32, i32]
+        L.gqo_philox4x32.restype = None
+        L.gqo_uniform_bits.argtypes = [u64, u32, u32, u32, u64]
+        L.gqo_uniform_bits.restype = u32
+        L.gqo_sumsq.argtypes = [P, P, i64]
+        L.gqo_sumsq.restype = ctypes.c_double
+        L.gqo_maxabs.argtypes = [P, P, i64]
+        L.gqo_maxabs.restype = f32
+        L.gqo_global_scale.argtypes = [P, P, i32, i64, i32, P, P]
+        L.gqo_quantize.argtypes = [P, P, i32, i64, P, i32, i32, i32, u64, u32, f32, P]
+        L.gqo_code_value.argtypes = [i32, i32, i32]
+        L.gqo_code_value.restype = i32
+        L.gqo_packed_row_bytes.argtypes = [i32, i64]
+        L.gqo_packed_row_bytes.restype = i64
+        L.gqo_pack.argtypes = [P, i32, i64, i32, P]
+        L.gqo_unpack.argtypes = [P, i32, i64, i32, P]
+        L.gqo_aggregate.argtypes = [P, i32, i64, i32, i32, P]
+        L.gqo_decode_mean.argtypes = [P, i64, i32, i32, i32, i32, f32, P]
+        L.gqo_error_feedback.argtypes = [P, P, P, i32, i64, i32, i32, i32, f32, P]
+        L.gqo_logq_quantize.argtypes = [P, i32, i32, P, f32, u64, u32, P, P]
+        L.gqo_logq_decode_sum.argtypes = [P, P, i32, i32, P, f32, P]
+        L.gqo_logq_map.argtypes = [f32, f32]
+        L.gqo_logq_map.restype = f32
+        L.gqo_logq_decode_one.argtypes = [i32, f32, f32]
+        L.gqo_logq_decode_one.restype = f32
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (rc={rc})")
+
+
+def philox4x32(ctr, key, rounds=10):
+    c = np.ascontiguousarray(np.asarray(ctr, dtype=np.uint32).copy())
+    lib().gqo_philox4x32(_p(c), int(key[0]) & 0xFFFFFFFF, int(key[1]) & 0xFFFFFFFF,
+                         rounds)
+    return c
+
+
+def uniform_bits(seed, tag, step, worker, j):
+    return lib().gqo_uniform_bits(seed, tag, step, worker, j)
+
+
+def sumsq(g, e=None):
+    g = _f32(g)
+    e = _f32(e)
+    return lib().gqo_sumsq(_p(g), _p(e), g.size)
+
+
+def global_scale(g, e=None, scale_kind=SCALE_L2):
+    """g, e: [W][d] float32.  Returns (S, norms[W] float64)."""
+    g = _f32(g)
+    e = _f32(e)
+    W, d = g.shape
+    S = np.zeros(1, np.float32)
+    norms = np.zeros(W, np.float64)
+    _check(lib().gqo_global_scale(_p(g), _p(e), W, d, scale_kind, _p(S), _p(norms)),
+           "global_scale")
+    return np.float32(S[0]), norms
+
+
+def quantize(g, e=None, *, levels=UNIFORM, s=15, L=8, seed=0, step=0, S, js=None):
+    """Codes [W][n] int32 for v = g + e at coordinates js (default 0..n-1)."""
+    g = _f32(g)
+    e = _f32(e)
+    W, n = g.shape
+    jsa = None if js is None else np.ascontiguousarray(js, dtype=np.int64)
+    out = np.zeros((W, n), np.int32)
+    _check(lib().gqo_quantize(_p(g), _p(e), W, n, _p(jsa), levels, s, L, seed, step,
+                              float(S), _p(out)), "quantize")
+    return out
+
+
+def code_value(code, levels, L=8):
+    return lib().gqo_code_value(int(code), levels, L)
+
+
+def packed_row_bytes(bits, d):
+    return lib().gqo_packed_row_bytes(bits, d)
+
+
+def pack(codes, bits):
+    codes = np.ascontiguousarray(codes, dtype=np.int32)
+    W, d = codes.shape
+    rb = packed_row_bytes(bits, d)
+    if rb < 0:
+        raise ValueError("bad bit width")
+    out = np.zeros((W, rb), np.uint8)
+    _check(lib().gqo_pack(_p(codes), W, d, bits, _p(out)), "pack")
+    return out
+
+
+def unpack(packed, W, d, bits):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    out = np.zeros((W, d), np.int32)
+    _check(lib().gqo_unpack(_p(packed), W, d, bits, _p(out)), "unpack")
+    return out
+
+
+def aggregate(codes, *, levels=UNIFORM, L=8):
+    codes = np.ascontiguousarray(codes, dtype=np.int32)
+    W, n = codes.shape
+    out = np.zeros(n, np.int32)
+    _check(lib().gqo_aggregate(_p(codes), W, n, levels, L, _p(out)), "aggregate")
+    return out
+
+
+def decode_mean(sum_, W, *, levels=UNIFORM, s=15, L=8, S):
+    sum_ = np.ascontiguousarray(sum_, dtype=np.int32)
+    out = np.zeros(sum_.shape[0], np.float32)
+    _check(lib().gqo_decode_mean(_p(sum_), sum_.shape[0], W, levels, s, L, float(S),
+                                 _p(out)), "decode_mean")
+    return out
+
+
+def error_feedback(g, e, codes, *, levels=UNIFORM, s=15, L=8, S):
+    g = _f32(g)
+    e = _f32(e)
+    codes = np.ascontiguousarray(codes, dtype=np.int32)
+    W, n = g.shape
+    out = np.zeros((W, n), np.float32)
+    _check(lib().gqo_error_feedback(_p(g), _p(e), _p(codes), W, n, levels, s, L,
+                                    float(S), _p(out)), "error_feedback")
+    return out
+
+
+def step(g, e=None, *, levels=UNIFORM, s=15, L=8, scale_kind=SCALE_L2, seed=0,
+         step=0, ef=False, bits=None, S=None):
+    """The whole path on [W][d] inputs: scale, codes, packed bytes, integer sum,
+    decoded mean and (ef=True) the new error buffer.  S, when given, replaces
+    the computed scale (the GPU's scale, for bit-exact comparison)."""
+    g = _f32(g)
+    e = _f32(e) if ef else None
+    S_ref, norms = global_scale(g, e, scale_kind)
+    S_use = S_ref if S is None else np.float32(S)
+    codes = quantize(g, e, levels=levels, s=s, L=L, seed=seed, step=step, S=S_use)
+    packed = pack(codes, bits) if bits else None
+    total = aggregate(codes, levels=levels, L=L)
+    out = decode_mean(total, g.shape[0], levels=levels, s=s, L=L, S=S_use)
+    e_new = error_feedback(g, e, codes, levels=levels, s=s, L=L, S=S_use) if ef else None
+    return dict(S=S_ref, norms=norms, codes=codes, packed=packed, sum=total, out=out,
+                e=e_new)
+
+
+def logq_quantize(x, sizes, *, alpha=10.0, seed=0, step=0):
+    """x: [W][sum(sizes)] float32.  Returns (maxabs[W][nmats], codes int8)."""
+    x = _f32(x)
+    W = x.shape[0]
+    sz = np.ascontiguousarray(sizes, dtype=np.int64)
+    mx = np.zeros((W, sz.size), np.float32)
+    codes = np.zeros(x.shape, np.int8)
+    _check(lib().gqo_logq_quantize(_p(x), W, sz.size, _p(sz), alpha, seed, step, _p(mx),
+                                   _p(codes)), "logq_quantize")
+    return mx, codes
+
+
+def logq_decode_sum(codes, maxabs, sizes, *, alpha=10.0):
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    maxabs = _f32(maxabs)
+    sz = np.ascontiguousarray(sizes, dtype=np.int64)
+    out = np.zeros(codes.shape[1], np.float32)
+    _check(lib().gqo_logq_decode_sum(_p(codes), _p(maxabs), codes.shape[0], sz.size,
+                                     _p(sz), alpha, _p(out)), "logq_decode_sum")
+    return out
+
+
+def logq_map(xn, alpha=10.0):
+    return lib().gqo_logq_map(xn, alpha)
+
+
+def logq_decode_one(k, m, alpha=10.0):
+    return lib().gqo_logq_decode_one(k, m, alpha)

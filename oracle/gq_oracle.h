@@ -1,0 +1,137 @@
+/*
+ * gq_oracle.h -- the CPU oracle for allreduce-compatible global gradient
+ * quantization.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is the slow, single-threaded, obviously
+ * correct restatement of what the GPU path computes.  Only the test suite,
+ * the smoke check and the benchmark's CPU-baseline leg may load it.  It
+ * shares no code, header, table or constant generator with the CUDA library
+ * under allreduce_compatible_gradient_global_b200/csrc, and the library never
+ * calls it.
+ *
+ * Sources (page title, then the passage):
+ *  [GQ]  "Quantize Once, Train Fast: Allreduce-Compatible Compression with
+ *        Provable Guarantees" -- Abstract: one global norm scale shared by all
+ *        workers makes the quantized gradients summable by Allreduce; the
+ *        compressor is of the unbiased kind.
+ *  [SM]  "Unbiased Single-scale and Multi-scale Quantizers for Distributed
+ *        Optimization" -- Abstract: all-reduce compatible compressors.
+ *  [NUQ] "NUQSGD: Provably Communication-efficient Data-parallel SGD via
+ *        Nonuniform Quantization" -- Abstract: QSGD, its max-norm heuristic
+ *        QSGDinf, and nonuniform levels.
+ *  [LQ]  "Trustworthy Efficient Communication for Distributed Learning using
+ *        LQ-SGD Algorithm" -- review sections "Core claim" (log map, 2^b bins,
+ *        b = 8, r(n+m)*b bits), "What carries the argument" (error feedback
+ *        E_t = G'_t - Ghat_t), and referee major comment 1 on Section IV-A,
+ *        Eqs. (5)-(6) (normalise by the maximum magnitude; Eq. (6) inverts
+ *        the map).
+ *
+ * Where the pages leave a step open, the reading taken is stated at the
+ * function.  Floating-point steps are fp32 in a fixed order with no FMA
+ * contraction (the file is built with -ffp-contract=off); norms are fp64.
+ *
+ * Pins: every function here is checked by the CPU tests against closed forms,
+ * exact enumeration, Monte Carlo bounds, invariants, and (for Philox) the
+ * cuRAND host generator, never against the GPU path.
+ */
+#ifndef GQ_ORACLE_H
+#define GQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { GQO_UNIFORM = 0, GQO_EXP = 1 };
+enum { GQO_SCALE_L2 = 0, GQO_SCALE_MAXABS = 1 };
+
+/* Philox-4x32 with `rounds` rounds (10 for Philox-4x32-10), written from
+ * Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3"
+ * (SC'11).  ctr is updated in place to the output block. */
+void gqo_philox4x32(uint32_t ctr[4], uint32_t k0, uint32_t k1, int rounds);
+
+/* The 23-bit uniform integer f (u = f * 2^-23) drawn for coordinate j of
+ * worker `worker` at step `step`: key = (lo32 seed, hi32 seed ^ tag),
+ * counter = (lo32(j>>2), step, worker, hi32(j>>2)), output word j & 3,
+ * low 23 bits. */
+uint32_t gqo_uniform_bits(uint64_t seed, uint32_t tag, uint32_t step,
+                          uint32_t worker, uint64_t j);
+
+/* fp64 sum of squares of fl(g[i] + e[i]) (or g[i] when e is NULL), i
+ * ascending from 0 to n-1.  Chunked calls accumulate in the same order when
+ * the caller adds the partials in ascending chunk order. */
+double gqo_sumsq(const float* g, const float* e, int64_t n);
+
+/* max |fl(g+e)| over n entries; NaN if any entry is NaN. */
+float gqo_maxabs(const float* g, const float* e, int64_t n);
+
+/* Global scale [GQ]: L2 -> S = (float) max_w sqrt(sum_j v_wj^2) (fp64);
+ * MAXABS ([NUQ] QSGDinf) -> S = max_{w,j} |v_wj|.  norms_out (may be NULL)
+ * gets the W per-worker norms (fp64; for MAXABS the per-worker max).
+ * Returns 0, or -1 on bad arguments. */
+int gqo_global_scale(const float* g, const float* e, int W, int64_t d,
+                     int scale_kind, float* S_out, double* norms_out);
+
+/* Stochastic quantization of v = fl(g + e) (e may be NULL) given the scale S.
+ * g and e are [W][n]; coordinate index of column i is js[i] (or i when js is
+ * NULL), which keys the uniform.  codes_out is [W][n] int32.
+ * levels: GQO_UNIFORM with s >= 1, or GQO_EXP with 1 <= L <= 15.
+ * Returns 0, or -1 on bad arguments. */
+int gqo_quantize(const float* g, const float* e, int W, int64_t n,
+                 const int64_t* js, int levels, int s, int L,
+                 uint64_t seed, uint32_t step, float S, int32_t* codes_out);
+
+/* The integer each code contributes to the sum: the code itself (UNIFORM) or
+ * sign * 2^(idx-1) units of the finest level 2^-(L-1) (EXP, idx = |code|). */
+int32_t gqo_code_value(int32_t code, int levels, int L);
+
+/* Bytes per worker row of packed codes at `bits` in {4,5,8,16}:
+ * ceil(d/128) blocks of 16*bits bytes. */
+int64_t gqo_packed_row_bytes(int bits, int64_t d);
+
+/* Pack [W][d] int32 codes at wire width into [W][row_bytes] bytes.
+ * 4/5 bits: little-endian bitstream, code j in bits [b*j, b*j+b) of the row,
+ * two's complement, zero padding.  8: int8 per code.  16: int16 per code.
+ * Returns 0, -1 on bad arguments, -2 if a code does not fit. */
+int gqo_pack(const int32_t* codes, int W, int64_t d, int bits, uint8_t* out);
+int gqo_unpack(const uint8_t* packed, int W, int64_t d, int bits,
+               int32_t* codes_out);
+
+/* Simulated Allreduce [GQ][SM]: sum_out[i] = sum_w value(code[w][i]) in
+ * int32, w ascending. */
+int gqo_aggregate(const int32_t* codes, int W, int64_t n, int levels, int L,
+                  int32_t* sum_out);
+
+/* Decode the summed integers to the mean: c = fl(S/s) (UNIFORM) or
+ * fl(S * 2^-(L-1)) (EXP); out = fl(fl((float)sum * c) / (float)W). */
+int gqo_decode_mean(const int32_t* sum, int64_t n, int W, int levels, int s,
+                    int L, float S, float* out);
+
+/* Error feedback: e_out = fl(v - fl((float)value(code) * c)), v = fl(g+e_in)
+ * (e_in may be NULL = zeros), c as in gqo_decode_mean.  [W][n] arrays. */
+int gqo_error_feedback(const float* g, const float* e_in,
+                       const int32_t* codes, int W, int64_t n, int levels,
+                       int s, int L, float S, float* e_out);
+
+/* [LQ] log quantizer.  x is [W][total] with the nmats matrices of each
+ * worker concatenated; sizes[m] = rows*cols of matrix m.  maxabs_out is
+ * [W][nmats]; codes_out is [W][total] int8.  Returns 0 or -1. */
+int gqo_logq_quantize(const float* x, int W, int nmats, const int64_t* sizes,
+                      float alpha, uint64_t seed, uint32_t step,
+                      float* maxabs_out, int8_t* codes_out);
+
+/* [LQ] Eq. (6) decode of every worker's codes, fp32 sum over workers in
+ * ascending order.  out is [total]. */
+int gqo_logq_decode_sum(const int8_t* codes, const float* maxabs, int W,
+                        int nmats, const int64_t* sizes, float alpha,
+                        float* out);
+
+/* Single-entry forms of the log map, for the property tests. */
+float gqo_logq_map(float xn, float alpha);           /* log1p(a*xn)/log1p(a) */
+float gqo_logq_decode_one(int32_t k, float m, float alpha);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
