@@ -1,0 +1,328 @@
+"""Python binding of libgq: allreduce-compatible global gradient quantization
+on one B200 (sm_100a).
+
+A thin ctypes layer over the C ABI in ``include/gq_api.h``: every function has
+the C entry point's name, takes torch tensors (device memory and streams come
+from PyTorch), checks dtypes and shapes, passes raw pointers and raises
+``GQError`` on a non-zero status.  All arithmetic runs in the CUDA kernels of
+libgq.so; there is no fallback: if the library is missing, importing this
+package fails with instructions to build it.
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgq.so")
+
+GQ_OK = 0
+GQ_ERR_ARG = -1
+GQ_ERR_OVERFLOW = -2
+GQ_ERR_ALIGN = -3
+GQ_ERR_CUDA = -4
+GQ_ERR_NONFINITE = -5
+
+UNIFORM, EXP, LOG = 0, 1, 2
+SCALE_L2, SCALE_MAXABS = 0, 1
+WIRE_INT8, WIRE_INT16 = 1, 2
+
+_LEVELS = {"uniform": UNIFORM, "exp": EXP, "log": LOG}
+_SCALES = {"l2": SCALE_L2, "maxabs": SCALE_MAXABS}
+_WIRES = {"int8": WIRE_INT8, "int16": WIRE_INT16}
+
+
+class GQError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {gq_status_string(status)} (status {status})")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("levels", ctypes.c_int), ("s", ctypes.c_int), ("L", ctypes.c_int),
+                ("bits", ctypes.c_int), ("scale_kind", ctypes.c_int), ("wire", ctypes.c_int),
+                ("ef", ctypes.c_int), ("alpha", ctypes.c_float),
+                ("seed", ctypes.c_ulonglong), ("step", ctypes.c_uint)]
+
+
+@dataclass
+class GQConfig:
+    """Mirror of ``gq_config``.  String forms are accepted for the enums."""
+    levels: object = "uniform"
+    s: int = 15
+    L: int = 8
+    bits: int = 5
+    scale_kind: object = "l2"
+    wire: object = "int8"
+    ef: bool = False
+    alpha: float = 10.0
+    seed: int = 0
+    step: int = 0
+
+    def c(self) -> _Config:
+        lv = _LEVELS.get(self.levels, self.levels)
+        sk = _SCALES.get(self.scale_kind, self.scale_kind)
+        wr = _WIRES.get(self.wire, self.wire)
+        return _Config(int(lv), int(self.s), int(self.L), int(self.bits), int(sk), int(wr),
+                       1 if self.ef else 0, float(self.alpha),
+                       int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.step) & 0xFFFFFFFF)
+
+    @property
+    def wire_dtype(self):
+        return torch.int8 if _WIRES.get(self.wire, self.wire) == WIRE_INT8 else torch.int16
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m allreduce_compatible_gradient_global_b200.build` "
+            "(or __graft_entry__.build()); there is no CPU fallback")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
+    CP = ctypes.POINTER(_Config)
+    sig = {
+        "gq_version": ([], I),
+        "gq_status_string": ([I], ctypes.c_char_p),
+        "gq_validate": ([CP, I, LL], I),
+        "gq_packed_row_bytes": ([CP, LL, ctypes.POINTER(LL)], I),
+        "gq_workspace_bytes": ([CP, I, LL, ctypes.POINTER(ctypes.c_size_t)], I),
+        "gq_workspace_init": ([P, ctypes.c_size_t, P], I),
+        "gq_get_device_status": ([P, P], I),
+        "gq_global_norm": ([P, P, I, LL, CP, P, P, P, P], I),
+        "gq_quantize_pack": ([P, P, I, LL, CP, P, P, P, P], I),
+        "gq_aggregate": ([P, I, LL, CP, P, P, P], I),
+        "gq_dequantize_ef": ([P, P, P, P, I, LL, CP, P, P, P, P], I),
+        "gq_quantize_aggregate": ([P, P, I, LL, CP, P, P, P, P, P, P], I),
+        "gq_step_fused": ([P, P, I, LL, CP, P, P, P, P, P, P, P], I),
+        "gq_step_fused_host": ([P, P, P, I, LL, CP, P, P, P, P, P, P, P, P], I),
+        "gq_logq_quantize": ([P, I, I, P, P, CP, P, P, P, P], I),
+        "gq_logq_decode_sum": ([P, P, I, I, P, P, CP, P, P], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def gq_version() -> int:
+    return _lib.gq_version()
+
+
+def gq_status_string(status: int) -> str:
+    return _lib.gq_status_string(int(status)).decode()
+
+
+# ------------------------------------------------------------------ marshalling
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc, what):
+    if rc != GQ_OK:
+        raise GQError(rc, what)
+
+
+def _need(t, dtype, shape, name, cuda=True):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if cuda and not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _wd(g):
+    if g.dim() != 2:
+        raise ValueError("gradients must be [W][d]")
+    return int(g.shape[0]), int(g.shape[1])
+
+
+# ------------------------------------------------------------------ sizes
+def gq_validate(cfg: GQConfig, W: int, d: int) -> int:
+    c = cfg.c()
+    return _lib.gq_validate(ctypes.byref(c), int(W), int(d))
+
+
+def gq_packed_row_bytes(cfg: GQConfig, d: int) -> int:
+    c = cfg.c()
+    out = ctypes.c_longlong()
+    _check(_lib.gq_packed_row_bytes(ctypes.byref(c), int(d), ctypes.byref(out)),
+           "gq_packed_row_bytes")
+    return out.value
+
+
+def gq_workspace_bytes(cfg: GQConfig, W: int, d: int) -> int:
+    c = cfg.c()
+    out = ctypes.c_size_t()
+    _check(_lib.gq_workspace_bytes(ctypes.byref(c), int(W), int(d), ctypes.byref(out)),
+           "gq_workspace_bytes")
+    return out.value
+
+
+def gq_workspace_init(ws, stream=None):
+    _check(_lib.gq_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "gq_workspace_init")
+
+
+def gq_get_device_status(ws, stream=None) -> int:
+    """Synchronizes the stream; returns GQ_OK or GQ_ERR_NONFINITE (and clears it)."""
+    rc = _lib.gq_get_device_status(_ptr(ws), _stream(stream))
+    if rc not in (GQ_OK, GQ_ERR_NONFINITE):
+        raise GQError(rc, "gq_get_device_status")
+    return rc
+
+
+# ------------------------------------------------------------------ the path
+def gq_global_norm(g, e, cfg: GQConfig, scale, norms, ws, stream=None):
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(scale, torch.float32, (1,), "scale")
+    _need(norms, torch.float64, (W,), "norms")
+    c = cfg.c()
+    _check(_lib.gq_global_norm(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale), _ptr(norms),
+                               _ptr(ws), _stream(stream)), "gq_global_norm")
+
+
+def gq_quantize_pack(g, e, cfg: GQConfig, scale, codes, ws, stream=None):
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
+    c = cfg.c()
+    _check(_lib.gq_quantize_pack(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale),
+                                 _ptr(codes), _ptr(ws), _stream(stream)), "gq_quantize_pack")
+
+
+def gq_aggregate(codes, W, d, cfg: GQConfig, sum_out, ws, stream=None):
+    _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
+    _need(sum_out, cfg.wire_dtype, (d,), "sum")
+    c = cfg.c()
+    _check(_lib.gq_aggregate(_ptr(codes), int(W), int(d), ctypes.byref(c), _ptr(sum_out),
+                             _ptr(ws), _stream(stream)), "gq_aggregate")
+
+
+def gq_dequantize_ef(sum_in, codes, g, e, W, d, cfg: GQConfig, scale, out, ws, stream=None):
+    _need(sum_in, cfg.wire_dtype, (d,), "sum")
+    _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(out, torch.float32, (d,), "out")
+    c = cfg.c()
+    _check(_lib.gq_dequantize_ef(_ptr(sum_in), _ptr(codes), _ptr(g), _ptr(e), int(W), int(d),
+                                 ctypes.byref(c), _ptr(scale), _ptr(out), _ptr(ws),
+                                 _stream(stream)), "gq_dequantize_ef")
+
+
+def gq_quantize_aggregate(g, e, cfg: GQConfig, scale, codes, sum_out, out, ws, stream=None):
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
+    _need(sum_out, cfg.wire_dtype, (d,), "sum")
+    _need(out, torch.float32, (d,), "out")
+    c = cfg.c()
+    _check(_lib.gq_quantize_aggregate(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale),
+                                      _ptr(codes), _ptr(sum_out), _ptr(out), _ptr(ws),
+                                      _stream(stream)), "gq_quantize_aggregate")
+
+
+def gq_step_fused(g, e, cfg: GQConfig, scale, norms, codes, sum_out, out, ws, stream=None):
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(scale, torch.float32, (1,), "scale")
+    _need(norms, torch.float64, (W,), "norms")
+    _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
+    _need(sum_out, cfg.wire_dtype, (d,), "sum")
+    _need(out, torch.float32, (d,), "out")
+    c = cfg.c()
+    _check(_lib.gq_step_fused(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale), _ptr(norms),
+                              _ptr(codes), _ptr(sum_out), _ptr(out), _ptr(ws), _stream(stream)),
+           "gq_step_fused")
+
+
+def gq_step_fused_host(g_host, g_dev, e, cfg: GQConfig, scale, codes, sum_out, out, out_host,
+                       scale_host, ws, stream=None):
+    """g_host / out_host / scale_host: CPU tensors (pinned for full speed)."""
+    W, d = _wd(g_dev)
+    _need(g_host, torch.float32, (W, d), "g_host", cuda=False)
+    _need(out_host, torch.float32, (d,), "out_host", cuda=False)
+    _need(scale_host, torch.float32, (1,), "scale_host", cuda=False)
+    _need(g_dev, torch.float32, (W, d), "g_dev")
+    _need(out, torch.float32, (d,), "out")
+    c = cfg.c()
+    _check(_lib.gq_step_fused_host(_ptr(g_host), _ptr(g_dev), _ptr(e), W, d, ctypes.byref(c),
+                                   _ptr(scale), _ptr(codes), _ptr(sum_out), _ptr(out),
+                                   _ptr(out_host), _ptr(scale_host), _ptr(ws), _stream(stream)),
+           "gq_step_fused_host")
+
+
+def _shapes(rows, cols):
+    r = (ctypes.c_int * len(rows))(*[int(x) for x in rows])
+    c = (ctypes.c_int * len(cols))(*[int(x) for x in cols])
+    return r, c
+
+
+def gq_logq_quantize(x, rows, cols, cfg: GQConfig, maxabs, codes, ws, stream=None):
+    W, n = _wd(x)
+    if len(rows) != len(cols) or sum(int(a) * int(b) for a, b in zip(rows, cols)) != n:
+        raise ValueError("rows/cols do not add up to the factor buffer")
+    _need(x, torch.float32, (W, n), "x")
+    _need(maxabs, torch.float32, (W, len(rows)), "maxabs")
+    _need(codes, torch.int8, (W, n), "codes")
+    r, cc = _shapes(rows, cols)
+    c = cfg.c()
+    _check(_lib.gq_logq_quantize(_ptr(x), W, len(rows), r, cc, ctypes.byref(c), _ptr(maxabs),
+                                 _ptr(codes), _ptr(ws), _stream(stream)), "gq_logq_quantize")
+
+
+def gq_logq_decode_sum(codes, maxabs, rows, cols, cfg: GQConfig, out, stream=None):
+    W, n = _wd(codes)
+    _need(codes, torch.int8, (W, n), "codes")
+    _need(maxabs, torch.float32, (W, len(rows)), "maxabs")
+    _need(out, torch.float32, (n,), "out")
+    r, cc = _shapes(rows, cols)
+    c = cfg.c()
+    _check(_lib.gq_logq_decode_sum(_ptr(codes), _ptr(maxabs), W, len(rows), r, cc,
+                                   ctypes.byref(c), _ptr(out), _stream(stream)),
+           "gq_logq_decode_sum")
+
+
+# ------------------------------------------------------------------ buffers
+class StepBuffers:
+    """Device buffers of one step for W workers and d coordinates."""
+
+    def __init__(self, cfg: GQConfig, W: int, d: int, device="cuda", codes=True, ef=None):
+        self.cfg, self.W, self.d = cfg, W, d
+        ef = cfg.ef if ef is None else ef
+        self.scale = torch.zeros(1, dtype=torch.float32, device=device)
+        self.norms = torch.zeros(W, dtype=torch.float64, device=device)
+        self.codes = (torch.empty((W, gq_packed_row_bytes(cfg, d)), dtype=torch.uint8,
+                                  device=device) if codes else None)
+        self.sum = torch.empty(d, dtype=cfg.wire_dtype, device=device)
+        self.out = torch.empty(d, dtype=torch.float32, device=device)
+        self.e = torch.zeros((W, d), dtype=torch.float32, device=device) if ef else None
+        nbytes = gq_workspace_bytes(cfg, W, d)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        gq_workspace_init(self.ws)

@@ -1,0 +1,463 @@
+// gq_api.cu -- host side of the libgq C ABI: argument checks, launch shapes,
+// and the composition of the kernels into the calls declared in gq_api.h.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "gq_api.h"
+#include "gq_internal.h"
+
+using namespace gq;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// Resident 256-thread blocks per SM the streaming kernels are sized for.
+constexpr int kBlocksPerSm = 8;
+
+int max_code(const gq_config& c) { return c.levels == GQ_UNIFORM ? c.s : c.L; }
+
+// Largest value one worker adds to the sum (in the sum's units).
+long long max_value(const gq_config& c) {
+    return c.levels == GQ_UNIFORM ? (long long)c.s : (1LL << (c.L - 1));
+}
+
+int check_levels(const gq_config* c) {
+    if (!c) return GQ_ERR_ARG;
+    if (c->levels == GQ_UNIFORM) {
+        if (c->s < 1 || c->s > 32767) return GQ_ERR_ARG;
+    } else if (c->levels == GQ_EXP) {
+        if (c->L < 1 || c->L > 15) return GQ_ERR_ARG;
+    } else {
+        return GQ_ERR_ARG;
+    }
+    return GQ_OK;
+}
+
+int check_bits(const gq_config* c) {
+    if (c->bits != 4 && c->bits != 5 && c->bits != 8 && c->bits != 16) return GQ_ERR_ARG;
+    // codes -max..max need 2*max+1 distinct two's-complement values
+    const long long need = 2LL * max_code(*c) + 1;
+    if (need > (1LL << c->bits)) return GQ_ERR_ARG;
+    return GQ_OK;
+}
+
+int check_wire(const gq_config* c, int W) {
+    if (c->wire != GQ_WIRE_INT8 && c->wire != GQ_WIRE_INT16) return GQ_ERR_ARG;
+    const long long lim = c->wire == GQ_WIRE_INT8 ? 127 : 32767;
+    if ((long long)W * max_value(*c) > lim) return GQ_ERR_OVERFLOW;
+    return GQ_OK;
+}
+
+int check_scale_kind(const gq_config* c) {
+    return (c->scale_kind == GQ_SCALE_L2 || c->scale_kind == GQ_SCALE_MAXABS) ? GQ_OK : GQ_ERR_ARG;
+}
+
+int check_sizes(int W, long long d) {
+    if (W < 1 || d < 0) return GQ_ERR_ARG;
+    // codes rows, offsets and Philox counters are 64-bit; keep W*d addressable
+    if (d > (1LL << 40) || (long long)W * d > (1LL << 42)) return GQ_ERR_ARG;
+    return GQ_OK;
+}
+
+int norm_blocks_per_worker(int W, long long d) {
+    const long long want = ((long long)sm_count() * kBlocksPerSm + W - 1) / W;
+    const long long useful = (d + (long long)kThreads * 16 - 1) / ((long long)kThreads * 16);
+    long long nb = want < useful ? want : useful;
+    if (nb < 1) nb = 1;
+    if (nb > kMaxNormBlocks) nb = kMaxNormBlocks;
+    return (int)nb;
+}
+
+int stream_grid(long long d) {
+    const long long blocks128 = (d + 127) / 128;                 // one warp each
+    const long long need = (blocks128 + (kThreads / 32) - 1) / (kThreads / 32);
+    const long long cap = (long long)sm_count() * kBlocksPerSm;
+    long long g = need < cap ? need : cap;
+    return g < 1 ? 1 : (int)g;
+}
+
+void round_keys(unsigned long long seed, uint32_t tag, RoundKeys& rk) {
+    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32) ^ tag;
+    for (int r = 0; r < 10; ++r) {
+        rk.k[2 * r] = k0;
+        rk.k[2 * r + 1] = k1;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+}
+
+long long row_bytes_of(int bits, long long d) { return ((d + 127) / 128) * 16LL * bits; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? GQ_OK : GQ_ERR_CUDA; }
+
+WsHeader* header_of(void* ws) { return reinterpret_cast<WsHeader*>(ws); }
+unsigned long long* partials_of(void* ws) {
+    return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(ws) + kWorkspaceHeader);
+}
+
+void fill_quant_args(QuantArgs& a, const gq_config* cfg, int W, long long d) {
+    std::memset(&a, 0, sizeof(a));
+    round_keys(cfg->seed, 0u, a.rk);
+    a.d = d;
+    a.W = W;
+    a.wire = cfg->wire;
+    a.step = cfg->step;
+    a.L = cfg->L;
+    a.smax = (float)cfg->s;
+    a.finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, -(cfg->L - 1)) : 1.0f;
+    a.inv_finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, cfg->L - 1) : 1.0f;
+    a.w_pow2 = is_pow2(W) ? 1 : 0;
+    a.inv_w = a.w_pow2 ? 1.0f / (float)W : 0.0f;
+}
+
+}  // namespace
+
+extern "C" {
+
+GQ_API int gq_version(void) { return kVersion; }
+
+GQ_API const char* gq_status_string(int status) {
+    switch (status) {
+        case GQ_OK: return "ok";
+        case GQ_ERR_ARG: return "invalid argument";
+        case GQ_ERR_OVERFLOW: return "W * max code value overflows the sum type";
+        case GQ_ERR_ALIGN: return "buffer not 16-byte aligned";
+        case GQ_ERR_CUDA: return "CUDA error";
+        case GQ_ERR_NONFINITE: return "non-finite scale (NaN or Inf in the input)";
+        default: return "unknown status";
+    }
+}
+
+GQ_API int gq_validate(const gq_config* cfg, int W, long long d) {
+    int rc = check_levels(cfg);
+    if (rc) return rc;
+    if ((rc = check_sizes(W, d))) return rc;
+    if ((rc = check_bits(cfg))) return rc;
+    if ((rc = check_scale_kind(cfg))) return rc;
+    if (cfg->ef != 0 && cfg->ef != 1) return GQ_ERR_ARG;
+    return check_wire(cfg, W);
+}
+
+GQ_API int gq_packed_row_bytes(const gq_config* cfg, long long d, long long* bytes) {
+    if (!cfg || !bytes || d < 0) return GQ_ERR_ARG;
+    if (cfg->bits != 4 && cfg->bits != 5 && cfg->bits != 8 && cfg->bits != 16) return GQ_ERR_ARG;
+    *bytes = row_bytes_of(cfg->bits, d);
+    return GQ_OK;
+}
+
+GQ_API int gq_workspace_bytes(const gq_config* cfg, int W, long long d, size_t* bytes) {
+    (void)cfg;
+    if (!bytes || W < 1 || d < 0) return GQ_ERR_ARG;
+    *bytes = (size_t)kWorkspaceHeader + (size_t)W * kMaxNormBlocks * sizeof(unsigned long long);
+    return GQ_OK;
+}
+
+GQ_API int gq_workspace_init(void* ws_dev, size_t bytes, cudaStream_t stream) {
+    if (!ws_dev || bytes < (size_t)kWorkspaceHeader) return GQ_ERR_ARG;
+    if (!aligned16(ws_dev)) return GQ_ERR_ALIGN;
+    return cuda_status(cudaMemsetAsync(ws_dev, 0, bytes, stream));
+}
+
+GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream) {
+    if (!ws_dev) return GQ_ERR_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GQ_ERR_CUDA;
+    unsigned int flags = 0;
+    if (cudaMemcpy(&flags, &header_of(ws_dev)->flags, sizeof(flags), cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+        return GQ_ERR_CUDA;
+    if (flags == 0) return GQ_OK;
+    if (cudaMemset(&header_of(ws_dev)->flags, 0, sizeof(flags)) != cudaSuccess) return GQ_ERR_CUDA;
+    return GQ_ERR_NONFINITE;
+}
+
+GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long long d,
+                          const gq_config* cfg, float* scale_dev, double* norms_dev, void* ws_dev,
+                          cudaStream_t stream) {
+    if (!cfg || !g_dev || !scale_dev || !ws_dev) return GQ_ERR_ARG;
+    int rc = check_sizes(W, d);
+    if (rc) return rc;
+    if ((rc = check_scale_kind(cfg))) return rc;
+    if (cfg->ef && !e_dev) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || (e_dev && !aligned16(e_dev)) || !aligned16(ws_dev) ||
+        !aligned4(scale_dev) || (norms_dev && !aligned8(norms_dev)))
+        return GQ_ERR_ALIGN;
+    NormArgs a;
+    a.g = g_dev;
+    a.e = cfg->ef ? e_dev : nullptr;
+    a.d = d;
+    a.W = W;
+    a.nb = norm_blocks_per_worker(W, d);
+    a.kind = cfg->scale_kind;
+    a.scale = scale_dev;
+    a.norms = norms_dev;
+    a.partials = partials_of(ws_dev);
+    a.hdr = header_of(ws_dev);
+    return cuda_status(launch_norm(a, (d % 4) == 0, stream));
+}
+
+static int quant_common(const float* g_dev, float* e_dev, int W, long long d, const gq_config* cfg,
+                        const float* scale_dev, void* codes_dev, void* sum_dev, float* out_dev,
+                        void* ws_dev, bool allow_ef, cudaStream_t stream) {
+    (void)ws_dev;
+    int rc = gq_validate(cfg, W, d);
+    if (rc) return rc;
+    if (!g_dev || !scale_dev) return GQ_ERR_ARG;
+    const bool ef = allow_ef && cfg->ef;
+    if (ef && !e_dev) return GQ_ERR_ARG;
+    if (!codes_dev && !sum_dev && !out_dev && !ef) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || (ef && !aligned16(e_dev)) || !aligned4(scale_dev) ||
+        (codes_dev && !aligned16(codes_dev)) || (sum_dev && !aligned16(sum_dev)) ||
+        (out_dev && !aligned16(out_dev)))
+        return GQ_ERR_ALIGN;
+    if (d == 0) return GQ_OK;
+    QuantArgs a;
+    fill_quant_args(a, cfg, W, d);
+    a.g = g_dev;
+    a.e = ef ? e_dev : nullptr;
+    a.scale = scale_dev;
+    a.codes = reinterpret_cast<unsigned char*>(codes_dev);
+    a.row_bytes = row_bytes_of(cfg->bits, d);
+    a.update_e = ef ? 1 : 0;
+    a.sum = sum_dev;
+    a.out = out_dev;
+    const int bits = codes_dev ? cfg->bits : 0;
+    return cuda_status(
+        launch_quant(a, cfg->levels, bits, ef, (d % 4) == 0, stream_grid(d), stream));
+}
+
+GQ_API int gq_quantize_pack(const float* g_dev, const float* e_dev, int W, long long d,
+                            const gq_config* cfg, const float* scale_dev, void* codes_dev,
+                            void* ws_dev, cudaStream_t stream) {
+    if (!codes_dev) return GQ_ERR_ARG;
+    // v = g + e is read but e is not updated here: the update belongs to step 5
+    gq_config c;
+    if (!cfg) return GQ_ERR_ARG;
+    c = *cfg;
+    if (c.ef && !e_dev) return GQ_ERR_ARG;
+    if (c.ef && !aligned16(e_dev)) return GQ_ERR_ALIGN;
+    int rc = gq_validate(&c, W, d);
+    if (rc) return rc;
+    if (!g_dev || !scale_dev) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || !aligned4(scale_dev) || !aligned16(codes_dev)) return GQ_ERR_ALIGN;
+    if (d == 0) return GQ_OK;
+    (void)ws_dev;
+    QuantArgs a;
+    fill_quant_args(a, &c, W, d);
+    a.g = g_dev;
+    a.e = c.ef ? const_cast<float*>(e_dev) : nullptr;  // read only: update_e = 0
+    a.update_e = 0;
+    a.scale = scale_dev;
+    a.codes = reinterpret_cast<unsigned char*>(codes_dev);
+    a.row_bytes = row_bytes_of(c.bits, d);
+    return cuda_status(
+        launch_quant(a, c.levels, c.bits, c.ef != 0, (d % 4) == 0, stream_grid(d), stream));
+}
+
+GQ_API int gq_aggregate(const void* codes_dev, int W, long long d, const gq_config* cfg,
+                        void* sum_dev, void* ws_dev, cudaStream_t stream) {
+    (void)ws_dev;
+    int rc = gq_validate(cfg, W, d);
+    if (rc) return rc;
+    if (!codes_dev || !sum_dev) return GQ_ERR_ARG;
+    if (!aligned16(codes_dev) || !aligned16(sum_dev)) return GQ_ERR_ALIGN;
+    if (d == 0) return GQ_OK;
+    AggArgs a;
+    a.codes = reinterpret_cast<const unsigned char*>(codes_dev);
+    a.row_bytes = row_bytes_of(cfg->bits, d);
+    a.sum = sum_dev;
+    a.d = d;
+    a.W = W;
+    a.wire = cfg->wire;
+    return cuda_status(launch_aggregate(a, cfg->levels, cfg->bits, stream_grid(d), stream));
+}
+
+GQ_API int gq_dequantize_ef(const void* sum_dev, const void* codes_dev, const float* g_dev,
+                            float* e_dev, int W, long long d, const gq_config* cfg,
+                            const float* scale_dev, float* out_dev, void* ws_dev,
+                            cudaStream_t stream) {
+    (void)ws_dev;
+    int rc = gq_validate(cfg, W, d);
+    if (rc) return rc;
+    if (!scale_dev) return GQ_ERR_ARG;
+    const bool dec = sum_dev != nullptr;
+    const bool ef = cfg->ef && e_dev;
+    if (dec && !out_dev) return GQ_ERR_ARG;
+    if (!dec && !ef) return GQ_ERR_ARG;
+    if (ef && (!codes_dev || !g_dev)) return GQ_ERR_ARG;
+    if (!aligned4(scale_dev) || (dec && (!aligned16(sum_dev) || !aligned16(out_dev))) ||
+        (ef && (!aligned16(codes_dev) || !aligned16(g_dev) || !aligned16(e_dev))))
+        return GQ_ERR_ALIGN;
+    if (d == 0) return GQ_OK;
+    DequantArgs a;
+    a.sum = dec ? sum_dev : nullptr;
+    a.codes = reinterpret_cast<const unsigned char*>(codes_dev);
+    a.row_bytes = row_bytes_of(cfg->bits, d);
+    a.g = g_dev;
+    a.e = ef ? e_dev : nullptr;
+    a.scale = scale_dev;
+    a.out = out_dev;
+    a.d = d;
+    a.W = W;
+    a.wire = cfg->wire;
+    a.smax = (float)cfg->s;
+    a.finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, -(cfg->L - 1)) : 1.0f;
+    a.w_pow2 = is_pow2(W) ? 1 : 0;
+    a.inv_w = a.w_pow2 ? 1.0f / (float)W : 0.0f;
+    return cuda_status(
+        launch_dequant(a, cfg->levels, cfg->bits, (d % 4) == 0, stream_grid(d), stream));
+}
+
+GQ_API int gq_quantize_aggregate(const float* g_dev, float* e_dev, int W, long long d,
+                                 const gq_config* cfg, const float* scale_dev, void* codes_dev,
+                                 void* sum_dev, float* out_dev, void* ws_dev, cudaStream_t stream) {
+    return quant_common(g_dev, e_dev, W, d, cfg, scale_dev, codes_dev, sum_dev, out_dev, ws_dev,
+                        true, stream);
+}
+
+GQ_API int gq_step_fused(const float* g_dev, float* e_dev, int W, long long d,
+                         const gq_config* cfg, float* scale_dev, double* norms_dev,
+                         void* codes_dev, void* sum_dev, float* out_dev, void* ws_dev,
+                         cudaStream_t stream) {
+    int rc = gq_validate(cfg, W, d);
+    if (rc) return rc;
+    if (cfg->ef && !e_dev) return GQ_ERR_ARG;
+    if (!codes_dev && !sum_dev && !out_dev && !cfg->ef) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || (cfg->ef && !aligned16(e_dev)) ||
+        (codes_dev && !aligned16(codes_dev)) || (sum_dev && !aligned16(sum_dev)) ||
+        (out_dev && !aligned16(out_dev)))
+        return GQ_ERR_ALIGN;
+    rc = gq_global_norm(g_dev, cfg->ef ? e_dev : nullptr, W, d, cfg, scale_dev, norms_dev, ws_dev,
+                        stream);
+    if (rc) return rc;
+    return gq_quantize_aggregate(g_dev, e_dev, W, d, cfg, scale_dev, codes_dev, sum_dev, out_dev,
+                                 ws_dev, stream);
+}
+
+GQ_API int gq_step_fused_host(const float* g_host, float* g_dev, float* e_dev, int W, long long d,
+                              const gq_config* cfg, float* scale_dev, void* codes_dev,
+                              void* sum_dev, float* out_dev, float* out_host, float* scale_host,
+                              void* ws_dev, cudaStream_t stream) {
+    int rc = gq_validate(cfg, W, d);
+    if (rc) return rc;
+    if (!g_host || !g_dev || !out_dev || !out_host) return GQ_ERR_ARG;
+    const size_t gbytes = (size_t)W * (size_t)d * sizeof(float);
+    if (cudaMemcpyAsync(g_dev, g_host, gbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return GQ_ERR_CUDA;
+    rc = gq_step_fused(g_dev, e_dev, W, d, cfg, scale_dev, nullptr, codes_dev, sum_dev, out_dev,
+                       ws_dev, stream);
+    if (rc) return rc;
+    if (cudaMemcpyAsync(out_host, out_dev, (size_t)d * sizeof(float), cudaMemcpyDeviceToHost,
+                        stream) != cudaSuccess)
+        return GQ_ERR_CUDA;
+    if (scale_host && cudaMemcpyAsync(scale_host, scale_dev, sizeof(float), cudaMemcpyDeviceToHost,
+                                      stream) != cudaSuccess)
+        return GQ_ERR_CUDA;
+    return GQ_OK;
+}
+
+static int logq_offsets(int nmats, const int* rows, const int* cols, long long* total) {
+    if (nmats < 1 || nmats > 4096 || !rows || !cols) return GQ_ERR_ARG;
+    long long t = 0;
+    for (int m = 0; m < nmats; ++m) {
+        if (rows[m] < 0 || cols[m] < 0) return GQ_ERR_ARG;
+        t += (long long)rows[m] * cols[m];
+    }
+    *total = t;
+    return GQ_OK;
+}
+
+static void logq_group(LogqArgs& a, int m0, int count, const int* rows, const int* cols) {
+    a.m0 = m0;
+    a.count = count;
+    long long off = 0;
+    for (int m = 0; m < m0; ++m) off += (long long)rows[m] * cols[m];
+    a.off[0] = off;
+    for (int i = 0; i < count; ++i) a.off[i + 1] = a.off[i] + (long long)rows[m0 + i] * cols[m0 + i];
+}
+
+GQ_API int gq_logq_quantize(const float* x_dev, int W, int nmats, const int* rows_host,
+                            const int* cols_host, const gq_config* cfg, float* maxabs_dev,
+                            signed char* codes_dev, void* ws_dev, cudaStream_t stream) {
+    if (!cfg || cfg->levels != GQ_LOG || !(cfg->alpha > 0.f) || !(cfg->alpha <= 3.0e38f))
+        return GQ_ERR_ARG;
+    if (!x_dev || !maxabs_dev || !codes_dev || !ws_dev || W < 1) return GQ_ERR_ARG;
+    long long total = 0;
+    int rc = logq_offsets(nmats, rows_host, cols_host, &total);
+    if (rc) return rc;
+    if (!aligned16(x_dev) || !aligned4(maxabs_dev) || !aligned16(ws_dev)) return GQ_ERR_ALIGN;
+    LogqArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.x = x_dev;
+    a.codes = codes_dev;
+    a.maxabs = maxabs_dev;
+    a.total = total;
+    a.W = W;
+    a.nmats = nmats;
+    a.step = cfg->step;
+    a.seed_lo = (uint32_t)cfg->seed;
+    a.seed_hi = (uint32_t)(cfg->seed >> 32);
+    a.alpha = cfg->alpha;
+    a.hdr = header_of(ws_dev);
+    for (int m0 = 0; m0 < nmats; m0 += kLogqGroup) {
+        const int count = nmats - m0 < kLogqGroup ? nmats - m0 : kLogqGroup;
+        logq_group(a, m0, count, rows_host, cols_host);
+        if ((rc = cuda_status(launch_logq_quantize(a, stream)))) return rc;
+    }
+    return GQ_OK;
+}
+
+GQ_API int gq_logq_decode_sum(const signed char* codes_dev, const float* maxabs_dev, int W,
+                              int nmats, const int* rows_host, const int* cols_host,
+                              const gq_config* cfg, float* out_dev, cudaStream_t stream) {
+    if (!cfg || cfg->levels != GQ_LOG || !(cfg->alpha > 0.f) || !(cfg->alpha <= 3.0e38f))
+        return GQ_ERR_ARG;
+    if (!codes_dev || !maxabs_dev || !out_dev || W < 1) return GQ_ERR_ARG;
+    long long total = 0;
+    int rc = logq_offsets(nmats, rows_host, cols_host, &total);
+    if (rc) return rc;
+    if (!aligned4(maxabs_dev) || !aligned4(out_dev)) return GQ_ERR_ALIGN;
+    LogqArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.ccodes = codes_dev;
+    a.cmaxabs = maxabs_dev;
+    a.out = out_dev;
+    a.total = total;
+    a.W = W;
+    a.nmats = nmats;
+    a.alpha = cfg->alpha;
+    for (int m0 = 0; m0 < nmats; m0 += kLogqGroup) {
+        const int count = nmats - m0 < kLogqGroup ? nmats - m0 : kLogqGroup;
+        logq_group(a, m0, count, rows_host, cols_host);
+        if ((rc = cuda_status(launch_logq_decode(a, stream)))) return rc;
+    }
+    return GQ_OK;
+}
+
+}  // extern "C"

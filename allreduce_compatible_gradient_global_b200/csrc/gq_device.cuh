@@ -1,0 +1,217 @@
+// gq_device.cuh -- device building blocks of libgq (sm_100a).
+//
+// Philox-4x32-10 in registers, the stochastic-rounding quantizers, and the
+// warp-level packing of codes at wire width.  Every floating-point step that
+// decides a code or an output uses an explicit _rn/_rd intrinsic, so the
+// compiler can neither contract nor reorder it.
+#pragma once
+
+#include <cstdint>
+
+namespace gq {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// ---------------------------------------------------------------------------
+// Philox-4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC'11): ten rounds of two 32x32->64 multiplies whose high
+// halves are XORed with the other two counter words and the round key.  The
+// round keys (key + r * Weyl constants) are the same for every thread, so the
+// host computes them once and passes them in the kernel parameters.
+// ---------------------------------------------------------------------------
+struct RoundKeys {
+    uint32_t k[20];  // k[2r], k[2r+1]: key words of round r
+};
+
+__device__ __forceinline__ uint4 philox10(uint4 c, const RoundKeys& rk) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const unsigned long long p0 = (unsigned long long)c.x * 0xD2511F53ull;
+        const unsigned long long p1 = (unsigned long long)c.z * 0xCD9E8D57ull;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        c = make_uint4(hi1 ^ c.y ^ rk.k[2 * r], lo1, hi0 ^ c.w ^ rk.k[2 * r + 1], lo0);
+    }
+    return c;
+}
+
+// Counter of the block that serves coordinates 4q..4q+3 of `worker` at `step`.
+__device__ __forceinline__ uint4 philox_counter(unsigned long long q, uint32_t step,
+                                                uint32_t worker) {
+    return make_uint4((uint32_t)q, step, worker, (uint32_t)(q >> 32));
+}
+
+// ---------------------------------------------------------------------------
+// Stochastic rounding.  A magnitude y >= 0 becomes floor(y + u) with
+// u = f * 2^-23, f the low 23 bits of a Philox word: that is floor(y) + 1
+// exactly when frac(y) + u >= 1, an event of probability frac(y), so the
+// rounding is unbiased.
+//
+// floor(y + u) is computed without a conversion instruction: U = 1 + u is
+// built from bits (exact), t1 = fl_down(y + U) has the same floor as y + U
+// (that floor is an integer <= 2^24, hence a float, and rounding down cannot
+// cross it), and fl_down(t1 + 2^23) is 2^23 + floor(t1) exactly because floats
+// in [2^23, 2^24) are the integers.  So the integer is the bit pattern minus
+// that of 2^23, minus 1 for the U offset.  Valid for 0 <= y < 2^23 - 2.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float unit_plus_u(uint32_t word) {
+    return __uint_as_float(0x3F800000u | (word & 0x007FFFFFu));
+}
+
+__device__ __forceinline__ int floor_y_plus_u(float y, float U) {
+    const float t1 = __fadd_rd(y, U);
+    const float t2 = __fadd_rd(t1, 8388608.0f);
+    return __float_as_int(t2) - 0x4B000001;
+}
+
+// Apply the sign of v (its sign bit, so -0.0 and +0.0 both give +k / -k = 0).
+__device__ __forceinline__ int with_sign_of(int k, float v) {
+    const int sgn = __float_as_int(v) >> 31;  // 0 or -1
+    return (k ^ sgn) - sgn;
+}
+
+// Uniform levels {0, 1/s, ..., 1}: a = fl(s/S), r = min(fl(|v| a), s).
+// fminf also maps a NaN product to s, so no input can escape the range.
+__device__ __forceinline__ int quant_uniform(float v, float a, float smax, uint32_t word) {
+    const float r = fminf(__fmul_rn(fabsf(v), a), smax);
+    return with_sign_of(floor_y_plus_u(r, unit_plus_u(word)), v);
+}
+
+// Exponential levels {0, 2^-(L-1), ..., 1/2, 1}: a = fl(1/S), r = min(fl(|v| a), 1).
+// For r >= 2^-(L-1), r = (1 + m 2^-23) 2^E with m the mantissa field: the
+// bracket is [2^E, 2^(E+1)], the lower level has index L + E, and the
+// round-up probability (r - 2^E)/2^E equals m 2^-23, so the decision
+// frac + u >= 1 is the integer test m + f >= 2^23.  Below 2^-(L-1) the bracket
+// is [0, 2^-(L-1)] and p = r 2^(L-1) (exact); p + u >= 1 iff fl_down(p + U) >= 2.
+__device__ __forceinline__ int quant_exp(float v, float a, int L, float finest, float inv_finest,
+                                         uint32_t word) {
+    const float r = fminf(__fmul_rn(fabsf(v), a), 1.0f);
+    const uint32_t f = word & 0x007FFFFFu;
+    int idx;
+    if (r >= finest) {
+        const uint32_t rb = __float_as_uint(r);
+        const int E = (int)(rb >> 23) - 127;
+        idx = L + E + (int)(((rb & 0x007FFFFFu) + f) >> 23);
+    } else {
+        const float p = __fmul_rn(r, inv_finest);
+        idx = __fadd_rd(p, __uint_as_float(0x3F800000u | f)) >= 2.0f ? 1 : 0;
+    }
+    return with_sign_of(idx, v);
+}
+
+// Value a code adds to the sum: the code itself (uniform levels) or
+// sign * 2^(idx-1) units of the finest level (exponential levels).
+template <int LEVELS>
+__device__ __forceinline__ int code_value(int code) {
+    if (LEVELS == 0) return code;
+    const int sgn = code >> 31;
+    const int idx = (code ^ sgn) - sgn;
+    const int mag = (1 << idx) >> 1;
+    return (mag ^ sgn) - sgn;
+}
+
+// Exact int -> float for |x| < 2^22: 1.5 * 2^23 + x lies in [2^23, 2^24), where
+// floats are the integers, so building it from bits and subtracting is exact.
+__device__ __forceinline__ float small_int_to_float(int x) {
+    return __fsub_rn(__int_as_float(0x4B400000 + x), 12582912.0f);
+}
+
+// ---------------------------------------------------------------------------
+// Warp packing.  A warp covers one 128-coordinate block of one worker's row;
+// lane l holds codes 4l..4l+3.  Wire layout: bits 4/5 -- little-endian
+// bitstream (code j at stream bits [b j, b j + b)); 8 -- int8; 16 -- int16.
+// One block is 16 * BITS bytes, so every warp store is aligned and in range.
+// ---------------------------------------------------------------------------
+template <int BITS>
+struct Packer {
+    int src0;  // bits 5: first lane whose 20-bit chunk reaches this lane's word
+    int off;   // bits 5: bit offset of that chunk inside the word
+    __device__ __forceinline__ void init(int lane) {
+        if (BITS == 5) {
+            src0 = min((8 * lane) / 5, 30);
+            off = lane < 20 ? 32 * lane - 20 * src0 : 0;  // lanes >= 20 store nothing
+        }
+    }
+    // Pack and store the 4 codes of this lane; dst is the block's first byte.
+    __device__ __forceinline__ void store(int lane, int c0, int c1, int c2, int c3,
+                                          unsigned char* dst) const {
+        if (BITS == 5) {
+            const uint32_t x = (uint32_t)(c0 & 31) | ((uint32_t)(c1 & 31) << 5) |
+                               ((uint32_t)(c2 & 31) << 10) | ((uint32_t)(c3 & 31) << 15);
+            const uint32_t x0 = __shfl_sync(kFull, x, src0);
+            const uint32_t x1 = __shfl_sync(kFull, x, src0 + 1);
+            const uint32_t x2 = __shfl_sync(kFull, x, min(src0 + 2, 31));
+            const unsigned long long y = (unsigned long long)x0 |
+                                         ((unsigned long long)x1 << 20) |
+                                         ((unsigned long long)x2 << 40);
+            const uint32_t word = (uint32_t)(y >> off);
+            if (lane < 20) reinterpret_cast<uint32_t*>(dst)[lane] = word;
+        } else if (BITS == 4) {
+            const uint32_t x = (uint32_t)(c0 & 15) | ((uint32_t)(c1 & 15) << 4) |
+                               ((uint32_t)(c2 & 15) << 8) | ((uint32_t)(c3 & 15) << 12);
+            const uint32_t xa = __shfl_sync(kFull, x, (2 * lane) & 31);
+            const uint32_t xb = __shfl_sync(kFull, x, (2 * lane + 1) & 31);
+            if (lane < 16) reinterpret_cast<uint32_t*>(dst)[lane] = xa | (xb << 16);
+        } else if (BITS == 8) {
+            const uint32_t x = (uint32_t)(c0 & 255) | ((uint32_t)(c1 & 255) << 8) |
+                               ((uint32_t)(c2 & 255) << 16) | ((uint32_t)(c3 & 255) << 24);
+            reinterpret_cast<uint32_t*>(dst)[lane] = x;
+        } else if (BITS == 16) {
+            uint2 x;
+            x.x = (uint32_t)(c0 & 0xFFFF) | ((uint32_t)c1 << 16);
+            x.y = (uint32_t)(c2 & 0xFFFF) | ((uint32_t)c3 << 16);
+            reinterpret_cast<uint2*>(dst)[lane] = x;
+        }
+    }
+};
+
+// Unpacking: the inverse, reading one block of one worker's row.
+template <int BITS>
+struct Unpacker {
+    int w0;   // bits 5: first word holding this lane's chunk
+    int off;  // bits 5: bit offset of the chunk in that word
+    __device__ __forceinline__ void init(int lane) {
+        if (BITS == 5) {
+            w0 = (20 * lane) >> 5;
+            off = (20 * lane) & 31;
+        }
+    }
+    __device__ __forceinline__ static int sext(uint32_t field, int bits) {
+        return ((int)(field << (32 - bits))) >> (32 - bits);
+    }
+    __device__ __forceinline__ void load(int lane, const unsigned char* src, int& c0, int& c1,
+                                         int& c2, int& c3) const {
+        if (BITS == 5) {
+            const uint32_t mine = lane < 20 ? reinterpret_cast<const uint32_t*>(src)[lane] : 0u;
+            const uint32_t a = __shfl_sync(kFull, mine, w0);
+            const uint32_t b = __shfl_sync(kFull, mine, min(w0 + 1, 31));
+            const uint32_t x = __funnelshift_r(a, b, off);
+            c0 = sext(x, 5);
+            c1 = sext(x >> 5, 5);
+            c2 = sext(x >> 10, 5);
+            c3 = sext(x >> 15, 5);
+        } else if (BITS == 4) {
+            const uint32_t mine = lane < 16 ? reinterpret_cast<const uint32_t*>(src)[lane] : 0u;
+            const uint32_t wv = __shfl_sync(kFull, mine, lane >> 1);
+            const uint32_t x = (lane & 1) ? (wv >> 16) : wv;
+            c0 = sext(x, 4);
+            c1 = sext(x >> 4, 4);
+            c2 = sext(x >> 8, 4);
+            c3 = sext(x >> 12, 4);
+        } else if (BITS == 8) {
+            const uint32_t x = reinterpret_cast<const uint32_t*>(src)[lane];
+            c0 = sext(x, 8);
+            c1 = sext(x >> 8, 8);
+            c2 = sext(x >> 16, 8);
+            c3 = sext(x >> 24, 8);
+        } else {
+            const uint2 x = reinterpret_cast<const uint2*>(src)[lane];
+            c0 = sext(x.x, 16);
+            c1 = sext(x.x >> 16, 16);
+            c2 = sext(x.y, 16);
+            c3 = sext(x.y >> 16, 16);
+        }
+    }
+};
+
+}  // namespace gq

@@ -1,0 +1,118 @@
+// gq_internal.h -- kernel argument blocks and launchers shared by the host
+// entry points (gq_api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "gq_device.cuh"
+
+namespace gq {
+
+constexpr int kThreads = 256;          // threads per block of every streaming kernel
+constexpr int kMaxNormBlocks = 2048;   // per-worker partial slots in the workspace
+constexpr int kWorkspaceHeader = 256;  // flag word, ticket counter, padding
+
+// Workspace header words.
+struct WsHeader {
+    unsigned int flags;    // bit 0: non-finite scale; bit 1: non-finite LQ max
+    unsigned int counter;  // last-block ticket of the norm kernel (0 between calls)
+};
+
+constexpr unsigned kFlagNonfiniteScale = 1u;
+constexpr unsigned kFlagNonfiniteLogqMax = 2u;
+
+struct NormArgs {
+    const float* g;
+    const float* e;
+    long long d;
+    int W;
+    int nb;  // blocks per worker (gridDim.x)
+    int kind;
+    float* scale;
+    double* norms;
+    unsigned long long* partials;  // [W][nb]
+    WsHeader* hdr;
+};
+
+struct QuantArgs {
+    RoundKeys rk;
+    const float* g;
+    float* e;  // v = g + e is read when error feedback is on
+    int update_e;  // 1: also write e <- v - Q(v) (step 5); 0: read only
+    const float* scale;
+    unsigned char* codes;  // [W][row_bytes] or null
+    long long row_bytes;
+    void* sum;  // [d] int8/int16 or null
+    float* out; // [d] or null
+    long long d;
+    int W;
+    int wire;  // bytes per sum element
+    unsigned int step;
+    int L;
+    float smax;        // (float)s
+    float finest;      // 2^-(L-1)
+    float inv_finest;  // 2^(L-1)
+    float inv_w;       // 1/W when W is a power of two
+    int w_pow2;
+};
+
+struct AggArgs {
+    const unsigned char* codes;
+    long long row_bytes;
+    void* sum;
+    long long d;
+    int W;
+    int wire;
+};
+
+struct DequantArgs {
+    const void* sum;  // null: no output decode
+    const unsigned char* codes;
+    long long row_bytes;
+    const float* g;
+    float* e;  // null: no error feedback
+    const float* scale;
+    float* out;
+    long long d;
+    int W;
+    int wire;
+    float smax;
+    float finest;
+    float inv_w;
+    int w_pow2;
+};
+
+constexpr int kLogqGroup = 128;  // matrices per LQ launch (offsets ride in the parameters)
+
+struct LogqArgs {
+    const float* x;
+    signed char* codes;
+    float* maxabs;
+    const signed char* ccodes;  // decode: input codes
+    const float* cmaxabs;       // decode: input max-abs
+    float* out;                 // decode: output sum
+    long long total;            // elements per worker
+    int W;
+    int nmats;  // total matrices (row stride of maxabs)
+    int m0;     // first matrix of this launch
+    int count;  // matrices in this launch
+    long long off[kLogqGroup + 1];
+    unsigned int step;
+    unsigned int seed_lo, seed_hi;
+    float alpha;
+    WsHeader* hdr;
+};
+
+// Launchers (return the cudaGetLastError() of the launch).
+cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st);
+cudaError_t launch_quant(const QuantArgs& a, int levels, int bits, bool ef, bool vec, int grid,
+                         cudaStream_t st);
+cudaError_t launch_aggregate(const AggArgs& a, int levels, int bits, int grid, cudaStream_t st);
+cudaError_t launch_dequant(const DequantArgs& a, int levels, int bits, bool vec, int grid,
+                           cudaStream_t st);
+cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st);
+cudaError_t launch_logq_decode(const LogqArgs& a, cudaStream_t st);
+
+}  // namespace gq

@@ -1,0 +1,392 @@
+"""Benchmark of the quantize + aggregate path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline] [--no-e2e]
+
+One step = one pass of the whole path over one batch of W synthetic worker
+gradients already resident in HBM: gq_global_norm (read 1) then
+gq_quantize_aggregate (read 2: Philox uniforms, stochastic rounding, packed
+codes at wire width, integer sum over workers, decoded mean).  These two calls
+are exactly what gq_step_fused issues; the benchmark makes them separately so
+that CUDA events bracket the dominant kernel on its own stream.
+
+Metric: fp32 gradient GB/s = 4 * W * d bytes / step time (whole job: summed
+over ranks under torchrun, each rank an independent replica, timed as the max
+over ranks).  Prints one JSON line on rank 0.
+
+--impl reference times the CPU oracle (the plain restatement of the method
+used by the tests) on the host cores, on a bounded sample of the same
+workload, with the same metric.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synthetic  # noqa: E402
+
+METRIC = "quantize+aggregate fp32-gradient GB/s at 1 B200; % of HBM roofline"
+DEFAULT_WORKLOAD = "resnet50_t3_w8"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "quant_kernel_traffic.json")
+KERNEL_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_kernels.cu",
+                  "allreduce_compatible_gradient_global_b200/csrc/gq_device.cuh",
+                  "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h"]
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    ent = rec.get("workloads", {}).get(workload)
+    return None if ent is None else float(ent["dram_bytes_per_launch"])
+
+
+# ----------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            uuid = None
+            try:
+                uuid = torch.cuda.get_device_properties(device_index).uuid
+            except Exception:
+                uuid = None
+            handle = None
+            if uuid is not None:
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    handle = None
+            if handle is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                phys = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() \
+                    else device_index
+                handle = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.handle = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # no NVML: report that instead of clocks
+            self.nvml = None
+            self.error = f"nvml unavailable: {exc}"
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append(mhz)
+                self.reasons |= int(rs)
+            except Exception:
+                pass
+            self._stop.wait(0.002)
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self.nvml is None:
+            return {"error": self.error}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------ runs
+def workload_config(gq, name):
+    wl = synthetic.WORKLOADS[name]
+    cfg = gq.GQConfig(levels=wl["levels"], s=wl.get("s", 15), L=wl.get("L", 8), bits=wl["bits"],
+                      scale_kind=wl["scale"], wire=wl["wire"], ef=wl["ef"], seed=0x5EED, step=0)
+    return wl, cfg
+
+
+def algorithmic_bytes(gq, cfg, W, d):
+    """(pass-1 bytes, pass-2 bytes) per step: what each kernel must move."""
+    wire = 1 if cfg.wire == "int8" else 2
+    p1 = 4 * W * d + (4 * W * d if cfg.ef else 0)
+    p2 = (4 * W * d + W * gq.gq_packed_row_bytes(cfg, d) + wire * d + 4 * d
+          + (8 * W * d if cfg.ef else 0))
+    return p1, p2
+
+
+def run_ours(args, rank, world, local_rank):
+    import allreduce_compatible_gradient_global_b200 as gq
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl, cfg = workload_config(gq, args.workload)
+    W, d = wl["W"], wl["d"]
+    g = synthetic.workload_gradients(args.workload, device=dev)
+    buf = gq.StepBuffers(cfg, W, d, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        cfg.step = i
+        if ev is not None:
+            ev[0].record(stream)
+        gq.gq_global_norm(g, buf.e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        gq.gq_quantize_aggregate(g, buf.e, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws,
+                                 stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    if gq.gq_get_device_status(buf.ws, stream) != gq.GQ_OK:
+        raise RuntimeError("non-finite scale in warm-up")
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(args.warmup + i, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    norm_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    quant_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / K
+    grad_bytes = 4 * W * d
+    value = world * grad_bytes * K / (elapsed_ms * 1e-3) / 1e9
+
+    # roofline of the dominant kernel (pass 2)
+    p1, p2 = algorithmic_bytes(gq, cfg, W, d)
+    q_avg = sum(quant_ms) / K
+    n_avg = sum(norm_ms) / K
+    peak, peak_kind = measured_hbm_peak()
+    achieved = p2 / (q_avg * 1e-3) / 1e9
+    traffic = recorded_traffic(args.workload)
+    roofline = {"bound": "hbm", "kernel": "quant_kernel (gq_quantize_aggregate)",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} (hbm_gbs)",
+                "traffic": traffic, "algorithmic_bytes": p2,
+                "avg_launch_ms": round(q_avg, 5),
+                "norm_kernel": {"achieved": round(p1 / (n_avg * 1e-3) / 1e9, 1),
+                                "frac": round(p1 / (n_avg * 1e-3) / 1e9 / peak, 4),
+                                "algorithmic_bytes": p1, "avg_launch_ms": round(n_avg, 5)},
+                "step": {"achieved": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9, 1),
+                         "frac": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+                         "frac_of_8000": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / 8000, 4)}}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(gq, args, cfg, g, buf, stream, world, dev)
+    result = dict(
+        metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=K,
+        warmup=args.warmup, ms_per_step=round(ms_per_step, 5), higher_is_better=True,
+        scaling="weak", vs_baseline=None, dtype="f32",
+        data="synthetic (seeded per-segment Student-t(3) gradients, ResNet-50-sized)"
+        if args.workload == DEFAULT_WORKLOAD else "synthetic",
+        config={"workload": args.workload, "W": W, "d": d, "levels": cfg.levels, "s": cfg.s,
+                "L": cfg.L, "bits": cfg.bits, "wire": cfg.wire, "scale": cfg.scale_kind,
+                "ef": cfg.ef, "parallelism": f"replicas x{world}",
+                "l2": f"inputs exceed L2: {grad_bytes / 1e6:.1f} MB of gradient per read "
+                      f"vs {L2_BYTES / 1e6:.0f} MB L2"},
+        roofline=roofline, gpu_launches=2 * K, clocks=sampler.summary(), e2e=e2e)
+    del g, buf
+    torch.cuda.empty_cache()
+    return result
+
+
+def run_e2e(gq, args, cfg, g, buf, stream, world, dev):
+    """Same metric through gq_step_fused_host: H2D of the step's gradients from
+    pinned memory, both kernels, D2H of the decoded mean and the scale."""
+    W, d = g.shape
+    g_host = g.cpu().pin_memory()
+    out_host = torch.empty(d, dtype=torch.float32).pin_memory()
+    scale_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    g_dev = torch.empty_like(g)
+    K = args.steps
+    for i in range(min(args.warmup, 3)):
+        cfg.step = i
+        gq.gq_step_fused_host(g_host, g_dev, buf.e, cfg, buf.scale, buf.codes, buf.sum, buf.out,
+                              out_host, scale_host, buf.ws, stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        cfg.step = 1000 + i
+        gq.gq_step_fused_host(g_host, g_dev, buf.e, cfg, buf.scale, buf.codes, buf.sum, buf.out,
+                              out_host, scale_host, buf.ws, stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    val = world * 4 * W * d * K / (ms * 1e-3) / 1e9
+    del g_host, g_dev
+    return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
+            "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4),
+            "api": "gq_step_fused_host"}
+
+
+def cpu_baseline(args, sample_coords=None):
+    """The oracle as it stands (single-threaded C) on a sample of the workload."""
+    import oracle
+    wl = synthetic.WORKLOADS[args.workload]
+    W, d = wl["W"], wl["d"]
+    n = d if sample_coords is None else min(d, sample_coords)
+    g = synthetic.workload_gradients(args.workload, device="cpu", d=n).numpy()
+    kw = dict(levels=0 if wl["levels"] == "uniform" else 1, s=wl.get("s", 15), L=wl.get("L", 8),
+              scale_kind=0 if wl["scale"] == "l2" else 1, bits=wl["bits"], seed=0x5EED)
+    oracle.lib()
+    t = time.perf_counter()
+    oracle.step(g, **kw)
+    dt = time.perf_counter() - t
+    return {"value": round(4 * W * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"one oracle step (scale, codes, pack, sum, decode) on W={W} x "
+                      f"{n} coordinates of the {args.workload} recipe "
+                      f"({'the full workload' if n == d else 'a prefix'}), {dt:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, each step a bounded sample."""
+    import oracle
+    wl = synthetic.WORKLOADS[args.workload]
+    W, d = wl["W"], wl["d"]
+    n = min(d, args.reference_coords)
+    g = synthetic.workload_gradients(args.workload, device="cpu", d=n).numpy()
+    kw = dict(levels=0 if wl["levels"] == "uniform" else 1, s=wl.get("s", 15), L=wl.get("L", 8),
+              scale_kind=0 if wl["scale"] == "l2" else 1, bits=wl["bits"], seed=0x5EED)
+    oracle.lib()
+    for i in range(args.warmup):
+        oracle.step(g, step=i, **kw)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        oracle.step(g, step=args.warmup + i, **kw)
+    dt = time.perf_counter() - t
+    value = 4 * W * n * args.steps / dt / 1e9
+    sample = (f"each step: one oracle step on W={W} x {n} coordinates (a prefix of the "
+              f"{args.workload} recipe, d={d})")
+    return dict(metric=METRIC, value=round(value, 4), unit="GB/s", n_gpus=args.gpus,
+                steps=args.steps, warmup=args.warmup, ms_per_step=round(dt / args.steps * 1e3, 3),
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f32",
+                data="synthetic", impl="reference",
+                config={"workload": args.workload, "W": W, "d": d, "sample_coords": n},
+                cpu_baseline={"value": round(value, 4), "unit": "GB/s", "cores": 1,
+                              "kind": "oracle", "sample": sample},
+                e2e={"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                     "d2h_bytes_per_step": 0})
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--reference-coords", type=int, default=1 << 21)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        result = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            result["cpu_baseline"] = None if (args.no_cpu_baseline or world > 1) \
+                else cpu_baseline(args)
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

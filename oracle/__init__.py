@@ -32,6 +32,8 @@ def lib():
         L.gqo_uniform_bits.restype = u32
         L.gqo_sumsq.argtypes = [P, P, i64]
         L.gqo_sumsq.restype = ctypes.c_double
+        L.gqo_sumsq_from.argtypes = [ctypes.c_double, P, P, i64]
+        L.gqo_sumsq_from.restype = ctypes.c_double
         L.gqo_maxabs.argtypes = [P, P, i64]
         L.gqo_maxabs.restype = f32
         L.gqo_global_scale.argtypes = [P, P, i32, i64, i32, P, P]
@@ -83,6 +85,19 @@ def sumsq(g, e=None):
     g = _f32(g)
     e = _f32(e)
     return lib().gqo_sumsq(_p(g), _p(e), g.size)
+
+
+def sumsq_from(acc, g, e=None):
+    """acc + sum of squares of fl(g+e), continuing one ascending fp64 sum."""
+    g = _f32(g)
+    e = _f32(e)
+    return lib().gqo_sumsq_from(float(acc), _p(g), _p(e), g.size)
+
+
+def maxabs(g, e=None):
+    g = _f32(g)
+    e = _f32(e)
+    return np.float32(lib().gqo_maxabs(_p(g), _p(e), g.size))
 
 
 def global_scale(g, e=None, scale_kind=SCALE_L2):

@@ -85,7 +85,11 @@ static int sign_negative(float v)
  * ---------------------------------------------------------------------- */
 double gqo_sumsq(const float* g, const float* e, int64_t n)
 {
-    double acc = 0.0;
+    return gqo_sumsq_from(0.0, g, e, n);
+}
+
+double gqo_sumsq_from(double acc, const float* g, const float* e, int64_t n)
+{
     for (int64_t i = 0; i < n; ++i) {
         float v = e ? g[i] + e[i] : g[i];
         double dv = (double)v;

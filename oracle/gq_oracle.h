@@ -63,6 +63,10 @@ uint32_t gqo_uniform_bits(uint64_t seed, uint32_t tag, uint32_t step,
  * the caller adds the partials in ascending chunk order. */
 double gqo_sumsq(const float* g, const float* e, int64_t n);
 
+/* The same sum continued from `acc`: acc + v_0^2 + v_1^2 + ... in order, so a
+ * row streamed in chunks gives exactly the one-pass value. */
+double gqo_sumsq_from(double acc, const float* g, const float* e, int64_t n);
+
 /* max |fl(g+e)| over n entries; NaN if any entry is NaN. */
 float gqo_maxabs(const float* g, const float* e, int64_t n);
 

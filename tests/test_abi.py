@@ -1,0 +1,145 @@
+"""The C ABI without a GPU: the library builds, loads, exports every entry point
+that include/gq_api.h declares, and its host-side checks (sizes, overflow
+rule, alignment) answer before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gq_api.h")
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"GQ_API\s+[\w\s\*]+?\b(gq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def gq():
+    from allreduce_compatible_gradient_global_b200 import build as b
+    b.build()
+    import allreduce_compatible_gradient_global_b200 as gq
+    return gq
+
+
+def test_header_declares_the_path():
+    names = declared_entry_points()
+    for required in ("gq_global_norm", "gq_quantize_pack", "gq_aggregate", "gq_dequantize_ef",
+                     "gq_step_fused", "gq_quantize_aggregate", "gq_step_fused_host",
+                     "gq_logq_quantize", "gq_logq_decode_sum", "gq_workspace_bytes"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(gq):
+    names = declared_entry_points()
+    nm = subprocess.run(["nm", "-D", "--defined-only", gq.LIB_PATH], capture_output=True,
+                        text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(gq_\w+)$", nm, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(gq.LIB_PATH)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_version_and_status_strings(gq):
+    assert gq.gq_version() >= 100
+    for st in (0, -1, -2, -3, -4, -5):
+        assert gq.gq_status_string(st) != "unknown status"
+
+
+def cfg(gq, **kw):
+    return gq.GQConfig(**kw)
+
+
+def test_overflow_rule(gq):
+    # uniform: W * s must fit the sum type
+    assert gq.gq_validate(cfg(gq, s=15, bits=5, wire="int8"), 8, 100) == gq.GQ_OK      # 120
+    assert gq.gq_validate(cfg(gq, s=15, bits=5, wire="int8"), 9, 100) == gq.GQ_ERR_OVERFLOW
+    assert gq.gq_validate(cfg(gq, s=127, bits=8, wire="int16"), 8, 100) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, s=127, bits=8, wire="int8"), 2, 100) == gq.GQ_ERR_OVERFLOW
+    # exponential: sums count 2^(L-1) units of the finest level per worker
+    assert gq.gq_validate(cfg(gq, levels="exp", L=8, bits=5, wire="int16"), 8, 10) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, levels="exp", L=8, bits=5, wire="int8"), 1, 10) == \
+        gq.GQ_ERR_OVERFLOW                                                             # 128
+    assert gq.gq_validate(cfg(gq, levels="exp", L=7, bits=4, wire="int8"), 1, 10) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, levels="exp", L=7, bits=4, wire="int8"), 2, 10) == \
+        gq.GQ_ERR_OVERFLOW
+    assert gq.gq_validate(cfg(gq, levels="exp", L=15, bits=5, wire="int16"), 1, 10) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, levels="exp", L=15, bits=5, wire="int16"), 2, 10) == \
+        gq.GQ_ERR_OVERFLOW
+
+
+def test_bits_must_hold_the_codes(gq):
+    assert gq.gq_validate(cfg(gq, s=7, bits=4, wire="int8"), 1, 10) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, s=8, bits=4, wire="int8"), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, s=15, bits=5, wire="int8"), 1, 10) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, s=16, bits=5, wire="int8"), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, s=127, bits=8, wire="int8"), 1, 10) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, s=128, bits=8, wire="int16"), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, levels="exp", L=7, bits=4, wire="int16"), 1, 10) == gq.GQ_OK
+    assert gq.gq_validate(cfg(gq, levels="exp", L=8, bits=4, wire="int16"), 1, 10) == \
+        gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, bits=6), 1, 10) == gq.GQ_ERR_ARG
+
+
+def test_bad_levels_and_sizes(gq):
+    assert gq.gq_validate(cfg(gq, s=0), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, levels="exp", L=0), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, levels="exp", L=16, bits=16, wire="int16"), 1, 10) == \
+        gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, levels=7), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, scale_kind=5), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, wire=3), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq), 0, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq), 1, -1) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq), 1, 0) == gq.GQ_OK
+
+
+def test_packed_row_bytes_and_workspace(gq):
+    for bits in (4, 5, 8, 16):
+        for d in (0, 1, 127, 128, 129, 25_557_032, 1 << 30):
+            assert gq.gq_packed_row_bytes(cfg(gq, bits=bits), d) == -(-d // 128) * 16 * bits
+    ws = gq.gq_workspace_bytes(cfg(gq), 8, 1 << 20)
+    assert ws >= 256 + 8 * 8 and ws % 16 == 0
+
+
+def test_entry_points_reject_before_launch(gq):
+    lib = gq.lib()
+    c = cfg(gq, s=15, bits=5, wire="int8").c()
+    P = ctypes.c_void_p
+    good = P(0x10000000)
+    odd = P(0x10000004)
+    # null / bad sizes
+    assert lib.gq_global_norm(None, None, 4, 100, ctypes.byref(c), good, None, good, None) == \
+        gq.GQ_ERR_ARG
+    assert lib.gq_global_norm(good, None, 0, 100, ctypes.byref(c), good, None, good, None) == \
+        gq.GQ_ERR_ARG
+    # misaligned gradient
+    assert lib.gq_global_norm(odd, None, 4, 100, ctypes.byref(c), good, None, good, None) == \
+        gq.GQ_ERR_ALIGN
+    # overflowing wire type is caught before the quantize launch
+    assert lib.gq_quantize_aggregate(good, None, 9, 100, ctypes.byref(c), good, good, good, good,
+                                     good, None) == gq.GQ_ERR_OVERFLOW
+    # EF requested without an error buffer
+    cef = cfg(gq, s=15, bits=5, wire="int8", ef=True).c()
+    assert lib.gq_step_fused(good, None, 4, 100, ctypes.byref(cef), good, None, good, good, good,
+                             good, None) == gq.GQ_ERR_ARG
+    # nothing requested
+    assert lib.gq_quantize_aggregate(good, None, 4, 100, ctypes.byref(c), good, None, None, None,
+                                     good, None) == gq.GQ_ERR_ARG
+    # LQ calls need the LOG level set and matching shapes
+    rows = (ctypes.c_int * 2)(4096, 4096)
+    cols = (ctypes.c_int * 2)(1, 1)
+    assert lib.gq_logq_quantize(good, 8, 2, rows, cols, ctypes.byref(c), good, good, good,
+                                None) == gq.GQ_ERR_ARG
+    clog = cfg(gq, levels="log", alpha=10.0).c()
+    assert lib.gq_logq_quantize(good, 8, 0, rows, cols, ctypes.byref(clog), good, good, good,
+                                None) == gq.GQ_ERR_ARG
+    clog_bad = cfg(gq, levels="log", alpha=-1.0).c()
+    assert lib.gq_logq_decode_sum(good, good, 8, 2, rows, cols, ctypes.byref(clog_bad), good,
+                                  None) == gq.GQ_ERR_ARG
