@@ -137,9 +137,13 @@ int gqo_global_scale(const float* g, const float* e, int W, int64_t d,
  * Quantizers.
  *
  * UNIFORM ([NUQ] Abstract names QSGD; [GQ] gives the shared scale): levels
- * {0, 1/s, ..., 1} of S.  a = fl(s/S); r = fl(|v|*a), clamped to s (the
- * product can overshoot s by rounding); l = floor(r), p = r - l (exact);
- * k = l + [p + u >= 1]; code = -k if v's sign bit is set, else k.
+ * {0, +-1/s, ..., +-1} of S.  a = fl(s/S); r = fl(v*a) (signed), clamped to
+ * [-s, s] (the product can overshoot by rounding); l = floor(r), p = r - l
+ * (exact, also for negative r); code = l + [p + u >= 1].  Rounding the signed
+ * value this way gives each coordinate the same two outcomes with the same
+ * probabilities as attaching v's sign to the rounded magnitude (for r = -2.3:
+ * -3 with probability 0.3, -2 with probability 0.7), so the quantizer is the
+ * same unbiased random variable; only the coupling to u differs.
  *
  * EXP ([NUQ] Abstract: nonuniform levels): levels {0, 2^-(L-1), ..., 1/2, 1}
  * of S.  a = fl(1/S); r = fl(|v|*a), clamped to 1.  If r >= 2^-(L-1) write
@@ -159,13 +163,13 @@ static float uniform_magnitude_ratio(int s, float S)
 
 static int32_t quantize_uniform(float v, float a, int s, uint32_t f)
 {
-    float r = fabsf(v) * a;
+    float r = v * a;
     float smax = (float)s;
     if (!(r <= smax)) r = smax; /* also maps NaN to s, as fminf does */
+    if (r < -smax) r = -smax;
     float l = floorf(r);
     float p = r - l;
-    int32_t k = (int32_t)l + round_up(p, f);
-    return sign_negative(v) ? -k : k;
+    return (int32_t)l + round_up(p, f);
 }
 
 static int32_t quantize_exp(float v, float a, int L, uint32_t f)
@@ -239,7 +243,12 @@ int32_t gqo_code_value(int32_t code, int levels, int L)
 
 /* ------------------------------------------------------------------------
  * Wire packing (a reading: the pages fix only the bit count, [LQ] "Core
- * claim": b-bit indices are sent instead of 32-bit floats).
+ * claim": b-bit indices are sent instead of 32-bit floats).  A row holds
+ * ceil(d/128) blocks of 128 codes; coordinates past d carry code 0.
+ *  bits 4, 5: little-endian bitstream, code j in stream bits [b*j, b*j + b),
+ *             stored in excess-2^(b-1) form (field = code + 2^(b-1), so the
+ *             codes -(2^(b-1)-1) .. 2^(b-1)-1 use fields 1 .. 2^b - 1);
+ *  bits 8, 16: one two's-complement int8 / int16 per code.
  * ---------------------------------------------------------------------- */
 int64_t gqo_packed_row_bytes(int bits, int64_t d)
 {
@@ -249,18 +258,25 @@ int64_t gqo_packed_row_bytes(int bits, int64_t d)
     return blocks * 16 * bits;
 }
 
+static int32_t field_bias(int bits)
+{
+    return (bits == 4 || bits == 5) ? (int32_t)1 << (bits - 1) : 0;
+}
+
 int gqo_pack(const int32_t* codes, int W, int64_t d, int bits, uint8_t* out)
 {
     int64_t rb = gqo_packed_row_bytes(bits, d);
     if (rb < 0 || !codes || !out || W < 1) return -1;
-    int32_t lo = -(1 << (bits - 1)), hi = (1 << (bits - 1)) - 1;
+    int32_t hi = (1 << (bits - 1)) - 1;
+    int32_t lo = (bits == 4 || bits == 5) ? -hi : -hi - 1;
+    int64_t padded = rb * 8 / bits; /* codes per row, padding included */
     memset(out, 0, (size_t)(rb * W));
     for (int w = 0; w < W; ++w) {
         uint8_t* row = out + (int64_t)w * rb;
-        for (int64_t j = 0; j < d; ++j) {
-            int32_t c = codes[(int64_t)w * d + j];
+        for (int64_t j = 0; j < padded; ++j) {
+            int32_t c = j < d ? codes[(int64_t)w * d + j] : 0;
             if (c < lo || c > hi) return -2;
-            uint32_t field = (uint32_t)c & ((1u << bits) - 1u);
+            uint32_t field = (uint32_t)(c + field_bias(bits)) & ((1u << bits) - 1u);
             if (bits == 8) {
                 row[j] = (uint8_t)field;
             } else if (bits == 16) {
@@ -298,8 +314,13 @@ int gqo_unpack(const uint8_t* packed, int W, int64_t d, int bits,
                     if ((row[k / 8] >> (k % 8)) & 1u) field |= 1u << t;
                 }
             }
-            int32_t c = (int32_t)field;
-            if (field & (1u << (bits - 1))) c -= (int32_t)1 << bits;
+            int32_t c;
+            if (bits == 4 || bits == 5) {
+                c = (int32_t)field - field_bias(bits);
+            } else {
+                c = (int32_t)field;
+                if (field & (1u << (bits - 1))) c -= (int32_t)1 << bits;
+            }
             codes_out[(int64_t)w * d + j] = c;
         }
     }

@@ -94,9 +94,11 @@ int32_t gqo_code_value(int32_t code, int levels, int L);
  * ceil(d/128) blocks of 16*bits bytes. */
 int64_t gqo_packed_row_bytes(int bits, int64_t d);
 
-/* Pack [W][d] int32 codes at wire width into [W][row_bytes] bytes.
+/* Pack [W][d] int32 codes at wire width into [W][row_bytes] bytes; the
+ * padding coordinates past d carry code 0.
  * 4/5 bits: little-endian bitstream, code j in bits [b*j, b*j+b) of the row,
- * two's complement, zero padding.  8: int8 per code.  16: int16 per code.
+ * excess-2^(b-1) fields (code + 2^(b-1)), codes in +-(2^(b-1) - 1).
+ * 8: int8 per code.  16: int16 per code (two's complement).
  * Returns 0, -1 on bad arguments, -2 if a code does not fit. */
 int gqo_pack(const int32_t* codes, int W, int64_t d, int bits, uint8_t* out);
 int gqo_unpack(const uint8_t* packed, int W, int64_t d, int bits,
