@@ -200,11 +200,11 @@ GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream) {
 GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long long d,
                           const gq_config* cfg, float* scale_dev, double* norms_dev, void* ws_dev,
                           cudaStream_t stream) {
-    if (!cfg || !g_dev || !scale_dev || !ws_dev) return GQ_ERR_ARG;
+    if (!cfg || (!g_dev && d > 0) || !scale_dev || !ws_dev) return GQ_ERR_ARG;
     int rc = check_sizes(W, d);
     if (rc) return rc;
     if ((rc = check_scale_kind(cfg))) return rc;
-    if (cfg->ef && !e_dev) return GQ_ERR_ARG;
+    if (cfg->ef && !e_dev && d > 0) return GQ_ERR_ARG;
     if (!aligned16(g_dev) || (e_dev && !aligned16(e_dev)) || !aligned16(ws_dev) ||
         !aligned4(scale_dev) || (norms_dev && !aligned8(norms_dev)))
         return GQ_ERR_ALIGN;

@@ -70,11 +70,17 @@ __device__ __forceinline__ int with_sign_of(int k, float v) {
     return (k ^ sgn) - sgn;
 }
 
-// Uniform levels {0, 1/s, ..., 1}: a = fl(s/S), r = min(fl(|v| a), s).
-// fminf also maps a NaN product to s, so no input can escape the range.
+// Uniform levels {0, +-1/s, ..., +-1}: a = fl(s/S), r = fl(v a) clamped to
+// [-s, s] (fminf also maps a NaN product to s), code = floor(r + u).  The
+// signed value is rounded directly: each coordinate gets the same two
+// outcomes with the same probabilities as sign(v) * floor(|r| + u), and no
+// sign handling is needed.  Same conversion-free floor as above, with base
+// 1.5 * 2^23 so that negative sums stay in [2^23, 2^24).
 __device__ __forceinline__ int quant_uniform(float v, float a, float smax, uint32_t word) {
-    const float r = fminf(__fmul_rn(fabsf(v), a), smax);
-    return with_sign_of(floor_y_plus_u(r, unit_plus_u(word)), v);
+    const float r = fmaxf(fminf(__fmul_rn(v, a), smax), -smax);
+    const float t1 = __fadd_rd(r, unit_plus_u(word));
+    const float t2 = __fadd_rd(t1, 12582912.0f);
+    return __float_as_int(t2) - 0x4B400001;
 }
 
 // Exponential levels {0, 2^-(L-1), ..., 1/2, 1}: a = fl(1/S), r = min(fl(|v| a), 1).
@@ -119,36 +125,57 @@ __device__ __forceinline__ float small_int_to_float(int x) {
 // ---------------------------------------------------------------------------
 // Warp packing.  A warp covers one 128-coordinate block of one worker's row;
 // lane l holds codes 4l..4l+3.  Wire layout: bits 4/5 -- little-endian
-// bitstream (code j at stream bits [b j, b j + b)); 8 -- int8; 16 -- int16.
-// One block is 16 * BITS bytes, so every warp store is aligned and in range.
+// bitstream of excess-2^(b-1) fields (code j at stream bits [b j, b j + b));
+// 8 -- int8; 16 -- int16.  One block is 16 * BITS bytes, so every warp store
+// is aligned and in range.
 // ---------------------------------------------------------------------------
+
+// PTX shifts clamp the amount to the register width (shift by >= 32 gives 0),
+// unlike C++ shifts, so a lane can OR in a neighbour's chunk unconditionally.
+__device__ __forceinline__ uint32_t shl_clamped(uint32_t x, uint32_t n) {
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
+    return r;
+}
+__device__ __forceinline__ uint32_t shr_clamped(uint32_t x, uint32_t n) {
+    uint32_t r;
+    asm("shr.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
+    return r;
+}
+
 template <int BITS>
 struct Packer {
-    int src0;  // bits 5: first lane whose 20-bit chunk reaches this lane's word
-    int off;   // bits 5: bit offset of that chunk inside the word
+    // bits 5: lane k < 20 stores word k = stream bits [32k, 32k + 32), which
+    // start inside the 20-bit chunk of lane src0 = floor(8k/5) at bit offset
+    // off = 32k - 20 src0 and reach at most two chunks further.  Only lane 19
+    // has src0 + 2 = 32; it reads lane 31 twice and its shift of 40 - off = 32
+    // clears the second copy.
+    int src0, src2;
+    uint32_t sh0, sh1, sh2;
     __device__ __forceinline__ void init(int lane) {
         if (BITS == 5) {
             src0 = min((8 * lane) / 5, 30);
-            off = lane < 20 ? 32 * lane - 20 * src0 : 0;  // lanes >= 20 store nothing
+            src2 = min(src0 + 2, 31);
+            const int off = lane < 20 ? 32 * lane - 20 * src0 : 0;  // lanes >= 20 store nothing
+            sh0 = (uint32_t)off;
+            sh1 = (uint32_t)(20 - off);
+            sh2 = (uint32_t)(40 - off);
         }
     }
     // Pack and store the 4 codes of this lane; dst is the block's first byte.
     __device__ __forceinline__ void store(int lane, int c0, int c1, int c2, int c3,
                                           unsigned char* dst) const {
         if (BITS == 5) {
-            const uint32_t x = (uint32_t)(c0 & 31) | ((uint32_t)(c1 & 31) << 5) |
-                               ((uint32_t)(c2 & 31) << 10) | ((uint32_t)(c3 & 31) << 15);
+            // excess-16 fields without masking: sum of c_i 32^i plus 16 * (1 + 32 + 1024 + 32768)
+            const uint32_t x = (uint32_t)(c0 + c1 * 32 + c2 * 1024 + c3 * 32768 + 541200);
             const uint32_t x0 = __shfl_sync(kFull, x, src0);
             const uint32_t x1 = __shfl_sync(kFull, x, src0 + 1);
-            const uint32_t x2 = __shfl_sync(kFull, x, min(src0 + 2, 31));
-            const unsigned long long y = (unsigned long long)x0 |
-                                         ((unsigned long long)x1 << 20) |
-                                         ((unsigned long long)x2 << 40);
-            const uint32_t word = (uint32_t)(y >> off);
+            const uint32_t x2 = __shfl_sync(kFull, x, src2);
+            const uint32_t word = shr_clamped(x0, sh0) | shl_clamped(x1, sh1) | shl_clamped(x2, sh2);
             if (lane < 20) reinterpret_cast<uint32_t*>(dst)[lane] = word;
         } else if (BITS == 4) {
-            const uint32_t x = (uint32_t)(c0 & 15) | ((uint32_t)(c1 & 15) << 4) |
-                               ((uint32_t)(c2 & 15) << 8) | ((uint32_t)(c3 & 15) << 12);
+            // excess-8 fields: sum of c_i 16^i plus 8 * (1 + 16 + 256 + 4096)
+            const uint32_t x = (uint32_t)(c0 + c1 * 16 + c2 * 256 + c3 * 4096 + 34952);
             const uint32_t xa = __shfl_sync(kFull, x, (2 * lane) & 31);
             const uint32_t xb = __shfl_sync(kFull, x, (2 * lane + 1) & 31);
             if (lane < 16) reinterpret_cast<uint32_t*>(dst)[lane] = xa | (xb << 16);
@@ -186,18 +213,18 @@ struct Unpacker {
             const uint32_t a = __shfl_sync(kFull, mine, w0);
             const uint32_t b = __shfl_sync(kFull, mine, min(w0 + 1, 31));
             const uint32_t x = __funnelshift_r(a, b, off);
-            c0 = sext(x, 5);
-            c1 = sext(x >> 5, 5);
-            c2 = sext(x >> 10, 5);
-            c3 = sext(x >> 15, 5);
+            c0 = (int)(x & 31) - 16;
+            c1 = (int)((x >> 5) & 31) - 16;
+            c2 = (int)((x >> 10) & 31) - 16;
+            c3 = (int)((x >> 15) & 31) - 16;
         } else if (BITS == 4) {
             const uint32_t mine = lane < 16 ? reinterpret_cast<const uint32_t*>(src)[lane] : 0u;
             const uint32_t wv = __shfl_sync(kFull, mine, lane >> 1);
             const uint32_t x = (lane & 1) ? (wv >> 16) : wv;
-            c0 = sext(x, 4);
-            c1 = sext(x >> 4, 4);
-            c2 = sext(x >> 8, 4);
-            c3 = sext(x >> 12, 4);
+            c0 = (int)(x & 15) - 8;
+            c1 = (int)((x >> 4) & 15) - 8;
+            c2 = (int)((x >> 8) & 15) - 8;
+            c3 = (int)((x >> 12) & 15) - 8;
         } else if (BITS == 8) {
             const uint32_t x = reinterpret_cast<const uint32_t*>(src)[lane];
             c0 = sext(x, 8);

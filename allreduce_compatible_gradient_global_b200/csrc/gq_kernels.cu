@@ -336,7 +336,20 @@ cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 // Steps 2-5 fused.
 // ---------------------------------------------------------------------------
-constexpr int kWorkerBatch = 8;  // worker rows loaded before any is processed
+// Tuning of the fused pass: worker rows loaded before any is processed,
+// resident blocks per SM the register budget is cut for, and whether warps
+// walk the 128-coordinate blocks from the end of the rows (the end of the rows
+// is what the norm pass left in L2).
+#ifndef GQ_WORKER_BATCH
+#define GQ_WORKER_BATCH 8
+#endif
+#ifndef GQ_QUANT_MIN_BLOCKS
+#define GQ_QUANT_MIN_BLOCKS 2
+#endif
+#ifndef GQ_QUANT_REVERSE
+#define GQ_QUANT_REVERSE 0
+#endif
+constexpr int kWorkerBatch = GQ_WORKER_BATCH;
 
 template <int LEVELS>
 __device__ __forceinline__ int quantize_one(float v, float aq, const QuantArgs& a, uint32_t word) {
@@ -345,7 +358,8 @@ __device__ __forceinline__ int quantize_one(float v, float aq, const QuantArgs& 
 }
 
 template <int LEVELS, int BITS, bool EF, bool VEC>
-__global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__ QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, GQ_QUANT_MIN_BLOCKS)
+    quant_kernel(const __grid_constant__ QuantArgs a) {
     const int lane = threadIdx.x & 31;
     const long long nblk = (a.d + 127) >> 7;
     const long long wid = ((long long)blockIdx.x * kThreads + threadIdx.x) >> 5;
@@ -355,7 +369,8 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     Packer<BITS> pk;
     pk.init(lane);
 
-    for (long long blk = wid; blk < nblk; blk += nwarps) {
+    for (long long it = wid; it < nblk; it += nwarps) {
+        const long long blk = GQ_QUANT_REVERSE ? nblk - 1 - it : it;
         const long long j0 = (blk << 7) + (lane << 2);
         const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
         int s0 = 0, s1 = 0, s2 = 0, s3 = 0;

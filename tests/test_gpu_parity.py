@@ -93,7 +93,8 @@ CASES = [
     (8, 40000, dict(levels="exp", L=8, bits=5, wire="int16", scale_kind="maxabs")),
     (8, 40001, dict(levels="exp", L=8, bits=5, wire="int16", scale_kind="l2", seed=5)),
     (2, 3333, dict(levels="exp", L=3, bits=4, wire="int8", step=2)),
-    (4, 12345, dict(levels="exp", L=15, bits=5, wire="int16")),
+    (4, 12345, dict(levels="exp", L=13, bits=5, wire="int16")),
+    (1, 2222, dict(levels="exp", L=15, bits=5, wire="int16")),
     (4, 9000, dict(s=15, bits=5, wire="int8", scale_kind="maxabs")),
     (12, 5000, dict(s=2, bits=4, wire="int8", seed=0xFFFFFFFFFFFFFFFF, step=0xFFFFFFFF)),
 ]
@@ -139,11 +140,12 @@ def test_error_feedback_steps_match_oracle(gq, oracle, W, d, kw, split):
         e_ref = ref["e"]
 
 
-def test_zero_input_and_empty(gq):
+def test_zero_input_and_empty(gq, oracle):
     cfg = gq.GQConfig(s=15, bits=5, wire="int8")
     g = torch.zeros((4, 1000), device="cuda")
     r = gpu_step(gq, g, None, cfg)
-    assert r["S"] == 0 and not r["codes"].any() and not r["sum"].any() and not r["out"].any()
+    assert r["S"] == 0 and not r["sum"].any() and not r["out"].any()
+    assert np.array_equal(r["codes"], oracle.pack(np.zeros((4, 1000), np.int32), 5))
     g0 = torch.zeros((4, 0), device="cuda")
     buf = gq.StepBuffers(cfg, 4, 0)
     gq.gq_global_norm(g0, None, cfg, buf.scale, buf.norms, buf.ws)
