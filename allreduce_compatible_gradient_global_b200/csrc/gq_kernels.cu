@@ -341,10 +341,10 @@ cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st) {
 // walk the 128-coordinate blocks from the end of the rows (the end of the rows
 // is what the norm pass left in L2).
 #ifndef GQ_WORKER_BATCH
-#define GQ_WORKER_BATCH 8
+#define GQ_WORKER_BATCH 4
 #endif
 #ifndef GQ_QUANT_MIN_BLOCKS
-#define GQ_QUANT_MIN_BLOCKS 2
+#define GQ_QUANT_MIN_BLOCKS 3
 #endif
 #ifndef GQ_QUANT_REVERSE
 #define GQ_QUANT_REVERSE 0
