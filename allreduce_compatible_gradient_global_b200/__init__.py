@@ -5,8 +5,9 @@ A thin ctypes layer over the C ABI in ``include/gq_api.h``: every function has
 the C entry point's name, takes torch tensors (device memory and streams come
 from PyTorch), checks dtypes and shapes, passes raw pointers and raises
 ``GQError`` on a non-zero status.  All arithmetic runs in the CUDA kernels of
-libgq.so; there is no fallback: if the library is missing, importing this
-package fails with instructions to build it.
+libgq.so; there is no fallback: if the library is missing, the first call
+raises ImportError with instructions to build it (importing the package alone
+does not load it, so that the build step can run from a fresh checkout).
 """
 import ctypes
 import os
@@ -107,19 +108,23 @@ def _load():
     return lib
 
 
-_lib = _load()
+_lib = None
 
 
 def lib():
+    """The loaded libgq.so (loaded on first use; raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
     return _lib
 
 
 def gq_version() -> int:
-    return _lib.gq_version()
+    return lib().gq_version()
 
 
 def gq_status_string(status: int) -> str:
-    return _lib.gq_status_string(int(status)).decode()
+    return lib().gq_status_string(int(status)).decode()
 
 
 # ------------------------------------------------------------------ marshalling
@@ -160,13 +165,13 @@ def _wd(g):
 # ------------------------------------------------------------------ sizes
 def gq_validate(cfg: GQConfig, W: int, d: int) -> int:
     c = cfg.c()
-    return _lib.gq_validate(ctypes.byref(c), int(W), int(d))
+    return lib().gq_validate(ctypes.byref(c), int(W), int(d))
 
 
 def gq_packed_row_bytes(cfg: GQConfig, d: int) -> int:
     c = cfg.c()
     out = ctypes.c_longlong()
-    _check(_lib.gq_packed_row_bytes(ctypes.byref(c), int(d), ctypes.byref(out)),
+    _check(lib().gq_packed_row_bytes(ctypes.byref(c), int(d), ctypes.byref(out)),
            "gq_packed_row_bytes")
     return out.value
 
@@ -174,19 +179,19 @@ def gq_packed_row_bytes(cfg: GQConfig, d: int) -> int:
 def gq_workspace_bytes(cfg: GQConfig, W: int, d: int) -> int:
     c = cfg.c()
     out = ctypes.c_size_t()
-    _check(_lib.gq_workspace_bytes(ctypes.byref(c), int(W), int(d), ctypes.byref(out)),
+    _check(lib().gq_workspace_bytes(ctypes.byref(c), int(W), int(d), ctypes.byref(out)),
            "gq_workspace_bytes")
     return out.value
 
 
 def gq_workspace_init(ws, stream=None):
-    _check(_lib.gq_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+    _check(lib().gq_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "gq_workspace_init")
 
 
 def gq_get_device_status(ws, stream=None) -> int:
     """Synchronizes the stream; returns GQ_OK or GQ_ERR_NONFINITE (and clears it)."""
-    rc = _lib.gq_get_device_status(_ptr(ws), _stream(stream))
+    rc = lib().gq_get_device_status(_ptr(ws), _stream(stream))
     if rc not in (GQ_OK, GQ_ERR_NONFINITE):
         raise GQError(rc, "gq_get_device_status")
     return rc
@@ -200,7 +205,7 @@ def gq_global_norm(g, e, cfg: GQConfig, scale, norms, ws, stream=None):
     _need(scale, torch.float32, (1,), "scale")
     _need(norms, torch.float64, (W,), "norms")
     c = cfg.c()
-    _check(_lib.gq_global_norm(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale), _ptr(norms),
+    _check(lib().gq_global_norm(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale), _ptr(norms),
                                _ptr(ws), _stream(stream)), "gq_global_norm")
 
 
@@ -210,7 +215,7 @@ def gq_quantize_pack(g, e, cfg: GQConfig, scale, codes, ws, stream=None):
     _need(e, torch.float32, (W, d), "e")
     _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
     c = cfg.c()
-    _check(_lib.gq_quantize_pack(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale),
+    _check(lib().gq_quantize_pack(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale),
                                  _ptr(codes), _ptr(ws), _stream(stream)), "gq_quantize_pack")
 
 
@@ -218,7 +223,7 @@ def gq_aggregate(codes, W, d, cfg: GQConfig, sum_out, ws, stream=None):
     _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
     _need(sum_out, cfg.wire_dtype, (d,), "sum")
     c = cfg.c()
-    _check(_lib.gq_aggregate(_ptr(codes), int(W), int(d), ctypes.byref(c), _ptr(sum_out),
+    _check(lib().gq_aggregate(_ptr(codes), int(W), int(d), ctypes.byref(c), _ptr(sum_out),
                              _ptr(ws), _stream(stream)), "gq_aggregate")
 
 
@@ -229,7 +234,7 @@ def gq_dequantize_ef(sum_in, codes, g, e, W, d, cfg: GQConfig, scale, out, ws, s
     _need(e, torch.float32, (W, d), "e")
     _need(out, torch.float32, (d,), "out")
     c = cfg.c()
-    _check(_lib.gq_dequantize_ef(_ptr(sum_in), _ptr(codes), _ptr(g), _ptr(e), int(W), int(d),
+    _check(lib().gq_dequantize_ef(_ptr(sum_in), _ptr(codes), _ptr(g), _ptr(e), int(W), int(d),
                                  ctypes.byref(c), _ptr(scale), _ptr(out), _ptr(ws),
                                  _stream(stream)), "gq_dequantize_ef")
 
@@ -242,7 +247,7 @@ def gq_quantize_aggregate(g, e, cfg: GQConfig, scale, codes, sum_out, out, ws, s
     _need(sum_out, cfg.wire_dtype, (d,), "sum")
     _need(out, torch.float32, (d,), "out")
     c = cfg.c()
-    _check(_lib.gq_quantize_aggregate(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale),
+    _check(lib().gq_quantize_aggregate(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale),
                                       _ptr(codes), _ptr(sum_out), _ptr(out), _ptr(ws),
                                       _stream(stream)), "gq_quantize_aggregate")
 
@@ -257,7 +262,7 @@ def gq_step_fused(g, e, cfg: GQConfig, scale, norms, codes, sum_out, out, ws, st
     _need(sum_out, cfg.wire_dtype, (d,), "sum")
     _need(out, torch.float32, (d,), "out")
     c = cfg.c()
-    _check(_lib.gq_step_fused(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale), _ptr(norms),
+    _check(lib().gq_step_fused(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale), _ptr(norms),
                               _ptr(codes), _ptr(sum_out), _ptr(out), _ptr(ws), _stream(stream)),
            "gq_step_fused")
 
@@ -272,7 +277,7 @@ def gq_step_fused_host(g_host, g_dev, e, cfg: GQConfig, scale, codes, sum_out, o
     _need(g_dev, torch.float32, (W, d), "g_dev")
     _need(out, torch.float32, (d,), "out")
     c = cfg.c()
-    _check(_lib.gq_step_fused_host(_ptr(g_host), _ptr(g_dev), _ptr(e), W, d, ctypes.byref(c),
+    _check(lib().gq_step_fused_host(_ptr(g_host), _ptr(g_dev), _ptr(e), W, d, ctypes.byref(c),
                                    _ptr(scale), _ptr(codes), _ptr(sum_out), _ptr(out),
                                    _ptr(out_host), _ptr(scale_host), _ptr(ws), _stream(stream)),
            "gq_step_fused_host")
@@ -293,7 +298,7 @@ def gq_logq_quantize(x, rows, cols, cfg: GQConfig, maxabs, codes, ws, stream=Non
     _need(codes, torch.int8, (W, n), "codes")
     r, cc = _shapes(rows, cols)
     c = cfg.c()
-    _check(_lib.gq_logq_quantize(_ptr(x), W, len(rows), r, cc, ctypes.byref(c), _ptr(maxabs),
+    _check(lib().gq_logq_quantize(_ptr(x), W, len(rows), r, cc, ctypes.byref(c), _ptr(maxabs),
                                  _ptr(codes), _ptr(ws), _stream(stream)), "gq_logq_quantize")
 
 
@@ -304,7 +309,7 @@ def gq_logq_decode_sum(codes, maxabs, rows, cols, cfg: GQConfig, out, stream=Non
     _need(out, torch.float32, (n,), "out")
     r, cc = _shapes(rows, cols)
     c = cfg.c()
-    _check(_lib.gq_logq_decode_sum(_ptr(codes), _ptr(maxabs), W, len(rows), r, cc,
+    _check(lib().gq_logq_decode_sum(_ptr(codes), _ptr(maxabs), W, len(rows), r, cc,
                                    ctypes.byref(c), _ptr(out), _stream(stream)),
            "gq_logq_decode_sum")
 
