@@ -24,6 +24,7 @@ GQ_ERR_OVERFLOW = -2
 GQ_ERR_ALIGN = -3
 GQ_ERR_CUDA = -4
 GQ_ERR_NONFINITE = -5
+GQ_ERR_SIZE = -6
 
 UNIFORM, EXP, LOG = 0, 1, 2
 SCALE_L2, SCALE_MAXABS = 0, 1
@@ -92,6 +93,7 @@ def _load():
         "gq_workspace_init": ([P, ctypes.c_size_t, P], I),
         "gq_get_device_status": ([P, P], I),
         "gq_global_norm": ([P, P, I, LL, CP, P, P, P, P], I),
+        "gq_global_norm_noalloc": ([P, P, I, LL, CP, P, P, P], I),
         "gq_quantize_pack": ([P, P, I, LL, CP, P, P, P, P], I),
         "gq_aggregate": ([P, I, LL, CP, P, P, P], I),
         "gq_dequantize_ef": ([P, P, P, P, I, LL, CP, P, P, P, P], I),
@@ -207,6 +209,20 @@ def gq_global_norm(g, e, cfg: GQConfig, scale, norms, ws, stream=None):
     c = cfg.c()
     _check(lib().gq_global_norm(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale), _ptr(norms),
                                _ptr(ws), _stream(stream)), "gq_global_norm")
+
+
+def gq_global_norm_noalloc(g, e, cfg: GQConfig, scale, norms, stream=None):
+    """gq_global_norm without a workspace, for callers that cannot allocate:
+    the library's own fixed device scratch holds the partial sums (W <= 4096;
+    calls that overlap on the GPU race on that scratch)."""
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(scale, torch.float32, (1,), "scale")
+    _need(norms, torch.float64, (W,), "norms")
+    c = cfg.c()
+    _check(lib().gq_global_norm_noalloc(_ptr(g), _ptr(e), W, d, ctypes.byref(c), _ptr(scale),
+                                       _ptr(norms), _stream(stream)), "gq_global_norm_noalloc")
 
 
 def gq_quantize_pack(g, e, cfg: GQConfig, scale, codes, ws, stream=None):

@@ -151,6 +151,7 @@ GQ_API const char* gq_status_string(int status) {
         case GQ_ERR_ALIGN: return "buffer not 16-byte aligned";
         case GQ_ERR_CUDA: return "CUDA error";
         case GQ_ERR_NONFINITE: return "non-finite scale (NaN or Inf in the input)";
+        case GQ_ERR_SIZE: return "size beyond the fixed maximum of this entry point";
         default: return "unknown status";
     }
 }

@@ -71,6 +71,7 @@ extern "C" {
 #define GQ_ERR_ALIGN (-3)      /* a buffer is not 16-byte aligned */
 #define GQ_ERR_CUDA (-4)       /* a CUDA runtime call or launch failed */
 #define GQ_ERR_NONFINITE (-5)  /* device flag: a scale or LQ max was not finite */
+#define GQ_ERR_SIZE (-6)       /* beyond the fixed maximum of gq_global_norm_noalloc */
 
 /* Level sets. */
 #define GQ_UNIFORM 0 /* {0, 1/s, ..., 1}: QSGD levels */
@@ -142,6 +143,30 @@ GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream);
 GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long long d,
                           const gq_config* cfg, float* scale_dev, double* norms_dev,
                           void* ws_dev, cudaStream_t stream);
+
+/* Step 1 for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this call: it is a convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc or hand over a workspace: code that runs
+ * where another allocator owns the device memory (a framework's caching
+ * allocator, or a fixed arena that forbids outside allocations), or a hot path
+ * that cannot afford cudaMalloc's cost and its implicit device-wide
+ * synchronization.  This call computes exactly what gq_global_norm computes
+ * (same kernel, same arguments minus the workspace) but keeps its block
+ * partials and ticket counter in a fixed device array inside the library:
+ * 256 + 8192 * 8 bytes, held by every GPU that loads the library until the
+ * process exits.  It allocates nothing and calls no allocating routine.
+ *
+ * Limits: W <= 4096, else GQ_ERR_SIZE (nothing is launched).  The first call
+ * on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it, so make that first call before
+ * any stream capture.  All calls share the one array: each call clears its
+ * counter and flag word on `stream` before launching, and calls that overlap
+ * on the GPU (other streams, other threads) race on it.  A NaN or Inf input
+ * shows as a non-finite scale_dev[0]; this call has no flag word to read. */
+GQ_API int gq_global_norm_noalloc(const float* g_dev, const float* e_dev, int W, long long d,
+                                  const gq_config* cfg, float* scale_dev, double* norms_dev,
+                                  cudaStream_t stream);
 
 /* Steps 2-3 -- stochastic quantization and packing, given the scale on the
  * device.  UNIFORM: a = fl(s/S), r = min(fl(|v|*a), s), code = sign(v) *
