@@ -25,6 +25,7 @@ GQ_ERR_ALIGN = -3
 GQ_ERR_CUDA = -4
 GQ_ERR_NONFINITE = -5
 GQ_ERR_SIZE = -6
+GQ_ERR_TIMEOUT = -7
 
 UNIFORM, EXP, LOG = 0, 1, 2
 SCALE_L2, SCALE_MAXABS = 0, 1
@@ -192,7 +193,8 @@ def gq_workspace_init(ws, stream=None):
 
 
 def gq_get_device_status(ws, stream=None) -> int:
-    """Synchronizes the stream; returns GQ_OK or GQ_ERR_NONFINITE (and clears it)."""
+    """Synchronizes the stream; returns GQ_OK or GQ_ERR_NONFINITE (and clears the
+    flag).  A timed-out pipeline wait raises GQError(GQ_ERR_TIMEOUT)."""
     rc = lib().gq_get_device_status(_ptr(ws), _stream(stream))
     if rc not in (GQ_OK, GQ_ERR_NONFINITE):
         raise GQError(rc, "gq_get_device_status")

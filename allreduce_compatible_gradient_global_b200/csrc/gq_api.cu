@@ -93,6 +93,48 @@ int norm_blocks_per_worker(int W, long long d) {
     return (int)nb;
 }
 
+int stream_grid(long long d);
+
+// The bulk-copy pipeline of the fused pass: stages per block (compile-time
+// knob), and whether it is used at all.
+#ifndef GQ_TMA_STAGES
+#define GQ_TMA_STAGES 3
+#endif
+#ifndef GQ_USE_TMA
+#define GQ_USE_TMA 1
+#endif
+constexpr size_t kSmemPerBlockMax = 232448;  // 227 KiB of dynamic shared memory
+constexpr size_t kSmemPerSm = 233472;        // 228 KiB per SM, 1 KiB reserved per block
+
+// Stages that fit one block for W rows (2W with error feedback), or 0 when the
+// rows do not fit even two stages (then the register-staged kernel runs).
+int tma_stages(int W, bool ef) {
+    for (int s = GQ_TMA_STAGES; s >= 2; --s)
+        if (tma_smem_bytes(W, ef, s) <= kSmemPerBlockMax) return s;
+    return 0;
+}
+
+int tma_grid(long long d, int W, bool ef, int stages) {
+    const long long tiles = (d + 1023) / 1024;
+    long long per_sm = (long long)(kSmemPerSm / (tma_smem_bytes(W, ef, stages) + 1024));
+    if (per_sm < 1) per_sm = 1;
+    const long long cap = (long long)sm_count() * per_sm;
+    const long long g = tiles < cap ? tiles : cap;
+    return g < 1 ? 1 : (int)g;
+}
+
+// Launch the fused pass on the best path for the shape.
+cudaError_t launch_fused(QuantArgs& a, int levels, int bits, bool ef_read, void* ws, long long d,
+                         cudaStream_t stream) {
+    const bool vec = (d % 4) == 0;
+    const int stages = (GQ_USE_TMA && vec) ? tma_stages(a.W, ef_read) : 0;
+    a.hdr = reinterpret_cast<WsHeader*>(ws);
+    if (stages > 0)
+        return launch_quant_tma(a, levels, bits, ef_read, stages,
+                                tma_grid(d, a.W, ef_read, stages), stream);
+    return launch_quant(a, levels, bits, ef_read, vec, stream_grid(d), stream);
+}
+
 int stream_grid(long long d) {
     const long long blocks128 = (d + 127) / 128;                 // one warp each
     const long long need = (blocks128 + (kThreads / 32) - 1) / (kThreads / 32);
@@ -152,6 +194,7 @@ GQ_API const char* gq_status_string(int status) {
         case GQ_ERR_CUDA: return "CUDA error";
         case GQ_ERR_NONFINITE: return "non-finite scale (NaN or Inf in the input)";
         case GQ_ERR_SIZE: return "size beyond the fixed maximum of this entry point";
+        case GQ_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
         default: return "unknown status";
     }
 }
@@ -195,7 +238,7 @@ GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream) {
         return GQ_ERR_CUDA;
     if (flags == 0) return GQ_OK;
     if (cudaMemset(&header_of(ws_dev)->flags, 0, sizeof(flags)) != cudaSuccess) return GQ_ERR_CUDA;
-    return GQ_ERR_NONFINITE;
+    return (flags & kFlagPipelineTimeout) ? GQ_ERR_TIMEOUT : GQ_ERR_NONFINITE;
 }
 
 GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long long d,
@@ -226,10 +269,9 @@ GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long lo
 static int quant_common(const float* g_dev, float* e_dev, int W, long long d, const gq_config* cfg,
                         const float* scale_dev, void* codes_dev, void* sum_dev, float* out_dev,
                         void* ws_dev, bool allow_ef, cudaStream_t stream) {
-    (void)ws_dev;
     int rc = gq_validate(cfg, W, d);
     if (rc) return rc;
-    if (!g_dev || !scale_dev) return GQ_ERR_ARG;
+    if (!g_dev || !scale_dev || !ws_dev) return GQ_ERR_ARG;
     const bool ef = allow_ef && cfg->ef;
     if (ef && !e_dev) return GQ_ERR_ARG;
     if (!codes_dev && !sum_dev && !out_dev && !ef) return GQ_ERR_ARG;
@@ -249,8 +291,7 @@ static int quant_common(const float* g_dev, float* e_dev, int W, long long d, co
     a.sum = sum_dev;
     a.out = out_dev;
     const int bits = codes_dev ? cfg->bits : 0;
-    return cuda_status(
-        launch_quant(a, cfg->levels, bits, ef, (d % 4) == 0, stream_grid(d), stream));
+    return cuda_status(launch_fused(a, cfg->levels, bits, ef, ws_dev, d, stream));
 }
 
 GQ_API int gq_quantize_pack(const float* g_dev, const float* e_dev, int W, long long d,
@@ -265,10 +306,9 @@ GQ_API int gq_quantize_pack(const float* g_dev, const float* e_dev, int W, long 
     if (c.ef && !aligned16(e_dev)) return GQ_ERR_ALIGN;
     int rc = gq_validate(&c, W, d);
     if (rc) return rc;
-    if (!g_dev || !scale_dev) return GQ_ERR_ARG;
+    if (!g_dev || !scale_dev || !ws_dev) return GQ_ERR_ARG;
     if (!aligned16(g_dev) || !aligned4(scale_dev) || !aligned16(codes_dev)) return GQ_ERR_ALIGN;
     if (d == 0) return GQ_OK;
-    (void)ws_dev;
     QuantArgs a;
     fill_quant_args(a, &c, W, d);
     a.g = g_dev;
@@ -277,8 +317,7 @@ GQ_API int gq_quantize_pack(const float* g_dev, const float* e_dev, int W, long 
     a.scale = scale_dev;
     a.codes = reinterpret_cast<unsigned char*>(codes_dev);
     a.row_bytes = row_bytes_of(c.bits, d);
-    return cuda_status(
-        launch_quant(a, c.levels, c.bits, c.ef != 0, (d % 4) == 0, stream_grid(d), stream));
+    return cuda_status(launch_fused(a, c.levels, c.bits, c.ef != 0, ws_dev, d, stream));
 }
 
 GQ_API int gq_aggregate(const void* codes_dev, int W, long long d, const gq_config* cfg,

@@ -22,6 +22,7 @@ struct WsHeader {
 
 constexpr unsigned kFlagNonfiniteScale = 1u;
 constexpr unsigned kFlagNonfiniteLogqMax = 2u;
+constexpr unsigned kFlagPipelineTimeout = 4u;  // a bounded mbarrier wait expired
 
 struct NormArgs {
     const float* g;
@@ -56,6 +57,7 @@ struct QuantArgs {
     float inv_finest;  // 2^(L-1)
     float inv_w;       // 1/W when W is a power of two
     int w_pow2;
+    WsHeader* hdr;  // flag word for pipeline timeouts
 };
 
 struct AggArgs {
@@ -112,6 +114,11 @@ cudaError_t launch_quant(const QuantArgs& a, int levels, int bits, bool ef, bool
 cudaError_t launch_aggregate(const AggArgs& a, int levels, int bits, int grid, cudaStream_t st);
 cudaError_t launch_dequant(const DequantArgs& a, int levels, int bits, bool vec, int grid,
                            cudaStream_t st);
+// The fused pass with the worker rows staged in shared memory by bulk copies
+// (d % 4 == 0 and 16-byte-aligned rows only).
+size_t tma_smem_bytes(int W, bool ef, int stages);
+cudaError_t launch_quant_tma(const QuantArgs& a, int levels, int bits, bool ef, int stages,
+                             int grid, cudaStream_t st);
 cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st);
 cudaError_t launch_logq_decode(const LogqArgs& a, cudaStream_t st);
 

@@ -56,91 +56,6 @@ __device__ __forceinline__ void store4(float* row, long long j0, long long d, fl
     if (j0 + 2 < d) __stcs(row + j0 + 2, v.z);
 }
 
-// The [d] mean output: its base is 16-byte aligned and j0 % 4 == 0.
-__device__ __forceinline__ void store_out4(float* out, long long j0, long long d, float4 v) {
-    if (j0 + 3 < d) {
-        __stcs(reinterpret_cast<float4*>(out + j0), v);
-        return;
-    }
-    if (j0 < d) out[j0] = v.x;
-    if (j0 + 1 < d) out[j0 + 1] = v.y;
-    if (j0 + 2 < d) out[j0 + 2] = v.z;
-}
-
-__device__ __forceinline__ float4 add4(float4 a, float4 b) {
-    return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
-                       __fadd_rn(a.w, b.w));
-}
-
-// The [d] outputs (sum, mean) are vectors of their own: j0 is a multiple of 4,
-// so a 4-wide store is aligned whenever all 4 coordinates are in range.
-__device__ __forceinline__ void store_sum(void* sum, int wire, long long j0, long long d, int s0,
-                                          int s1, int s2, int s3) {
-    if (wire == 1) {
-        signed char* p = reinterpret_cast<signed char*>(sum) + j0;
-        if (j0 + 3 < d) {
-            const uint32_t x = (uint32_t)(s0 & 255) | ((uint32_t)(s1 & 255) << 8) |
-                               ((uint32_t)(s2 & 255) << 16) | ((uint32_t)(s3 & 255) << 24);
-            __stcs(reinterpret_cast<unsigned int*>(p), x);
-        } else {
-            if (j0 < d) p[0] = (signed char)s0;
-            if (j0 + 1 < d) p[1] = (signed char)s1;
-            if (j0 + 2 < d) p[2] = (signed char)s2;
-        }
-    } else {
-        short* p = reinterpret_cast<short*>(sum) + j0;
-        if (j0 + 3 < d) {
-            uint2 x;
-            x.x = (uint32_t)(s0 & 0xFFFF) | ((uint32_t)s1 << 16);
-            x.y = (uint32_t)(s2 & 0xFFFF) | ((uint32_t)s3 << 16);
-            __stcs(reinterpret_cast<uint2*>(p), x);
-        } else {
-            if (j0 < d) p[0] = (short)s0;
-            if (j0 + 1 < d) p[1] = (short)s1;
-            if (j0 + 2 < d) p[2] = (short)s2;
-        }
-    }
-}
-
-__device__ __forceinline__ void load_sum(const void* sum, int wire, long long j0, long long d,
-                                         int& s0, int& s1, int& s2, int& s3) {
-    if (wire == 1) {
-        const signed char* p = reinterpret_cast<const signed char*>(sum) + j0;
-        if (j0 + 3 < d) {
-            const uint32_t x = __ldcs(reinterpret_cast<const unsigned int*>(p));
-            s0 = (int)(signed char)(x & 255);
-            s1 = (int)(signed char)((x >> 8) & 255);
-            s2 = (int)(signed char)((x >> 16) & 255);
-            s3 = (int)(signed char)(x >> 24);
-        } else {
-            s0 = j0 < d ? p[0] : 0;
-            s1 = j0 + 1 < d ? p[1] : 0;
-            s2 = j0 + 2 < d ? p[2] : 0;
-            s3 = 0;
-        }
-    } else {
-        const short* p = reinterpret_cast<const short*>(sum) + j0;
-        if (j0 + 3 < d) {
-            const uint2 x = __ldcs(reinterpret_cast<const uint2*>(p));
-            s0 = (int)(short)(x.x & 0xFFFF);
-            s1 = (int)(short)(x.x >> 16);
-            s2 = (int)(short)(x.y & 0xFFFF);
-            s3 = (int)(short)(x.y >> 16);
-        } else {
-            s0 = j0 < d ? p[0] : 0;
-            s1 = j0 + 1 < d ? p[1] : 0;
-            s2 = j0 + 2 < d ? p[2] : 0;
-            s3 = 0;
-        }
-    }
-}
-
-// Decoded mean of one summed integer: fl(fl(sum * c) / W).
-__device__ __forceinline__ float decode_mean(int s, float c, float inv_w, int w_pow2, int W) {
-    const float y = __fmul_rn(small_int_to_float(s), c);
-    return w_pow2 ? __fmul_rn(y, inv_w) : __fdiv_rn(y, (float)W);
-}
-
 // Scale-derived constants: a (magnitude multiplier) and c (value of one unit).
 template <int LEVELS>
 __device__ __forceinline__ void scale_constants(float S, float smax, float finest, float& a,

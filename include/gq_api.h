@@ -72,6 +72,7 @@ extern "C" {
 #define GQ_ERR_CUDA (-4)       /* a CUDA runtime call or launch failed */
 #define GQ_ERR_NONFINITE (-5)  /* device flag: a scale or LQ max was not finite */
 #define GQ_ERR_SIZE (-6)       /* beyond the fixed maximum of gq_global_norm_noalloc */
+#define GQ_ERR_TIMEOUT (-7)    /* device flag: a bounded wait inside a kernel expired */
 
 /* Level sets. */
 #define GQ_UNIFORM 0 /* {0, 1/s, ..., 1}: QSGD levels */
@@ -128,7 +129,9 @@ GQ_API int gq_workspace_bytes(const gq_config* cfg, int W, long long d, size_t* 
 GQ_API int gq_workspace_init(void* ws_dev, size_t bytes, cudaStream_t stream);
 
 /* Synchronize `stream`, then read and clear the device flag word of the
- * workspace.  Returns GQ_OK, GQ_ERR_NONFINITE, or GQ_ERR_CUDA. */
+ * workspace.  Returns GQ_OK, GQ_ERR_NONFINITE, GQ_ERR_TIMEOUT (a pipeline
+ * wait in the fused pass gave up after 2 s; its outputs are incomplete), or
+ * GQ_ERR_CUDA. */
 GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream);
 
 /* Step 1 -- global scale.  g_dev, e_dev (NULL unless cfg->ef): [W][d] fp32.
@@ -204,7 +207,10 @@ GQ_API int gq_dequantize_ef(const void* sum_dev, const void* codes_dev, const fl
  * codes (if codes_dev is not NULL), keeps the integer sum in registers, and
  * writes the sum (if sum_dev), the decoded mean (if out_dev) and the error
  * feedback update (if cfg->ef and e_dev).  Results are bit-identical to
- * gq_quantize_pack + gq_aggregate + gq_dequantize_ef. */
+ * gq_quantize_pack + gq_aggregate + gq_dequantize_ef.  When d % 4 == 0 and the
+ * worker rows of a few 1024-coordinate tiles fit in shared memory, a producer
+ * warp stages them with bulk asynchronous copies (ws_dev holds the flag that
+ * a timed-out wait raises); otherwise each lane loads its rows directly. */
 GQ_API int gq_quantize_aggregate(const float* g_dev, float* e_dev, int W, long long d,
                                  const gq_config* cfg, const float* scale_dev, void* codes_dev,
                                  void* sum_dev, float* out_dev, void* ws_dev,

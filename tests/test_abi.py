@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(gq):
 
 def test_version_and_status_strings(gq):
     assert gq.gq_version() >= 100
-    for st in (0, -1, -2, -3, -4, -5, -6):
+    for st in (0, -1, -2, -3, -4, -5, -6, -7):
         assert gq.gq_status_string(st) != "unknown status"
 
 

@@ -97,6 +97,9 @@ CASES = [
     (1, 2222, dict(levels="exp", L=15, bits=5, wire="int16")),
     (4, 9000, dict(s=15, bits=5, wire="int8", scale_kind="maxabs")),
     (12, 5000, dict(s=2, bits=4, wire="int8", seed=0xFFFFFFFFFFFFFFFF, step=0xFFFFFFFF)),
+    (40, 8192, dict(s=3, bits=4, wire="int8")),           # rows too many to stage: register path
+    (16, 50000, dict(s=7, bits=4, wire="int8", seed=8)),  # 16 staged rows
+    (8, 1 << 20, dict(s=15, bits=5, wire="int8", seed=9)),  # many tiles per block
 ]
 
 
