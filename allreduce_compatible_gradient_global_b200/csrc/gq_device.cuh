@@ -83,6 +83,19 @@ __device__ __forceinline__ int quant_uniform(float v, float a, float smax, uint3
     return __float_as_int(t2) - 0x4B400001;
 }
 
+// The same rounding, returned "biased": the float 1.5 * 2^23 + code, whose bit
+// pattern is kCodeBias + code.  Adding 1.5 * 2^23 - 1 instead of 1.5 * 2^23
+// absorbs the -1 of the U offset, so no per-element subtraction is needed: the
+// low 8 / 16 bits of the pattern are already the int8 / int16 code, sums of
+// patterns differ from sums of codes by a multiple of kCodeBias, and
+// (pattern as float) - 1.5 * 2^23 is the code as a float, exactly.
+constexpr uint32_t kCodeBias = 0x4B400000u;
+__device__ __forceinline__ float quant_uniform_biased(float v, float a, float smax, uint32_t word) {
+    const float r = fmaxf(fminf(__fmul_rn(v, a), smax), -smax);
+    const float t1 = __fadd_rd(r, unit_plus_u(word));
+    return __fadd_rd(t1, 12582911.0f);
+}
+
 // Exponential levels {0, 2^-(L-1), ..., 1/2, 1}: a = fl(1/S), r = min(fl(|v| a), 1).
 // For r >= 2^-(L-1), r = (1 + m 2^-23) 2^E with m the mantissa field: the
 // bracket is [2^E, 2^(E+1)], the lower level has index L + E, and the
@@ -163,11 +176,18 @@ struct Packer {
         }
     }
     // Pack and store the 4 codes of this lane; dst is the block's first byte.
+    // The inputs are code + BIAS (mod 2^32) for a BIAS whose low 16 bits are
+    // zero: the excess-field constants absorb it, and the int8 / int16 fields
+    // are the low bits, which BIAS leaves untouched.
+    template <uint32_t BIAS = 0u>
     __device__ __forceinline__ void store(int lane, int c0, int c1, int c2, int c3,
                                           unsigned char* dst) const {
+        static_assert((BIAS & 0xFFFFu) == 0u, "bias must keep the low 16 bits");
         if (BITS == 5) {
             // excess-16 fields without masking: sum of c_i 32^i plus 16 * (1 + 32 + 1024 + 32768)
-            const uint32_t x = (uint32_t)(c0 + c1 * 32 + c2 * 1024 + c3 * 32768 + 541200);
+            constexpr uint32_t k5 = 541200u - BIAS * 33825u;
+            const uint32_t x = (uint32_t)c0 + (uint32_t)c1 * 32u + (uint32_t)c2 * 1024u +
+                               (uint32_t)c3 * 32768u + k5;
             const uint32_t x0 = __shfl_sync(kFull, x, src0);
             const uint32_t x1 = __shfl_sync(kFull, x, src0 + 1);
             const uint32_t x2 = __shfl_sync(kFull, x, src2);
@@ -175,7 +195,9 @@ struct Packer {
             if (lane < 20) reinterpret_cast<uint32_t*>(dst)[lane] = word;
         } else if (BITS == 4) {
             // excess-8 fields: sum of c_i 16^i plus 8 * (1 + 16 + 256 + 4096)
-            const uint32_t x = (uint32_t)(c0 + c1 * 16 + c2 * 256 + c3 * 4096 + 34952);
+            constexpr uint32_t k4 = 34952u - BIAS * 4369u;
+            const uint32_t x = (uint32_t)c0 + (uint32_t)c1 * 16u + (uint32_t)c2 * 256u +
+                               (uint32_t)c3 * 4096u + k4;
             const uint32_t xa = __shfl_sync(kFull, x, (2 * lane) & 31);
             const uint32_t xb = __shfl_sync(kFull, x, (2 * lane + 1) & 31);
             if (lane < 16) reinterpret_cast<uint32_t*>(dst)[lane] = xa | (xb << 16);

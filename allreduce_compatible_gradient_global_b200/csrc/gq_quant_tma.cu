@@ -5,9 +5,9 @@
 // ~20 instructions per element on Philox, rounding and packing.  Holding the
 // in-flight rows in registers (one float4 per worker per lane) caps the
 // resident warps; here a producer warp streams each worker's row segment of
-// a 1024-coordinate tile with one cp.async.bulk into a ring of STAGES tiles,
+// a 1024-coordinate tile with one cp.async.bulk into a ring of `stages` tiles,
 // and eight compute warps read their 128-coordinate block of every row from
-// shared memory.  The copies run ahead by STAGES - 1 tiles regardless of how
+// shared memory.  The copies run ahead by stages - 1 tiles regardless of how
 // long the compute takes.
 //
 // Synchronization: per stage a "full" mbarrier (one producer arrival plus the
@@ -27,6 +27,16 @@ constexpr int kTmaTile = 1024;  // coordinates per worker row per stage
 constexpr int kTmaComputeWarps = kTmaTile / 128;
 constexpr int kTmaThreads = (kTmaComputeWarps + 1) * 32;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Blocks per SM the register budget is cut for (two 3-stage rings of eight
+// rows fit one SM's shared memory), and whether W = 8 gets its own fully
+// unrolled instantiation.
+#ifndef GQ_TMA_MIN_BLOCKS
+#define GQ_TMA_MIN_BLOCKS 2
+#endif
+#ifndef GQ_TMA_SPECIALIZE_W8
+#define GQ_TMA_SPECIALIZE_W8 1
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -51,14 +61,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
+// One bounded try: the thread may be suspended (issuing nothing) until the
+// phase completes or about kSuspendHintNs pass, whichever comes first.
+constexpr uint32_t kSuspendHintNs = 100000u;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -92,23 +105,26 @@ __device__ __forceinline__ int quantize_tma(float v, float aq, const QuantArgs& 
     return quant_exp(v, aq, a.L, a.finest, a.inv_finest, word);
 }
 
-template <int LEVELS, int BITS, bool EF, int STAGES>
-__global__ void __launch_bounds__(kTmaThreads, 1)
-    quant_tma_kernel(const __grid_constant__ QuantArgs a) {
+// WT: the number of workers when known at compile time (the worker loop is
+// then fully unrolled and the Philox chains of all workers interleave), or 0.
+template <int LEVELS, int BITS, bool EF, int WT>
+__global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
+    quant_tma_kernel(const __grid_constant__ QuantArgs a, int stages) {
     extern __shared__ __align__(128) unsigned char smem[];
-    const int rows = EF ? 2 * a.W : a.W;  // g rows, then e rows
+    const int W = WT > 0 ? WT : a.W;
+    const int rows = EF ? 2 * W : W;  // g rows, then e rows
     float* buf = reinterpret_cast<float*>(smem);
     unsigned long long* bars = reinterpret_cast<unsigned long long*>(
-        smem + (size_t)STAGES * rows * kTmaTile * sizeof(float));
+        smem + (size_t)stages * rows * kTmaTile * sizeof(float));
     const uint32_t full0 = smem_addr(bars);
-    const uint32_t empty0 = smem_addr(bars + STAGES);
+    const uint32_t empty0 = smem_addr(bars + stages);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long ntiles = (a.d + kTmaTile - 1) / kTmaTile;
     const long long nblk = (a.d + 127) >> 7;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < stages; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, kTmaComputeWarps);
         }
@@ -119,35 +135,38 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     if (warp == kTmaComputeWarps) {
         // ---------------- producer: one lane issues every copy ----------------
         if (lane == 0) {
-            long long issued = 0;  // tiles whose copies were issued
+            // stage s of round `round` holds this CTA's tile number round * stages + s
+            int s = 0;
+            uint32_t round = 0;
+            long long issued = 0;
             bool ok = true;
             for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++issued) {
-                const int s = (int)(issued % STAGES);
-                if (issued >= STAGES) {
-                    const uint32_t par = (uint32_t)((issued / STAGES - 1) & 1);
-                    if (!mbar_wait_bounded(empty0 + 8 * s, par, a.hdr)) {
-                        ok = false;
-                        break;
-                    }
+                if (round > 0 && !mbar_wait_bounded(empty0 + 8 * s, (round - 1) & 1u, a.hdr)) {
+                    ok = false;
+                    break;
                 }
                 const long long j0 = t * kTmaTile;
                 const long long n = a.d - j0 < kTmaTile ? a.d - j0 : kTmaTile;
                 const uint32_t bytes = (uint32_t)(n * sizeof(float));
                 mbar_arrive_expect_tx(full0 + 8 * s, bytes * (uint32_t)rows);
                 for (int r = 0; r < rows; ++r) {
-                    const float* src = (r < a.W ? a.g + (long long)r * a.d
-                                                : a.e + (long long)(r - a.W) * a.d) + j0;
+                    const float* src = (r < W ? a.g + (long long)r * a.d
+                                              : a.e + (long long)(r - W) * a.d) + j0;
                     bulk_g2s(smem_addr(buf + ((size_t)s * rows + r) * kTmaTile), src, bytes,
                              full0 + 8 * s);
+                }
+                if (++s == stages) {
+                    s = 0;
+                    ++round;
                 }
             }
             // Drain: every issued stage must have landed before the block exits.
             // On the normal path the consumers already waited for all of them;
-            // after a timeout, wait (bounded) for the last STAGES issued tiles.
+            // after a timeout, wait (bounded) for the last `stages` issued tiles.
             if (!ok) {
-                const long long first = issued > STAGES ? issued - STAGES : 0;
+                const long long first = issued > stages ? issued - stages : 0;
                 for (long long k = first; k < issued; ++k)
-                    mbar_wait_bounded(full0 + 8 * (int)(k % STAGES), (uint32_t)((k / STAGES) & 1),
+                    mbar_wait_bounded(full0 + 8 * (int)(k % stages), (uint32_t)((k / stages) & 1),
                                       a.hdr);
             }
         }
@@ -169,62 +188,100 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
     Packer<BITS> pk;
     pk.init(lane);
-    long long k = 0;
-    for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
-        const int s = (int)(k % STAGES);
-        if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)((k / STAGES) & 1), a.hdr)) break;
+    int s = 0;
+    uint32_t phase = 0;
+    for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        if (!mbar_wait_bounded(full0 + 8 * s, phase, a.hdr)) break;
         const long long blk = t * kTmaComputeWarps + warp;
         if (blk < nblk) {
             const long long j0 = (blk << 7) + (lane << 2);
             const bool in = j0 < a.d;  // d % 4 == 0: all four or none
             const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
             const float* stage = buf + (size_t)s * rows * kTmaTile + warp * 128 + lane * 4;
-            int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-#pragma unroll 2
-            for (int w = 0; w < a.W; ++w) {
+            // uniform levels accumulate the biased patterns (code + kCodeBias)
+            uint32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+#pragma unroll
+            for (int w = 0; w < (WT > 0 ? WT : a.W); ++w) {
                 float4 v = in ? *reinterpret_cast<const float4*>(stage + (size_t)w * kTmaTile)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
                 if (EF && in) {
                     const float4 ev =
-                        *reinterpret_cast<const float4*>(stage + (size_t)(a.W + w) * kTmaTile);
+                        *reinterpret_cast<const float4*>(stage + (size_t)(W + w) * kTmaTile);
                     v = make_float4(__fadd_rn(v.x, ev.x), __fadd_rn(v.y, ev.y),
                                     __fadd_rn(v.z, ev.z), __fadd_rn(v.w, ev.w));
                 }
                 const uint4 rnd = philox10(philox_counter(q, a.step, (uint32_t)w), a.rk);
-                const int c0 = quantize_tma<LEVELS>(v.x, aq, a, rnd.x);
-                const int c1 = quantize_tma<LEVELS>(v.y, aq, a, rnd.y);
-                const int c2 = quantize_tma<LEVELS>(v.z, aq, a, rnd.z);
-                const int c3 = quantize_tma<LEVELS>(v.w, aq, a, rnd.w);
-                const int v0 = code_value<LEVELS>(c0), v1 = code_value<LEVELS>(c1);
-                const int v2 = code_value<LEVELS>(c2), v3 = code_value<LEVELS>(c3);
-                s0 += v0;
-                s1 += v1;
-                s2 += v2;
-                s3 += v3;
-                if (BITS != 0)
-                    pk.store(lane, c0, c1, c2, c3,
-                             a.codes + (long long)w * a.row_bytes + blk * (16 * BITS));
+                unsigned char* cdst = a.codes + (long long)w * a.row_bytes + blk * (16 * BITS);
+                float4 qv;  // the values Q(v) in units of c, as floats
+                if (LEVELS == 0) {
+                    const float t0 = quant_uniform_biased(v.x, aq, a.smax, rnd.x);
+                    const float t1 = quant_uniform_biased(v.y, aq, a.smax, rnd.y);
+                    const float t2 = quant_uniform_biased(v.z, aq, a.smax, rnd.z);
+                    const float t3 = quant_uniform_biased(v.w, aq, a.smax, rnd.w);
+                    const uint32_t b0 = __float_as_uint(t0), b1 = __float_as_uint(t1);
+                    const uint32_t b2 = __float_as_uint(t2), b3 = __float_as_uint(t3);
+                    s0 += b0;
+                    s1 += b1;
+                    s2 += b2;
+                    s3 += b3;
+                    if (BITS != 0) pk.template store<kCodeBias>(lane, b0, b1, b2, b3, cdst);
+                    if (EF) {
+                        qv.x = __fsub_rn(t0, 12582912.0f);
+                        qv.y = __fsub_rn(t1, 12582912.0f);
+                        qv.z = __fsub_rn(t2, 12582912.0f);
+                        qv.w = __fsub_rn(t3, 12582912.0f);
+                    }
+                } else {
+                    const int c0 = quantize_tma<LEVELS>(v.x, aq, a, rnd.x);
+                    const int c1 = quantize_tma<LEVELS>(v.y, aq, a, rnd.y);
+                    const int c2 = quantize_tma<LEVELS>(v.z, aq, a, rnd.z);
+                    const int c3 = quantize_tma<LEVELS>(v.w, aq, a, rnd.w);
+                    const int v0 = code_value<LEVELS>(c0), v1 = code_value<LEVELS>(c1);
+                    const int v2 = code_value<LEVELS>(c2), v3 = code_value<LEVELS>(c3);
+                    s0 += (uint32_t)v0;
+                    s1 += (uint32_t)v1;
+                    s2 += (uint32_t)v2;
+                    s3 += (uint32_t)v3;
+                    if (BITS != 0) pk.store(lane, c0, c1, c2, c3, cdst);
+                    if (EF) {
+                        qv.x = small_int_to_float(v0);
+                        qv.y = small_int_to_float(v1);
+                        qv.z = small_int_to_float(v2);
+                        qv.w = small_int_to_float(v3);
+                    }
+                }
                 if (EF && a.update_e && in) {
                     float4 en;
-                    en.x = __fsub_rn(v.x, __fmul_rn(small_int_to_float(v0), c));
-                    en.y = __fsub_rn(v.y, __fmul_rn(small_int_to_float(v1), c));
-                    en.z = __fsub_rn(v.z, __fmul_rn(small_int_to_float(v2), c));
-                    en.w = __fsub_rn(v.w, __fmul_rn(small_int_to_float(v3), c));
+                    en.x = __fsub_rn(v.x, __fmul_rn(qv.x, c));
+                    en.y = __fsub_rn(v.y, __fmul_rn(qv.y, c));
+                    en.z = __fsub_rn(v.z, __fmul_rn(qv.z, c));
+                    en.w = __fsub_rn(v.w, __fmul_rn(qv.w, c));
                     __stcs(reinterpret_cast<float4*>(a.e + (long long)w * a.d + j0), en);
                 }
             }
-            if (a.sum) store_sum(a.sum, a.wire, j0, a.d, s0, s1, s2, s3);
+            if (LEVELS == 0) {
+                const uint32_t off = (uint32_t)W * kCodeBias;
+                s0 -= off;
+                s1 -= off;
+                s2 -= off;
+                s3 -= off;
+            }
+            if (a.sum) store_sum(a.sum, a.wire, j0, a.d, (int)s0, (int)s1, (int)s2, (int)s3);
             if (a.out) {
                 float4 o;
-                o.x = decode_mean(s0, c, a.inv_w, a.w_pow2, a.W);
-                o.y = decode_mean(s1, c, a.inv_w, a.w_pow2, a.W);
-                o.z = decode_mean(s2, c, a.inv_w, a.w_pow2, a.W);
-                o.w = decode_mean(s3, c, a.inv_w, a.w_pow2, a.W);
+                o.x = decode_mean((int)s0, c, a.inv_w, a.w_pow2, W);
+                o.y = decode_mean((int)s1, c, a.inv_w, a.w_pow2, W);
+                o.z = decode_mean((int)s2, c, a.inv_w, a.w_pow2, W);
+                o.w = decode_mean((int)s3, c, a.inv_w, a.w_pow2, W);
                 store_out4(a.out, j0, a.d, o);
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
+        if (++s == stages) {
+            s = 0;
+            phase ^= 1u;
+        }
     }
 }
 
@@ -233,36 +290,42 @@ size_t tma_smem_bytes(int W, bool ef, int stages) {
     return (size_t)stages * rows * kTmaTile * sizeof(float) + 2 * stages * sizeof(unsigned long long);
 }
 
-template <int LEVELS, int BITS, bool EF, int STAGES>
-static cudaError_t launch_tma_inst(const QuantArgs& a, int grid, cudaStream_t st) {
-    auto kern = quant_tma_kernel<LEVELS, BITS, EF, STAGES>;
-    const size_t smem = tma_smem_bytes(a.W, EF, STAGES);
+template <int LEVELS, int BITS, bool EF, int WT>
+static cudaError_t launch_tma_inst(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
+    auto kern = quant_tma_kernel<LEVELS, BITS, EF, WT>;
+    const size_t smem = tma_smem_bytes(a.W, EF, stages);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTmaThreads, smem, st>>>(a);
+    kern<<<grid, kTmaThreads, smem, st>>>(a, stages);
     return cudaGetLastError();
 }
 
-template <int LEVELS, bool EF, int STAGES>
-static cudaError_t launch_tma_bits(const QuantArgs& a, int bits, int grid, cudaStream_t st) {
+template <int LEVELS, int BITS, bool EF>
+static cudaError_t launch_tma_w(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
+    if (GQ_TMA_SPECIALIZE_W8 && a.W == 8)
+        return launch_tma_inst<LEVELS, BITS, EF, 8>(a, stages, grid, st);
+    return launch_tma_inst<LEVELS, BITS, EF, 0>(a, stages, grid, st);
+}
+
+template <int LEVELS, bool EF>
+static cudaError_t launch_tma_bits(const QuantArgs& a, int bits, int stages, int grid,
+                                   cudaStream_t st) {
     switch (bits) {
-        case 0: return launch_tma_inst<LEVELS, 0, EF, STAGES>(a, grid, st);
-        case 4: return launch_tma_inst<LEVELS, 4, EF, STAGES>(a, grid, st);
-        case 5: return launch_tma_inst<LEVELS, 5, EF, STAGES>(a, grid, st);
-        case 8: return launch_tma_inst<LEVELS, 8, EF, STAGES>(a, grid, st);
-        default: return launch_tma_inst<LEVELS, 16, EF, STAGES>(a, grid, st);
+        case 0: return launch_tma_w<LEVELS, 0, EF>(a, stages, grid, st);
+        case 4: return launch_tma_w<LEVELS, 4, EF>(a, stages, grid, st);
+        case 5: return launch_tma_w<LEVELS, 5, EF>(a, stages, grid, st);
+        case 8: return launch_tma_w<LEVELS, 8, EF>(a, stages, grid, st);
+        default: return launch_tma_w<LEVELS, 16, EF>(a, stages, grid, st);
     }
 }
 
 cudaError_t launch_quant_tma(const QuantArgs& a, int levels, int bits, bool ef, int stages,
                              int grid, cudaStream_t st) {
-#define GQ_TMA(LV, E)                                                            \
-    (stages == 2 ? launch_tma_bits<LV, E, 2>(a, bits, grid, st)                  \
-                 : stages == 3 ? launch_tma_bits<LV, E, 3>(a, bits, grid, st)    \
-                               : launch_tma_bits<LV, E, 4>(a, bits, grid, st))
-    if (levels == 0) return ef ? GQ_TMA(0, true) : GQ_TMA(0, false);
-    return ef ? GQ_TMA(1, true) : GQ_TMA(1, false);
-#undef GQ_TMA
+    if (levels == 0)
+        return ef ? launch_tma_bits<0, true>(a, bits, stages, grid, st)
+                  : launch_tma_bits<0, false>(a, bits, stages, grid, st);
+    return ef ? launch_tma_bits<1, true>(a, bits, stages, grid, st)
+              : launch_tma_bits<1, false>(a, bits, stages, grid, st);
 }
 
 }  // namespace gq
