@@ -84,8 +84,11 @@ int check_sizes(int W, long long d) {
     return GQ_OK;
 }
 
-int norm_blocks_per_worker(int W, long long d) {
-    const long long want = ((long long)sm_count() * kBlocksPerSm + W - 1) / W;
+// Blocks per worker of the norm pass: one full wave of resident blocks over
+// all workers, so that no block starts late and leaves a tail.
+int norm_blocks_per_worker(int W, long long d, int kind, bool has_e) {
+    const long long resident = (long long)sm_count() * norm_resident_blocks(kind, has_e, d % 4 == 0);
+    const long long want = resident / W > 0 ? resident / W : 1;
     const long long useful = (d + (long long)kThreads * 16 - 1) / ((long long)kThreads * 16);
     long long nb = want < useful ? want : useful;
     if (nb < 1) nb = 1;
@@ -257,7 +260,7 @@ GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long lo
     a.e = cfg->ef ? e_dev : nullptr;
     a.d = d;
     a.W = W;
-    a.nb = norm_blocks_per_worker(W, d);
+    a.nb = norm_blocks_per_worker(W, d, cfg->scale_kind, cfg->ef != 0);
     a.kind = cfg->scale_kind;
     a.scale = scale_dev;
     a.norms = norms_dev;

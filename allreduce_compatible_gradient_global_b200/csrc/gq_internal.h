@@ -109,6 +109,8 @@ struct LogqArgs {
 
 // Launchers (return the cudaGetLastError() of the launch).
 cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st);
+// Resident blocks per SM of the norm kernel instantiation for (kind, e?, vec).
+int norm_resident_blocks(int kind, bool has_e, bool vec);
 cudaError_t launch_quant(const QuantArgs& a, int levels, int bits, bool ef, bool vec, int grid,
                          cudaStream_t st);
 cudaError_t launch_aggregate(const AggArgs& a, int levels, int bits, int grid, cudaStream_t st);

@@ -103,7 +103,7 @@ __device__ __forceinline__ void norm_accum4(float4 x, float4 ex, float& s16, uns
 }
 
 template <int KIND, bool HAS_E, bool VEC>
-__global__ void __launch_bounds__(kThreads) norm_kernel(const __grid_constant__ NormArgs a) {
+__global__ void __launch_bounds__(kThreads, 8) norm_kernel(const __grid_constant__ NormArgs a) {
     const int w = blockIdx.y;
     const int b = blockIdx.x;
     const float* gw = a.g + (long long)w * a.d;
@@ -231,6 +231,27 @@ __global__ void __launch_bounds__(kThreads) norm_kernel(const __grid_constant__ 
         if (!(S <= FLT_MAX)) atomicOr(&a.hdr->flags, kFlagNonfiniteScale);
         a.hdr->counter = 0u;  // ready for the next call (stream order)
     }
+}
+
+int norm_resident_blocks(int kind, bool has_e, bool vec) {
+    // resident blocks per SM of the instantiation that will run (cached)
+    static int cache[2][2][2] = {};
+    int& c = cache[kind != 0][has_e][vec];
+    if (c == 0) {
+        const void* fn;
+        if (kind == 0) {
+            fn = has_e ? (vec ? (const void*)norm_kernel<0, true, true> : (const void*)norm_kernel<0, true, false>)
+                       : (vec ? (const void*)norm_kernel<0, false, true> : (const void*)norm_kernel<0, false, false>);
+        } else {
+            fn = has_e ? (vec ? (const void*)norm_kernel<1, true, true> : (const void*)norm_kernel<1, true, false>)
+                       : (vec ? (const void*)norm_kernel<1, false, true> : (const void*)norm_kernel<1, false, false>);
+        }
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, 0) != cudaSuccess || n < 1)
+            n = 1;
+        c = n;
+    }
+    return c;
 }
 
 cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st) {

@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     }
     Packer<BITS> pk;
     pk.init(lane);
+    const long long row_bytes = a.row_bytes;
     int s = 0;
     uint32_t phase = 0;
     for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -198,6 +199,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
             const bool in = j0 < a.d;  // d % 4 == 0: all four or none
             const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
             const float* stage = buf + (size_t)s * rows * kTmaTile + warp * 128 + lane * 4;
+            unsigned char* codes_blk = a.codes + blk * (16 * BITS);
             // uniform levels accumulate the biased patterns (code + kCodeBias)
             uint32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
 #pragma unroll
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                                     __fadd_rn(v.z, ev.z), __fadd_rn(v.w, ev.w));
                 }
                 const uint4 rnd = philox10(philox_counter(q, a.step, (uint32_t)w), a.rk);
-                unsigned char* cdst = a.codes + (long long)w * a.row_bytes + blk * (16 * BITS);
+                unsigned char* cdst = codes_blk + (long long)w * row_bytes;
                 float4 qv;  // the values Q(v) in units of c, as floats
                 if (LEVELS == 0) {
                     const float t0 = quant_uniform_biased(v.x, aq, a.smax, rnd.x);
