@@ -93,6 +93,7 @@ def _load():
         "gq_workspace_bytes": ([CP, I, LL, ctypes.POINTER(ctypes.c_size_t)], I),
         "gq_workspace_init": ([P, ctypes.c_size_t, P], I),
         "gq_get_device_status": ([P, P], I),
+        "gq_selftest_wait_timeout": ([P, ctypes.c_uint, P], I),
         "gq_global_norm": ([P, P, I, LL, CP, P, P, P, P], I),
         "gq_global_norm_noalloc": ([P, P, I, LL, CP, P, P, P], I),
         "gq_quantize_pack": ([P, P, I, LL, CP, P, P, P, P], I),
@@ -199,6 +200,14 @@ def gq_get_device_status(ws, stream=None) -> int:
     if rc not in (GQ_OK, GQ_ERR_NONFINITE):
         raise GQError(rc, "gq_get_device_status")
     return rc
+
+
+def gq_selftest_wait_timeout(ws, limit_ms=50, stream=None):
+    """Make one bounded device wait expire on purpose; returns the status that
+    gq_get_device_status then reports (GQ_ERR_TIMEOUT when detection works)."""
+    _check(lib().gq_selftest_wait_timeout(_ptr(ws), int(limit_ms), _stream(stream)),
+           "gq_selftest_wait_timeout")
+    return lib().gq_get_device_status(_ptr(ws), _stream(stream))
 
 
 # ------------------------------------------------------------------ the path

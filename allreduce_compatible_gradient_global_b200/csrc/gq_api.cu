@@ -222,7 +222,7 @@ GQ_API int gq_packed_row_bytes(const gq_config* cfg, long long d, long long* byt
 GQ_API int gq_workspace_bytes(const gq_config* cfg, int W, long long d, size_t* bytes) {
     (void)cfg;
     if (!bytes || W < 1 || d < 0) return GQ_ERR_ARG;
-    *bytes = (size_t)kWorkspaceHeader + (size_t)W * kMaxNormBlocks * sizeof(unsigned long long);
+    *bytes = (size_t)kWorkspaceHeader + (size_t)W * kMaxNormBlocks * 2 * sizeof(unsigned long long);
     return GQ_OK;
 }
 
@@ -242,6 +242,14 @@ GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream) {
     if (flags == 0) return GQ_OK;
     if (cudaMemset(&header_of(ws_dev)->flags, 0, sizeof(flags)) != cudaSuccess) return GQ_ERR_CUDA;
     return (flags & kFlagPipelineTimeout) ? GQ_ERR_TIMEOUT : GQ_ERR_NONFINITE;
+}
+
+GQ_API int gq_selftest_wait_timeout(void* ws_dev, unsigned int limit_ms, cudaStream_t stream) {
+    if (!ws_dev || limit_ms < 1 || limit_ms > 10000) return GQ_ERR_ARG;
+    if (!aligned16(ws_dev)) return GQ_ERR_ALIGN;
+    return cuda_status(launch_wait_timeout_selftest(header_of(ws_dev),
+                                                    (unsigned long long)limit_ms * 1000000ull,
+                                                    stream));
 }
 
 GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long long d,

@@ -70,7 +70,7 @@ __device__ __forceinline__ int with_sign_of(int k, float v) {
     return (k ^ sgn) - sgn;
 }
 
-// Uniform levels {0, +-1/s, ..., +-1}: a = fl(s/S), r = fl(v a) clamped to
+// Uniform levels {0, +-1/s, ..., +-1}: a = s/S rounded down, r = fl(v a) clamped to
 // [-s, s] (fminf also maps a NaN product to s), code = floor(r + u).  The
 // signed value is rounded directly: each coordinate gets the same two
 // outcomes with the same probabilities as sign(v) * floor(|r| + u), and no
@@ -96,6 +96,14 @@ __device__ __forceinline__ float quant_uniform_biased(float v, float a, float sm
     return __fadd_rd(t1, 12582911.0f);
 }
 
+// Without the clamp, for a scale S that bounds every input (|v| <= S, which
+// gq_global_norm guarantees) and a = s/S rounded down: then |v a| <= s
+// exactly, so |fl(v a)| <= s and the clamp could never act.
+__device__ __forceinline__ float quant_uniform_biased_unclamped(float v, float a, uint32_t word) {
+    const float t1 = __fadd_rd(__fmul_rn(v, a), unit_plus_u(word));
+    return __fadd_rd(t1, 12582911.0f);
+}
+
 // Exponential levels {0, 2^-(L-1), ..., 1/2, 1}: a = fl(1/S), r = min(fl(|v| a), 1).
 // For r >= 2^-(L-1), r = (1 + m 2^-23) 2^E with m the mantissa field: the
 // bracket is [2^E, 2^(E+1)], the lower level has index L + E, and the
@@ -116,6 +124,34 @@ __device__ __forceinline__ int quant_exp(float v, float a, int L, float finest, 
         idx = __fadd_rd(p, __uint_as_float(0x3F800000u | f)) >= 2.0f ? 1 : 0;
     }
     return with_sign_of(idx, v);
+}
+
+// Exponential levels without branches, for a = 1/S rounded down (so |r| <= 1
+// for every |v| <= S).  The signed level value Q (0, +-2^-(L-1), ..., +-1) is
+// built in the bit pattern of r: for |r| >= 2^-(L-1), adding the 23 random
+// bits f to the pattern carries out of the mantissa exactly when
+// m + f >= 2^23 -- the round-up event -- and bumps the exponent to the upper
+// level; masking to sign and exponent leaves +-2^E or +-2^(E+1).  Below the
+// finest level, r' = r + sign * 2^-(L-1) rounded toward zero has mantissa
+// floor(p 2^23) with p = |r| 2^(L-1), the same carry decides p + u >= 1, and
+// subtracting the added level leaves 0 or +-2^-(L-1).
+__device__ __forceinline__ float quant_exp_level(float v, float a, float finest, uint32_t word) {
+    const float r = __fmul_rn(v, a);
+    const uint32_t f = word & 0x007FFFFFu;
+    const float fin_s = __uint_as_float(__float_as_uint(finest) | (__float_as_uint(r) & 0x80000000u));
+    const bool small = fabsf(r) < finest;
+    const float x = small ? __fadd_rz(r, fin_s) : r;
+    const float q = __uint_as_float((__float_as_uint(x) + f) & 0xFF800000u);
+    return small ? __fsub_rn(q, fin_s) : q;
+}
+
+// The signed level index (the code) of a level value Q from its exponent:
+// Q = +-2^E has index L + E; Q = 0 has index 0.
+__device__ __forceinline__ int exp_code_of_level(float q, int L) {
+    const uint32_t qb = __float_as_uint(q);
+    const int idx = max((int)((qb >> 23) & 0xFFu) - (127 - L), 0);
+    const int sgn = (int)qb >> 31;
+    return (idx ^ sgn) - sgn;
 }
 
 // Value a code adds to the sum: the code itself (uniform levels) or

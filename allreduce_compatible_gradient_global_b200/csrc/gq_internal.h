@@ -11,7 +11,7 @@
 namespace gq {
 
 constexpr int kThreads = 256;          // threads per block of every streaming kernel
-constexpr int kMaxNormBlocks = 2048;   // per-worker partial slots in the workspace
+constexpr int kMaxNormBlocks = 2048;   // norm blocks per worker (two 8-byte workspace slots each)
 constexpr int kWorkspaceHeader = 256;  // flag word, ticket counter, padding
 
 // Workspace header words.
@@ -121,6 +121,9 @@ cudaError_t launch_dequant(const DequantArgs& a, int levels, int bits, bool vec,
 size_t tma_smem_bytes(int W, bool ef, int stages);
 cudaError_t launch_quant_tma(const QuantArgs& a, int levels, int bits, bool ef, int stages,
                              int grid, cudaStream_t st);
+// Bounded-wait self-test (raises kFlagPipelineTimeout after limit_ns).
+cudaError_t launch_wait_timeout_selftest(WsHeader* hdr, unsigned long long limit_ns,
+                                         cudaStream_t st);
 cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st);
 cudaError_t launch_logq_decode(const LogqArgs& a, cudaStream_t st);
 

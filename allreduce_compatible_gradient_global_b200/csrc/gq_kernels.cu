@@ -62,10 +62,10 @@ __device__ __forceinline__ void scale_constants(float S, float smax, float fines
                                                 float& c) {
     const bool ok = S > 0.f && S <= FLT_MAX;
     if (LEVELS == 0) {
-        a = ok ? __fdiv_rn(smax, S) : 0.f;
+        a = ok ? __fdiv_rd(smax, S) : 0.f;  // s/S rounded down: |v| a <= s when |v| <= S
         c = __fdiv_rn(S, smax);
     } else {
-        a = ok ? __fdiv_rn(1.0f, S) : 0.f;
+        a = ok ? __fdiv_rd(1.0f, S) : 0.f;  // 1/S rounded down: |v| a <= 1 when |v| <= S
         c = __fmul_rn(S, finest);
     }
 }
@@ -84,6 +84,10 @@ __device__ __forceinline__ unsigned warp_max_u(unsigned x) {
     return x;
 }
 
+// Both kinds track max |v|: it is the scale of the max-abs kind, and for the
+// L2 kind it is a floor the rounded norm must not fall below (see the end of
+// norm_kernel).  |v| as unsigned bits is order-preserving for non-negative
+// floats, and any NaN compares above +Inf, so a NaN input surfaces in the max.
 template <int KIND, bool HAS_E>
 __device__ __forceinline__ void norm_accum4(float4 x, float4 ex, float& s16, unsigned& mx) {
     if (HAS_E) x = add4(x, ex);
@@ -92,14 +96,11 @@ __device__ __forceinline__ void norm_accum4(float4 x, float4 ex, float& s16, uns
         s16 = __fmaf_rn(x.y, x.y, s16);
         s16 = __fmaf_rn(x.z, x.z, s16);
         s16 = __fmaf_rn(x.w, x.w, s16);
-    } else {
-        // |v| as unsigned bits: order-preserving for non-negative floats, and
-        // any NaN compares above +Inf, so a NaN input surfaces in the max.
-        mx = max(mx, __float_as_uint(fabsf(x.x)));
-        mx = max(mx, __float_as_uint(fabsf(x.y)));
-        mx = max(mx, __float_as_uint(fabsf(x.z)));
-        mx = max(mx, __float_as_uint(fabsf(x.w)));
     }
+    mx = max(mx, __float_as_uint(fabsf(x.x)));
+    mx = max(mx, __float_as_uint(fabsf(x.y)));
+    mx = max(mx, __float_as_uint(fabsf(x.z)));
+    mx = max(mx, __float_as_uint(fabsf(x.w)));
 }
 
 template <int KIND, bool HAS_E, bool VEC>
@@ -164,23 +165,20 @@ __global__ void __launch_bounds__(kThreads, 8) norm_kernel(const __grid_constant
     if (KIND == 0) {
         acc = warp_sum_d(acc);
         if (lane == 0) red_d[warp] = acc;
-    } else {
-        mx = warp_max_u(mx);
-        if (lane == 0) red_u[warp] = mx;
     }
+    mx = warp_max_u(mx);
+    if (lane == 0) red_u[warp] = mx;
     __syncthreads();
     if (threadIdx.x == 0) {
-        unsigned long long part;
-        if (KIND == 0) {
-            double t = 0.0;
+        double t = 0.0;
+        unsigned m = 0u;
+        if (KIND == 0)
             for (int k = 0; k < kThreads / 32; ++k) t += red_d[k];
-            part = (unsigned long long)__double_as_longlong(t);
-        } else {
-            unsigned t = 0u;
-            for (int k = 0; k < kThreads / 32; ++k) t = max(t, red_u[k]);
-            part = t;
-        }
-        a.partials[(long long)w * a.nb + b] = part;
+        for (int k = 0; k < kThreads / 32; ++k) m = max(m, red_u[k]);
+        // two slots per block: the sum of squares, then max |v|
+        unsigned long long* slot = a.partials + 2 * ((long long)w * a.nb + b);
+        slot[0] = (unsigned long long)__double_as_longlong(t);
+        slot[1] = m;
         __threadfence();
         const unsigned total = (unsigned)a.nb * (unsigned)a.W;
         const unsigned ticket = atomicAdd(&a.hdr->counter, 1u);
@@ -195,22 +193,30 @@ __global__ void __launch_bounds__(kThreads, 8) norm_kernel(const __grid_constant
     double best = 0.0;
     bool saw_nan = false;
     for (int ww = warp; ww < a.W; ww += kThreads / 32) {
-        const unsigned long long* pw = a.partials + (long long)ww * a.nb;
-        double nrm;
+        const unsigned long long* pw = a.partials + 2 * (long long)ww * a.nb;
+        unsigned m = 0u;
+        double t = 0.0;
+        for (int k = lane; k < a.nb; k += 32) {
+            if (KIND == 0) t += __longlong_as_double((long long)__ldcg(pw + 2 * k));
+            m = max(m, (unsigned)__ldcg(pw + 2 * k + 1));
+        }
+        m = warp_max_u(m);
+        const double mxv = (double)__uint_as_float(m);
+        double nrm, cand;
         if (KIND == 0) {
-            double t = 0.0;
-            for (int k = lane; k < a.nb; k += 32) t += __longlong_as_double((long long)__ldcg(pw + k));
-            t = warp_sum_d(t);
-            nrm = sqrt(t);
+            nrm = sqrt(warp_sum_d(t));
+            // In exact arithmetic ||v_w|| >= max|v_w|; the fp32 partial sums
+            // can round the norm just below a dominant entry, so the scale
+            // never takes a value below max|v|.  Then S >= |v| for every
+            // input, which the fused pass relies on to need no clamp.
+            cand = nrm != nrm ? nrm : fmax(nrm, mxv);
         } else {
-            unsigned t = 0u;
-            for (int k = lane; k < a.nb; k += 32) t = max(t, (unsigned)__ldcg(pw + k));
-            t = warp_max_u(t);
-            nrm = (double)__uint_as_float(t);
+            nrm = mxv;
+            cand = mxv;
         }
         if (lane == 0 && a.norms) a.norms[ww] = nrm;
-        if (nrm != nrm) saw_nan = true;
-        else best = fmax(best, nrm);
+        if (cand != cand || mxv != mxv) saw_nan = true;
+        else best = fmax(best, cand);
     }
     __shared__ double wbest[kThreads / 32];
     __shared__ int wnan[kThreads / 32];

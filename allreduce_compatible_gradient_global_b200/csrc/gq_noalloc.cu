@@ -61,7 +61,7 @@ int noalloc_blocks_per_worker(int W, long long d) {
     long long nb = ((long long)sms * 8 + W - 1) / W;
     const long long useful = (d + (long long)gq::kThreads * 16 - 1) / ((long long)gq::kThreads * 16);
     if (useful < nb) nb = useful;
-    if (nb > kNoallocSlots / W) nb = kNoallocSlots / W;
+    if (nb > kNoallocSlots / (2 * W)) nb = kNoallocSlots / (2 * W);  // two slots per block
     if (nb < 1) nb = 1;
     return (int)nb;
 }

@@ -77,17 +77,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete, for at most
-// kWaitLimitNs; false (and the flag raised) if it never did.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, WsHeader* hdr) {
+// limit_ns; false (and the flag raised) if it never did.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, WsHeader* hdr,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             atomicOr(&hdr->flags, kFlagPipelineTimeout);
             return false;
         }
     }
     return true;
+}
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// will ever complete (the first phase of a barrier expecting one arrival that
+// never comes), gives up after limit_ns and raises the timeout flag, exactly
+// as a stalled pipeline would.  Nothing faults and the context stays usable.
+__global__ void wait_timeout_selftest_kernel(WsHeader* hdr, unsigned long long limit_ns) {
+    __shared__ __align__(8) unsigned long long bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_addr(&bar);
+    mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait_bounded(b, 0u, hdr, limit_ns);
+}
+
+cudaError_t launch_wait_timeout_selftest(WsHeader* hdr, unsigned long long limit_ns,
+                                         cudaStream_t st) {
+    wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(hdr, limit_ns);
+    return cudaGetLastError();
 }
 
 // One bulk copy global -> shared (no multicast), completing on `bar`.
@@ -97,12 +117,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
         : "memory");
-}
-
-template <int LEVELS>
-__device__ __forceinline__ int quantize_tma(float v, float aq, const QuantArgs& a, uint32_t word) {
-    if (LEVELS == 0) return quant_uniform(v, aq, a.smax, word);
-    return quant_exp(v, aq, a.L, a.finest, a.inv_finest, word);
 }
 
 // WT: the number of workers when known at compile time (the worker loop is
@@ -179,10 +193,10 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
         const float S = __ldg(a.scale);
         const bool okS = S > 0.f && S <= FLT_MAX;
         if (LEVELS == 0) {
-            aq = okS ? __fdiv_rn(a.smax, S) : 0.f;
+            aq = okS ? __fdiv_rd(a.smax, S) : 0.f;  // |v| aq <= s for every |v| <= S
             c = __fdiv_rn(S, a.smax);
         } else {
-            aq = okS ? __fdiv_rn(1.0f, S) : 0.f;
+            aq = okS ? __fdiv_rd(1.0f, S) : 0.f;  // |v| aq <= 1 for every |v| <= S
             c = __fmul_rn(S, a.finest);
         }
     }
@@ -200,8 +214,11 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
             const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
             const float* stage = buf + (size_t)s * rows * kTmaTile + warp * 128 + lane * 4;
             unsigned char* codes_blk = a.codes + blk * (16 * BITS);
-            // uniform levels accumulate the biased patterns (code + kCodeBias)
+            // uniform levels accumulate the biased patterns (code + kCodeBias);
+            // exponential levels accumulate the level values as floats (exact:
+            // multiples of the finest level with fewer than 24 bits)
             uint32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+            float f0 = 0.f, f1 = 0.f, f2 = 0.f, f3 = 0.f;
 #pragma unroll
             for (int w = 0; w < (WT > 0 ? WT : a.W); ++w) {
                 float4 v = in ? *reinterpret_cast<const float4*>(stage + (size_t)w * kTmaTile)
@@ -216,10 +233,10 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 unsigned char* cdst = codes_blk + (long long)w * row_bytes;
                 float4 qv;  // the values Q(v) in units of c, as floats
                 if (LEVELS == 0) {
-                    const float t0 = quant_uniform_biased(v.x, aq, a.smax, rnd.x);
-                    const float t1 = quant_uniform_biased(v.y, aq, a.smax, rnd.y);
-                    const float t2 = quant_uniform_biased(v.z, aq, a.smax, rnd.z);
-                    const float t3 = quant_uniform_biased(v.w, aq, a.smax, rnd.w);
+                    const float t0 = quant_uniform_biased_unclamped(v.x, aq, rnd.x);
+                    const float t1 = quant_uniform_biased_unclamped(v.y, aq, rnd.y);
+                    const float t2 = quant_uniform_biased_unclamped(v.z, aq, rnd.z);
+                    const float t3 = quant_uniform_biased_unclamped(v.w, aq, rnd.w);
                     const uint32_t b0 = __float_as_uint(t0), b1 = __float_as_uint(t1);
                     const uint32_t b2 = __float_as_uint(t2), b3 = __float_as_uint(t3);
                     s0 += b0;
@@ -234,22 +251,22 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                         qv.w = __fsub_rn(t3, 12582912.0f);
                     }
                 } else {
-                    const int c0 = quantize_tma<LEVELS>(v.x, aq, a, rnd.x);
-                    const int c1 = quantize_tma<LEVELS>(v.y, aq, a, rnd.y);
-                    const int c2 = quantize_tma<LEVELS>(v.z, aq, a, rnd.z);
-                    const int c3 = quantize_tma<LEVELS>(v.w, aq, a, rnd.w);
-                    const int v0 = code_value<LEVELS>(c0), v1 = code_value<LEVELS>(c1);
-                    const int v2 = code_value<LEVELS>(c2), v3 = code_value<LEVELS>(c3);
-                    s0 += (uint32_t)v0;
-                    s1 += (uint32_t)v1;
-                    s2 += (uint32_t)v2;
-                    s3 += (uint32_t)v3;
-                    if (BITS != 0) pk.store(lane, c0, c1, c2, c3, cdst);
-                    if (EF) {
-                        qv.x = small_int_to_float(v0);
-                        qv.y = small_int_to_float(v1);
-                        qv.z = small_int_to_float(v2);
-                        qv.w = small_int_to_float(v3);
+                    const float q0 = quant_exp_level(v.x, aq, a.finest, rnd.x);
+                    const float q1 = quant_exp_level(v.y, aq, a.finest, rnd.y);
+                    const float q2 = quant_exp_level(v.z, aq, a.finest, rnd.z);
+                    const float q3 = quant_exp_level(v.w, aq, a.finest, rnd.w);
+                    f0 = __fadd_rn(f0, q0);
+                    f1 = __fadd_rn(f1, q1);
+                    f2 = __fadd_rn(f2, q2);
+                    f3 = __fadd_rn(f3, q3);
+                    if (BITS != 0)
+                        pk.store(lane, exp_code_of_level(q0, a.L), exp_code_of_level(q1, a.L),
+                                 exp_code_of_level(q2, a.L), exp_code_of_level(q3, a.L), cdst);
+                    if (EF) {  // value in units of the finest level (exact)
+                        qv.x = __fmul_rn(q0, a.inv_finest);
+                        qv.y = __fmul_rn(q1, a.inv_finest);
+                        qv.z = __fmul_rn(q2, a.inv_finest);
+                        qv.w = __fmul_rn(q3, a.inv_finest);
                     }
                 }
                 if (EF && a.update_e && in) {
@@ -267,6 +284,11 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 s1 -= off;
                 s2 -= off;
                 s3 -= off;
+            } else {  // level-value sums to integer units of the finest level
+                s0 = (uint32_t)__float2int_rn(__fmul_rn(f0, a.inv_finest));
+                s1 = (uint32_t)__float2int_rn(__fmul_rn(f1, a.inv_finest));
+                s2 = (uint32_t)__float2int_rn(__fmul_rn(f2, a.inv_finest));
+                s3 = (uint32_t)__float2int_rn(__fmul_rn(f3, a.inv_finest));
             }
             if (a.sum) store_sum(a.sum, a.wire, j0, a.d, (int)s0, (int)s1, (int)s2, (int)s3);
             if (a.out) {

@@ -42,7 +42,8 @@ DEFAULT_WORKLOAD = "resnet50_t3_w8"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "quant_kernel_traffic.json")
-KERNEL_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_kernels.cu",
+KERNEL_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_quant_tma.cu",
+                  "allreduce_compatible_gradient_global_b200/csrc/gq_kernels.cu",
                   "allreduce_compatible_gradient_global_b200/csrc/gq_device.cuh",
                   "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h"]
 
@@ -168,6 +169,20 @@ def algorithmic_bytes(gq, cfg, W, d):
     return p1, p2
 
 
+def job_time_ms(elapsed_ms, world, device):
+    """The job's time: the max over ranks of each rank's device-timed elapsed ms."""
+    if world == 1:
+        return float(elapsed_ms)
+    t = torch.tensor([float(elapsed_ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_rank_step, steps, job_ms, world):
+    """Whole-job throughput: every rank's bytes over the job's (max) time."""
+    return world * bytes_per_rank_step * steps / (job_ms * 1e-3) / 1e9
+
+
 def run_ours(args, rank, world, local_rank):
     import allreduce_compatible_gradient_global_b200 as gq
     torch.cuda.set_device(local_rank)
@@ -211,16 +226,12 @@ def run_ours(args, rank, world, local_rank):
     sampler.stop()
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
+    elapsed_ms = job_time_ms(t0.elapsed_time(t1), world, dev)
     norm_ms = [e[0].elapsed_time(e[1]) for e in evs]
     quant_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
     ms_per_step = elapsed_ms / K
     grad_bytes = 4 * W * d
-    value = world * grad_bytes * K / (elapsed_ms * 1e-3) / 1e9
+    value = job_gbs(grad_bytes, K, elapsed_ms, world)
 
     # roofline of the dominant kernel (pass 2)
     p1, p2 = algorithmic_bytes(gq, cfg, W, d)
@@ -229,7 +240,8 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = measured_hbm_peak()
     achieved = p2 / (q_avg * 1e-3) / 1e9
     traffic = recorded_traffic(args.workload)
-    roofline = {"bound": "hbm", "kernel": "quant_kernel (gq_quantize_aggregate)",
+    roofline = {"bound": "hbm", "kernel": "fused pass of gq_quantize_aggregate "
+                                          "(quant_tma_kernel when d % 4 == 0 and the rows fit)",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} (hbm_gbs)",
                 "traffic": traffic, "algorithmic_bytes": p2,
@@ -286,12 +298,8 @@ def run_e2e(gq, args, cfg, g, buf, stream, world, dev):
                               out_host, scale_host, buf.ws, stream)
     t1.record(stream)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    val = world * 4 * W * d * K / (ms * 1e-3) / 1e9
+    ms = job_time_ms(t0.elapsed_time(t1), world, dev)
+    val = job_gbs(4 * W * d, K, ms, world)
     del g_host, g_dev
     return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
             "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4),
@@ -348,6 +356,107 @@ def run_reference(args):
                      "d2h_bytes_per_step": 0})
 
 
+def time_step_pair(gq, g, e, cfg, buf, K, warmup, stream):
+    """Median per-kernel and mean step times (ms) of norm + fused pass."""
+    for i in range(warmup):
+        cfg.step = i
+        gq.gq_global_norm(g, e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws, stream)
+        gq.gq_quantize_aggregate(g, e, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws, stream)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(K):
+        cfg.step = warmup + i
+        evs[i][0].record(stream)
+        gq.gq_global_norm(g, e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws, stream)
+        evs[i][1].record(stream)
+        gq.gq_quantize_aggregate(g, e, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws, stream)
+        evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    if gq.gq_get_device_status(buf.ws, stream) != gq.GQ_OK:
+        raise RuntimeError("device flag raised during the sweep")
+    n = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    q = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    step = sum(e[0].elapsed_time(e[2]) for e in evs) / K
+    return n, q, step
+
+
+def run_sweep(args):
+    """Step throughput over d = 2^16 ... 2^30 at W = 8 (uniform s = 15, 5-bit
+    codes, int8 sums, L2 scale), error feedback off and on.  Below ~2^22 the
+    second read can hit L2; the fraction is reported but not targeted there."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = measured_hbm_peak()
+    rows = []
+    W = 8
+    for ef in (False, True):
+        for lg in range(16, 31, 2):
+            d = 1 << lg
+            cfg = gq.GQConfig(levels="uniform", s=15, bits=5, wire="int8", scale_kind="l2", ef=ef,
+                              seed=0x5EED)
+            g = synthetic.make_gradients(W, d, "normal", seed=lg, device="cuda")
+            buf = gq.StepBuffers(cfg, W, d)
+            K = max(20, min(400, int(2e9 // (4 * W * d))))
+            n_ms, q_ms, step_ms = time_step_pair(gq, g, buf.e, cfg, buf, K, 5, stream)
+            p1, p2 = algorithmic_bytes(gq, cfg, W, d)
+            rows.append({"d": d, "log2_d": lg, "ef": ef, "steps": K,
+                         "step_ms": round(step_ms, 5), "norm_ms": round(n_ms, 5),
+                         "quant_ms": round(q_ms, 5),
+                         "grad_gbs": round(4 * W * d / (step_ms * 1e-3) / 1e9, 1),
+                         "step_frac": round((p1 + p2) / (step_ms * 1e-3) / 1e9 / peak, 4),
+                         "quant_frac": round(p2 / (q_ms * 1e-3) / 1e9 / peak, 4)})
+            del g, buf
+            torch.cuda.empty_cache()
+    return {"metric": METRIC, "mode": "sweep", "unit": "GB/s", "peak": peak,
+            "peak_source": peak_kind, "W": W, "config": "uniform s=15, 5-bit, int8 sum, L2",
+            "sweep": rows}
+
+
+def run_lq(args):
+    """The LQ-SGD log quantizer: quantize + decode-sum of 24 factor pairs of
+    4096 x r per worker, W = 8, r in {1, 4, 7}."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    W = synthetic.LQ_WORKLOAD["W"]
+    rows = []
+    for r in synthetic.LQ_WORKLOAD["ranks"]:
+        x, sizes = synthetic.lq_factors(r, W=W, device="cuda")
+        n = x.shape[1]
+        R = [4096] * len(sizes)
+        C = [r] * len(sizes)
+        cfg = gq.GQConfig(levels="log", alpha=synthetic.LQ_WORKLOAD["alpha"], seed=1)
+        mx = torch.empty((W, len(sizes)), dtype=torch.float32, device="cuda")
+        codes = torch.empty((W, n), dtype=torch.int8, device="cuda")
+        out = torch.empty(n, dtype=torch.float32, device="cuda")
+        ws = torch.empty(gq.gq_workspace_bytes(gq.GQConfig(), W, 1), dtype=torch.uint8,
+                         device="cuda")
+        gq.gq_workspace_init(ws)
+        K = 200
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K + 5)]
+        for i in range(K + 5):
+            cfg.step = i
+            evs[i][0].record(stream)
+            gq.gq_logq_quantize(x, R, C, cfg, mx, codes, ws, stream)
+            evs[i][1].record(stream)
+            gq.gq_logq_decode_sum(codes, mx, R, C, cfg, out, stream)
+            evs[i][2].record(stream)
+        torch.cuda.synchronize()
+        qm = statistics.median(e[0].elapsed_time(e[1]) for e in evs[5:])
+        dm = statistics.median(e[1].elapsed_time(e[2]) for e in evs[5:])
+        # algorithmic bytes: two reads of the factors + int8 codes; codes + fp32 out
+        qb = 8 * W * n + W * n
+        db = W * n + 4 * n
+        rows.append({"rank": r, "elements_per_worker": n, "quantize_ms": round(qm, 5),
+                     "decode_sum_ms": round(dm, 5),
+                     "quantize_gbs": round(qb / (qm * 1e-3) / 1e9, 1),
+                     "decode_sum_gbs": round(db / (dm * 1e-3) / 1e9, 1),
+                     "code_bytes_per_worker": n, "fp32_bytes_per_worker": 4 * n})
+    return {"metric": "LQ-SGD log quantizer: factor GB/s", "mode": "lq", "unit": "GB/s",
+            "W": W, "rows": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -358,6 +467,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--reference-coords", type=int, default=1 << 21)
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line with the d = 2^16..2^30 sweep instead of the bench line")
+    ap.add_argument("--lq", action="store_true",
+                    help="one JSON line with the LQ-SGD log-quantizer timings")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -369,6 +482,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.sweep or args.lq:
+        if rank == 0:
+            print(json.dumps(run_sweep(args) if args.sweep else run_lq(args)), flush=True)
         return
 
     if world > 1:

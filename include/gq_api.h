@@ -134,11 +134,21 @@ GQ_API int gq_workspace_init(void* ws_dev, size_t bytes, cudaStream_t stream);
  * GQ_ERR_CUDA. */
 GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream);
 
+/* Self-test of the device-side failure detection (no counterpart in the
+ * pages): one thread waits, with the same bounded wait the bulk-copy pipeline
+ * of the fused pass uses, on an mbarrier phase that nothing completes; after
+ * limit_ms (1..10000) it gives up and raises the timeout flag in the
+ * workspace, so gq_get_device_status then returns GQ_ERR_TIMEOUT.  Nothing
+ * faults and the context stays usable. */
+GQ_API int gq_selftest_wait_timeout(void* ws_dev, unsigned int limit_ms, cudaStream_t stream);
+
 /* Step 1 -- global scale.  g_dev, e_dev (NULL unless cfg->ef): [W][d] fp32.
  * v = fl(g + e).  L2: per-worker sum of squares with fp32 squares, fp32
  * partial sums of at most 16 terms and fp64 accumulation, combined in a
- * fixed order; S = (float) max_w sqrt(sum) (within 1e-5 relative of the fp64
- * norm).  MAXABS: S = max |v|, exact.  Writes S to scale_dev[0] (device, 1
+ * fixed order; S = (float) max_w max(sqrt(sum_w), max_j |v_wj|) -- within
+ * 1e-5 relative of the fp64 norm; the max-abs term only undoes rounding (the
+ * exact norm is never below it) and guarantees S >= |v| for every input.
+ * MAXABS: S = max |v|, exact.  Writes S to scale_dev[0] (device, 1
  * float) and, if norms_dev is not NULL, the W per-worker norms (fp64; the
  * per-worker max-abs for MAXABS).  Two-stage reduction inside one launch: the
  * last block to finish (atomic ticket in the workspace) combines the
@@ -172,8 +182,11 @@ GQ_API int gq_global_norm_noalloc(const float* g_dev, const float* e_dev, int W,
                                   cudaStream_t stream);
 
 /* Steps 2-3 -- stochastic quantization and packing, given the scale on the
- * device.  UNIFORM: a = fl(s/S), r = min(fl(|v|*a), s), code = sign(v) *
- * floor(r + u), u = f*2^-23 with f the low 23 bits of Philox word j&3 of
+ * device, which must bound every input (|v| <= S, as gq_global_norm's does;
+ * with a smaller scale the codes are unspecified).  UNIFORM: a = s/S rounded
+ * toward zero, r = fl(v*a) (so |r| <= s), code = floor(r + u) (the signed
+ * value is rounded: each coordinate has the law of sign(v) * floor(|r| + u)),
+ * u = f*2^-23 with f the low 23 bits of Philox word j&3 of
  * counter (lo32(j>>2), step, worker, hi32(j>>2)), key (lo32 seed, hi32 seed).
  * EXP: a = fl(1/S), r = min(fl(|v|*a), 1), bracketed between adjacent levels
  * (exponent bits of r), rounded up with probability (r - lo)/(hi - lo)

@@ -40,6 +40,8 @@ def lib():
         L.gqo_quantize.argtypes = [P, P, i32, i64, P, i32, i32, i32, u64, u32, f32, P]
         L.gqo_code_value.argtypes = [i32, i32, i32]
         L.gqo_code_value.restype = i32
+        L.gqo_uniform_multiplier.argtypes = [i32, f32]
+        L.gqo_uniform_multiplier.restype = f32
         L.gqo_packed_row_bytes.argtypes = [i32, i64]
         L.gqo_packed_row_bytes.restype = i64
         L.gqo_pack.argtypes = [P, i32, i64, i32, P]
@@ -122,6 +124,10 @@ def quantize(g, e=None, *, levels=UNIFORM, s=15, L=8, seed=0, step=0, S, js=None
     _check(lib().gqo_quantize(_p(g), _p(e), W, n, _p(jsa), levels, s, L, seed, step,
                               float(S), _p(out)), "quantize")
     return out
+
+
+def uniform_multiplier(s, S):
+    return np.float32(lib().gqo_uniform_multiplier(int(s), float(S)))
 
 
 def code_value(code, levels, L=8):

@@ -137,8 +137,9 @@ int gqo_global_scale(const float* g, const float* e, int W, int64_t d,
  * Quantizers.
  *
  * UNIFORM ([NUQ] Abstract names QSGD; [GQ] gives the shared scale): levels
- * {0, +-1/s, ..., +-1} of S.  a = fl(s/S); r = fl(v*a) (signed), clamped to
- * [-s, s] (the product can overshoot by rounding); l = floor(r), p = r - l
+ * {0, +-1/s, ..., +-1} of S.  a = s/S rounded toward zero; r = fl(v*a)
+ * (signed), clamped to [-s, s] (a guard: with |v| <= S it never acts);
+ * l = floor(r), p = r - l
  * (exact, also for negative r); code = l + [p + u >= 1].  Rounding the signed
  * value this way gives each coordinate the same two outcomes with the same
  * probabilities as attaching v's sign to the rounded magnitude (for r = -2.3:
@@ -146,7 +147,8 @@ int gqo_global_scale(const float* g, const float* e, int W, int64_t d,
  * same unbiased random variable; only the coupling to u differs.
  *
  * EXP ([NUQ] Abstract: nonuniform levels): levels {0, 2^-(L-1), ..., 1/2, 1}
- * of S.  a = fl(1/S); r = fl(|v|*a), clamped to 1.  If r >= 2^-(L-1) write
+ * of S.  a = 1/S rounded toward zero; r = fl(|v|*a), clamped to 1 (a guard:
+ * with |v| <= S it never acts).  If r >= 2^-(L-1) write
  * r = f * 2^E with f in [1,2) (exponent read off the float, as frexp does):
  * the bracketing levels are 2^E and 2^(E+1), the lower one has index
  * L + E (index i stands for 2^(i-L)), and the round-up probability
@@ -155,10 +157,28 @@ int gqo_global_scale(const float* g, const float* e, int W, int64_t d,
  *
  * A scale that is zero or not finite gives a = 0, hence all codes 0.
  * ---------------------------------------------------------------------- */
+/* a = the largest float with a * S <= s, i.e. s/S rounded toward zero.
+ * Rounding down means |v| * a <= s exactly whenever |v| <= S, so no level
+ * above s is ever reached for a scale that bounds the inputs (the clamp below
+ * then never acts).  Found from the nearest float by stepping one ulp at a
+ * time; a * S is exact in double (24 + 24 significant bits). */
 static float uniform_magnitude_ratio(int s, float S)
 {
     if (!(S > 0.0f) || !isfinite(S)) return 0.0f;
-    return (float)s / S;
+    double sd = (double)s;
+    float a = (float)(sd / (double)S);
+    while ((double)a * (double)S > sd) a = nextafterf(a, 0.0f);
+    for (;;) {
+        float up = nextafterf(a, INFINITY);
+        if ((double)up * (double)S > sd) break;
+        a = up;
+    }
+    return a;
+}
+
+float gqo_uniform_multiplier(int s, float S)
+{
+    return uniform_magnitude_ratio(s, S);
 }
 
 static int32_t quantize_uniform(float v, float a, int s, uint32_t f)
@@ -206,11 +226,8 @@ int gqo_quantize(const float* g, const float* e, int W, int64_t n,
     } else {
         return -1;
     }
-    float a;
-    if (levels == GQO_UNIFORM)
-        a = uniform_magnitude_ratio(s, S);
-    else
-        a = (!(S > 0.0f) || !isfinite(S)) ? 0.0f : 1.0f / S;
+    /* uniform: s/S, exponential: 1/S, both rounded toward zero */
+    float a = uniform_magnitude_ratio(levels == GQO_UNIFORM ? s : 1, S);
     for (int w = 0; w < W; ++w) {
         for (int64_t i = 0; i < n; ++i) {
             int64_t at = (int64_t)w * n + i;

@@ -90,6 +90,10 @@ int gqo_quantize(const float* g, const float* e, int W, int64_t n,
  * sign * 2^(idx-1) units of the finest level 2^-(L-1) (EXP, idx = |code|). */
 int32_t gqo_code_value(int32_t code, int levels, int L);
 
+/* The uniform-level multiplier: the largest float a with a * S <= s (s/S
+ * rounded toward zero); 0 when S is zero or not finite. */
+float gqo_uniform_multiplier(int s, float S);
+
 /* Bytes per worker row of packed codes at `bits` in {4,5,8,16}:
  * ceil(d/128) blocks of 16*bits bytes. */
 int64_t gqo_packed_row_bytes(int bits, int64_t d);

@@ -235,3 +235,19 @@ def test_logq_matches_oracle(gq, oracle, rank):
     assert np.all(np.abs(o - out_ref)[agree] <= tol[agree])
     # where a code moved by one bin, the sum moves by at most one bin width
     assert np.all(np.abs(o - out_ref)[~agree] <= 0.03 * mcol.max(axis=0)[~agree] + tol[~agree])
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(gq):
+    cfg = gq.GQConfig(s=15, bits=5, wire="int8", seed=3)
+    buf = gq.StepBuffers(cfg, 8, 100000)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    assert gq.gq_selftest_wait_timeout(buf.ws, 50) == gq.GQ_ERR_TIMEOUT
+    t1.record()
+    torch.cuda.synchronize()
+    assert 40.0 <= t0.elapsed_time(t1) < 5000.0
+    # the flag was cleared by the read, and the device still runs the path
+    g = synthetic.make_gradients(8, 100000, "normal", seed=1, device="cuda")
+    gq.gq_step_fused(g, None, cfg, buf.scale, buf.norms, buf.codes, buf.sum, buf.out, buf.ws)
+    assert gq.gq_get_device_status(buf.ws) == gq.GQ_OK

@@ -308,9 +308,24 @@ def test_error_feedback_residual_definition(oracle):
         assert np.all(np.abs(r["e"] - (v - q)) <= tol)
 
 
-def test_rounding_overshoot_is_clamped(oracle):
-    """fl(|x| * fl(s/S)) can exceed s when |x| = S (a single-coordinate worker);
-    the code must still stay within s, i.e. the value within S."""
+def test_multiplier_is_s_over_S_rounded_down(oracle):
+    """a is the largest float with a * S <= s, checked in exact rationals."""
+    rng = np.random.default_rng(61)
+    for _ in range(3000):
+        s = int(rng.integers(1, 32768))
+        S = np.float32(10.0 ** rng.uniform(-30, 30))
+        a = oracle.uniform_multiplier(s, S)
+        up = np.nextafter(a, np.float32(np.inf))
+        assert Fraction(float(a)) * Fraction(float(S)) <= s
+        assert Fraction(float(up)) * Fraction(float(S)) > s
+    assert oracle.uniform_multiplier(15, np.float32(0.0)) == 0
+    assert oracle.uniform_multiplier(15, np.float32(np.inf)) == 0
+
+
+def test_no_level_beyond_s_at_the_scale(oracle):
+    """Inputs with |x| = S (a single-coordinate worker) are where a
+    round-to-nearest multiplier would overshoot s; the codes stay within s and
+    almost always equal +-s."""
     rng = np.random.default_rng(60)
     for s in (15, 127):
         x = rng.uniform(0.5, 2.0, 400000).astype(np.float32)
@@ -321,4 +336,14 @@ def test_rounding_overshoot_is_clamped(oracle):
             for sign in (1, -1):
                 codes = oracle.quantize(replicas([sign * xv], 1 << 19), s=s, seed=int(xv * 1e6),
                                         step=1, S=xv)
-                assert np.all(codes == sign * s)
+                assert np.abs(codes).max() <= s
+                assert (codes == sign * s).mean() > 0.999
+
+
+def test_inputs_beyond_the_scale_are_clamped(oracle):
+    """A scale below some |x| (not what the global scale produces) clamps the
+    code to +-s."""
+    x = np.array([2.0, -3.0, 0.5], np.float32)
+    codes = oracle.quantize(replicas(x, 256), s=15, seed=2, step=0, S=np.float32(1.0))
+    assert np.all(codes[:, 0] == 15) and np.all(codes[:, 1] == -15)
+    assert np.all(np.abs(codes[:, 2]) <= 15)
