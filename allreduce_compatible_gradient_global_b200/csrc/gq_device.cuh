@@ -43,7 +43,7 @@ __device__ __forceinline__ uint4 philox_counter(unsigned long long q, uint32_t s
 
 // ---------------------------------------------------------------------------
 // Stochastic rounding.  A magnitude y >= 0 becomes floor(y + u) with
-// u = f * 2^-23, f the low 23 bits of a Philox word: that is floor(y) + 1
+// u = f * 2^-23, f the top 23 bits of a Philox word: that is floor(y) + 1
 // exactly when frac(y) + u >= 1, an event of probability frac(y), so the
 // rounding is unbiased.
 //
@@ -54,8 +54,20 @@ __device__ __forceinline__ uint4 philox_counter(unsigned long long q, uint32_t s
 // in [2^23, 2^24) are the integers.  So the integer is the bit pattern minus
 // that of 2^23, minus 1 for the U offset.  Valid for 0 <= y < 2^23 - 2.
 // ---------------------------------------------------------------------------
+// f = word >> 9 as the high half of word * 2^23, so that it runs on the
+// multiply pipe (the logic pipe is the busier one in the fused pass).
+__device__ __forceinline__ uint32_t top23(uint32_t word) {
+    uint32_t r;
+    asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(word), "r"(0x00800000u));
+    return r;
+}
+
+// U = 1 + u as a float: exponent of 1.0 with f in the mantissa (the add is
+// exact: f < 2^23 never reaches the exponent field).
 __device__ __forceinline__ float unit_plus_u(uint32_t word) {
-    return __uint_as_float(0x3F800000u | (word & 0x007FFFFFu));
+    uint32_t r;
+    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(word), "r"(0x00800000u), "r"(0x3F800000u));
+    return __uint_as_float(r);
 }
 
 __device__ __forceinline__ int floor_y_plus_u(float y, float U) {
@@ -113,7 +125,7 @@ __device__ __forceinline__ float quant_uniform_biased_unclamped(float v, float a
 __device__ __forceinline__ int quant_exp(float v, float a, int L, float finest, float inv_finest,
                                          uint32_t word) {
     const float r = fminf(__fmul_rn(fabsf(v), a), 1.0f);
-    const uint32_t f = word & 0x007FFFFFu;
+    const uint32_t f = top23(word);
     int idx;
     if (r >= finest) {
         const uint32_t rb = __float_as_uint(r);
@@ -137,7 +149,7 @@ __device__ __forceinline__ int quant_exp(float v, float a, int L, float finest, 
 // subtracting the added level leaves 0 or +-2^-(L-1).
 __device__ __forceinline__ float quant_exp_level(float v, float a, float finest, uint32_t word) {
     const float r = __fmul_rn(v, a);
-    const uint32_t f = word & 0x007FFFFFu;
+    const uint32_t f = top23(word);
     const float fin_s = __uint_as_float(__float_as_uint(finest) | (__float_as_uint(r) & 0x80000000u));
     const bool small = fabsf(r) < finest;
     const float x = small ? __fadd_rz(r, fin_s) : r;

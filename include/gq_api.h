@@ -186,7 +186,7 @@ GQ_API int gq_global_norm_noalloc(const float* g_dev, const float* e_dev, int W,
  * with a smaller scale the codes are unspecified).  UNIFORM: a = s/S rounded
  * toward zero, r = fl(v*a) (so |r| <= s), code = floor(r + u) (the signed
  * value is rounded: each coordinate has the law of sign(v) * floor(|r| + u)),
- * u = f*2^-23 with f the low 23 bits of Philox word j&3 of
+ * u = f*2^-23 with f the top 23 bits of Philox word j&3 of
  * counter (lo32(j>>2), step, worker, hi32(j>>2)), key (lo32 seed, hi32 seed).
  * EXP: a = fl(1/S), r = min(fl(|v|*a), 1), bracketed between adjacent levels
  * (exponent bits of r), rounded up with probability (r - lo)/(hi - lo)

@@ -53,7 +53,7 @@ uint32_t gqo_uniform_bits(uint64_t seed, uint32_t tag, uint32_t step,
     ctr[2] = worker;
     ctr[3] = (uint32_t)(q >> 32);
     gqo_philox4x32(ctr, (uint32_t)seed, (uint32_t)(seed >> 32) ^ tag, 10);
-    return ctr[j & 3] & 0x007FFFFFu;
+    return ctr[j & 3] >> 9; /* the top 23 bits */
 }
 
 /* Stochastic rounding decision shared by every quantizer here.

@@ -54,7 +54,7 @@ void gqo_philox4x32(uint32_t ctr[4], uint32_t k0, uint32_t k1, int rounds);
 /* The 23-bit uniform integer f (u = f * 2^-23) drawn for coordinate j of
  * worker `worker` at step `step`: key = (lo32 seed, hi32 seed ^ tag),
  * counter = (lo32(j>>2), step, worker, hi32(j>>2)), output word j & 3,
- * low 23 bits. */
+ * top 23 bits (word >> 9). */
 uint32_t gqo_uniform_bits(uint64_t seed, uint32_t tag, uint32_t step,
                           uint32_t worker, uint64_t j);
 

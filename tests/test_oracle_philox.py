@@ -68,7 +68,7 @@ def test_philox_round_count_matters(oracle):
 
 def test_uniform_bits_follow_the_counter_layout(oracle):
     # coordinate j of worker w at step t uses block (j>>2) of the stream keyed by
-    # (seed, tag), word j & 3, low 23 bits; counter word 3 carries j >> 34.
+    # (seed, tag), word j & 3, top 23 bits; counter word 3 carries j >> 34.
     seed, tag = 0x0123456789ABCDEF, 0x4C510003
     rng = np.random.default_rng(3)
     for _ in range(200):
@@ -78,7 +78,7 @@ def test_uniform_bits_follow_the_counter_layout(oracle):
         q = j >> 2
         blk = oracle.philox4x32([q & 0xFFFFFFFF, t, w, q >> 32],
                                 (seed & 0xFFFFFFFF, (seed >> 32) ^ tag))
-        assert oracle.uniform_bits(seed, tag, t, w, j) == int(blk[j & 3]) & 0x7FFFFF
+        assert oracle.uniform_bits(seed, tag, t, w, j) == int(blk[j & 3]) >> 9
 
 
 def test_uniform_bits_are_uniform(oracle):
