@@ -1,0 +1,62 @@
+"""The bandwidth model (host arithmetic only)."""
+import math
+
+import numpy as np
+import pytest
+
+from allreduce_compatible_gradient_global_b200 import perfmodel as pm
+
+
+def test_fit_recovers_launch_and_bandwidth():
+    rng = np.random.default_rng(0)
+    sizes = np.array([1e6, 4e6, 1.6e7, 6.4e7, 2.6e8, 1e9])
+    t = 7e-6 + sizes / 5.5e12
+    launch, bw = pm.fit_launch_and_bandwidth(sizes, t)
+    assert abs(launch - 7e-6) < 1e-12 and abs(bw - 5.5e12) / 5.5e12 < 1e-9
+    noisy = t * (1 + 1e-3 * rng.standard_normal(t.size))
+    launch, bw = pm.fit_launch_and_bandwidth(sizes, noisy)
+    assert abs(bw - 5.5e12) / 5.5e12 < 0.01
+    with pytest.raises(ValueError):
+        pm.fit_launch_and_bandwidth([5, 5], [1, 2])
+
+
+def test_step_bytes_of_the_resnet50_sized_workload():
+    W, d = 8, 25_557_032
+    p1, p2 = pm.step_bytes(W, d, bits=5, sum_bytes=1)
+    assert p1 == 4 * W * d
+    assert p2 == 1_073_395_784  # read g, 5-bit padded rows, int8 sum, fp32 mean
+    q1, q2 = pm.step_bytes(W, d, bits=5, sum_bytes=1, ef=True)
+    assert q1 == 2 * p1 and q2 == p2 + 8 * W * d
+
+
+def test_ring_allreduce_cost():
+    assert pm.ring_allreduce_seconds(1e9, 1, 770e9, 1e-5) == 0.0
+    t2 = pm.ring_allreduce_seconds(1e9, 2, 770e9, 1e-5)
+    t8 = pm.ring_allreduce_seconds(1e9, 8, 770e9, 1e-5)
+    assert math.isclose(t2, 1e-5 + 1e9 / 770e9)
+    assert math.isclose(t8, 1e-5 + 1.75e9 / 770e9)
+
+
+def test_crossover_separates_the_regimes():
+    m = pm.Machine()
+    for ranks in (2, 4, 8):
+        d0 = pm.crossover_d(ranks, bits=5, sum_bytes=1, m=m)
+        assert d0 is not None and d0 > 1
+        for d in (d0, 2 * d0, 100 * d0):
+            assert pm.dp_step_seconds(d, ranks, 5, 1, m) < pm.dp_step_seconds(
+                d, ranks, 5, 1, m, compressed=False)
+        assert pm.dp_step_seconds(d0 - 1, ranks, 5, 1, m) >= pm.dp_step_seconds(
+            d0 - 1, ranks, 5, 1, m, compressed=False)
+    # a single GPU has no exchange: compression never pays
+    assert pm.crossover_d(1, m=m) is None
+
+
+def test_large_d_ratio_follows_the_byte_counts():
+    m = pm.Machine()
+    d, n = 1 << 40, 8
+    fast = pm.dp_step_seconds(d, n, 5, 1, m)
+    slow = pm.dp_step_seconds(d, n, 5, 1, m, compressed=False)
+    per_coord_fast = (4 / m.hbm + (4 + 5 / 8) / (m.hbm * m.pass2_efficiency) + 5 / m.hbm
+                      + 2 * (n - 1) / n / m.link)
+    per_coord_slow = 2 * (n - 1) / n * 4 / m.link
+    assert math.isclose(slow / fast, per_coord_slow / per_coord_fast, rel_tol=1e-3)
