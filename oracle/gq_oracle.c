@@ -181,6 +181,19 @@ float gqo_uniform_multiplier(int s, float S)
     return uniform_magnitude_ratio(s, S);
 }
 
+/* The same decision for a signed r = l + p, l = floor(r): round up exactly
+ * when r + u >= l + 1, i.e. code = floor(r + u).  The fraction p = r - l of a
+ * negative r is not always a float (r = -(u + 2^-26) with u in [1/8, 1/4) has
+ * p = 1 - u - 2^-26, which a float subtraction rounds to 1 - u), so the
+ * comparison is made on r + u itself, in double.  It is exact: r + u can
+ * round only when r carries bits below 2^-38, i.e. |r| < 2^-14, and then
+ * l + 1 is 0 or 1, which no such sum reaches by rounding. */
+static int round_up_signed(float r, float l, uint32_t f)
+{
+    double u = (double)f * (1.0 / 8388608.0);
+    return ((double)r + u) >= (double)l + 1.0;
+}
+
 static int32_t quantize_uniform(float v, float a, int s, uint32_t f)
 {
     float r = v * a;
@@ -188,8 +201,7 @@ static int32_t quantize_uniform(float v, float a, int s, uint32_t f)
     if (!(r <= smax)) r = smax; /* also maps NaN to s, as fminf does */
     if (r < -smax) r = -smax;
     float l = floorf(r);
-    float p = r - l;
-    return (int32_t)l + round_up(p, f);
+    return (int32_t)l + round_up_signed(r, l, f);
 }
 
 static int32_t quantize_exp(float v, float a, int L, uint32_t f)

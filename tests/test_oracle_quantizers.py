@@ -347,3 +347,53 @@ def test_inputs_beyond_the_scale_are_clamped(oracle):
     codes = oracle.quantize(replicas(x, 256), s=15, seed=2, step=0, S=np.float32(1.0))
     assert np.all(codes[:, 0] == 15) and np.all(codes[:, 1] == -15)
     assert np.all(np.abs(codes[:, 2]) <= 15)
+
+
+# ------------------------------------------------- the rounding decision, exactly
+def _exact_code(r, f):
+    """floor(r + f 2^-23) in rationals: the uniform-level code of r = fl(v a)."""
+    return math.floor(Fraction(float(r)) + Fraction(int(f), 1 << 23))
+
+
+def test_uniform_code_is_exact_floor_at_decision_boundaries(oracle):
+    """r = v a sitting a fraction of an ulp of (1 - p) away from the decision
+    boundary u = 1 - p, on both sides, and r = -u exactly.  With S = s the
+    multiplier is exactly 1, so r = v.  A fraction taken with a float
+    subtraction, fl(r - floor(r)), rounds 1 - u - 2^-26 to 1 - u and flips
+    the first kind to a round-up; the exact rule floor(r + u) does not."""
+    s, seed, step = 15, 7, 1
+    assert oracle.uniform_multiplier(s, np.float32(s)) == np.float32(1.0)
+    js, fs = [], []
+    for j in range(4000):
+        f = oracle.uniform_bits(seed, 0, step, 0, j)
+        if (1 << 20) <= f < (1 << 21):  # u in [1/8, 1/4): |r| has ulp 2^-26
+            js.append(j)
+            fs.append(f)
+    assert len(js) >= 200
+    js, fs = np.array(js[:240], np.int64), np.array(fs[:240], np.int64)
+    u = fs.astype(np.float64) / (1 << 23)
+    kinds = np.arange(js.size) % 3
+    r = np.where(kinds == 0, -(u + 2.0 ** -26),           # just past the boundary: -1
+                 np.where(kinds == 1, -(u - 2.0 ** -26),  # just short of it: 0
+                          -u))                             # on it: 0
+    v = r.astype(np.float32)
+    assert np.array_equal(v.astype(np.float64), r)  # all exactly representable
+    codes = oracle.quantize(v[None, :], s=s, seed=seed, step=step, S=np.float32(s), js=js)[0]
+    want = np.array([_exact_code(x, f) for x, f in zip(v, fs)])
+    assert np.array_equal(want[kinds == 0], -np.ones((kinds == 0).sum()))
+    assert not want[kinds != 0].any()
+    assert np.array_equal(codes, want)
+
+
+def test_uniform_code_is_exact_floor_random(oracle):
+    """20000 random r of both signs and magnitudes from 2^-40 to s, exact check."""
+    s, seed, step = 127, 3, 9
+    rng = np.random.default_rng(5)
+    n = 20000
+    mag = np.exp2(rng.uniform(-40, np.log2(s), n))
+    v = (mag * rng.choice([-1.0, 1.0], n)).astype(np.float32)
+    js = np.arange(n, dtype=np.int64) * 7 + 11
+    codes = oracle.quantize(v[None, :], s=s, seed=seed, step=step, S=np.float32(s), js=js)[0]
+    fs = [oracle.uniform_bits(seed, 0, step, 0, int(j)) for j in js]
+    want = np.array([_exact_code(x, f) for x, f in zip(v, fs)])
+    assert np.array_equal(codes, want)
