@@ -102,6 +102,11 @@ def _load():
         "gq_quantize_aggregate": ([P, P, I, LL, CP, P, P, P, P, P, P], I),
         "gq_step_fused": ([P, P, I, LL, CP, P, P, P, P, P, P, P], I),
         "gq_step_fused_host": ([P, P, P, I, LL, CP, P, P, P, P, P, P, P, P], I),
+        "gq_bucket_count": ([LL, I, ctypes.POINTER(LL)], I),
+        "gq_bucket_workspace_bytes": ([CP, I, LL, I, ctypes.POINTER(ctypes.c_size_t)], I),
+        "gq_bucket_scales": ([P, P, I, LL, I, CP, P, P, P], I),
+        "gq_quantize_aggregate_bucketed": ([P, P, I, LL, I, CP, P, P, P, P, P, P], I),
+        "gq_step_bucketed": ([P, P, I, LL, I, CP, P, P, P, P, P, P], I),
         "gq_logq_quantize": ([P, I, I, P, P, CP, P, P, P, P], I),
         "gq_logq_decode_sum": ([P, P, I, I, P, P, CP, P, P], I),
     }
@@ -339,6 +344,62 @@ def gq_logq_decode_sum(codes, maxabs, rows, cols, cfg: GQConfig, out, stream=Non
     _check(lib().gq_logq_decode_sum(_ptr(codes), _ptr(maxabs), W, len(rows), r, cc,
                                    ctypes.byref(c), _ptr(out), _stream(stream)),
            "gq_logq_decode_sum")
+
+
+# ------------------------------------------------------------------ per-bucket scales
+def gq_bucket_count(d: int, bucket_log2: int) -> int:
+    out = ctypes.c_longlong()
+    _check(lib().gq_bucket_count(int(d), int(bucket_log2), ctypes.byref(out)), "gq_bucket_count")
+    return out.value
+
+
+def gq_bucket_workspace_bytes(cfg: GQConfig, W: int, d: int, bucket_log2: int) -> int:
+    c = cfg.c()
+    out = ctypes.c_size_t()
+    _check(lib().gq_bucket_workspace_bytes(ctypes.byref(c), int(W), int(d), int(bucket_log2),
+                                           ctypes.byref(out)), "gq_bucket_workspace_bytes")
+    return out.value
+
+
+def gq_bucket_scales(g, e, bucket_log2, cfg: GQConfig, table, ws, stream=None):
+    """table: float32 [3 * K] = S_k | multipliers | units."""
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(table, torch.float32, (3 * gq_bucket_count(d, bucket_log2),), "table")
+    c = cfg.c()
+    _check(lib().gq_bucket_scales(_ptr(g), _ptr(e), W, d, int(bucket_log2), ctypes.byref(c),
+                                  _ptr(table), _ptr(ws), _stream(stream)), "gq_bucket_scales")
+
+
+def gq_quantize_aggregate_bucketed(g, e, bucket_log2, cfg: GQConfig, table, codes, sum_out, out,
+                                   ws, stream=None):
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(table, torch.float32, (3 * gq_bucket_count(d, bucket_log2),), "table")
+    _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
+    _need(sum_out, cfg.wire_dtype, (d,), "sum")
+    _need(out, torch.float32, (d,), "out")
+    c = cfg.c()
+    _check(lib().gq_quantize_aggregate_bucketed(
+        _ptr(g), _ptr(e), W, d, int(bucket_log2), ctypes.byref(c), _ptr(table), _ptr(codes),
+        _ptr(sum_out), _ptr(out), _ptr(ws), _stream(stream)), "gq_quantize_aggregate_bucketed")
+
+
+def gq_step_bucketed(g, e, bucket_log2, cfg: GQConfig, table, codes, sum_out, out, ws,
+                     stream=None):
+    W, d = _wd(g)
+    _need(g, torch.float32, (W, d), "g")
+    _need(e, torch.float32, (W, d), "e")
+    _need(table, torch.float32, (3 * gq_bucket_count(d, bucket_log2),), "table")
+    _need(codes, torch.uint8, (W, gq_packed_row_bytes(cfg, d)), "codes")
+    _need(sum_out, cfg.wire_dtype, (d,), "sum")
+    _need(out, torch.float32, (d,), "out")
+    c = cfg.c()
+    _check(lib().gq_step_bucketed(_ptr(g), _ptr(e), W, d, int(bucket_log2), ctypes.byref(c),
+                                  _ptr(table), _ptr(codes), _ptr(sum_out), _ptr(out), _ptr(ws),
+                                  _stream(stream)), "gq_step_bucketed")
 
 
 # ------------------------------------------------------------------ buffers

@@ -182,6 +182,21 @@ void fill_quant_args(QuantArgs& a, const gq_config* cfg, int W, long long d) {
     a.inv_w = a.w_pow2 ? 1.0f / (float)W : 0.0f;
 }
 
+// Per-bucket scales: buckets of 2^b coordinates, partials per chunk of
+// 2^min(b, 12) coordinates.
+constexpr int kBucketLog2Min = 7, kBucketLog2Max = 30, kChunkLog2Max = 12;
+
+int chunk_log2_of(int b) { return b < kChunkLog2Max ? b : kChunkLog2Max; }
+long long count_of(long long d, int log2) { return (d + (1LL << log2) - 1) >> log2; }
+
+size_t bucket_ws_bytes(int W, long long d, int b) {
+    const size_t items = (size_t)W * (size_t)count_of(d, chunk_log2_of(b));
+    const size_t own = kWorkspaceHeader + items * (sizeof(double) + sizeof(unsigned));
+    const size_t global = kWorkspaceHeader + (size_t)W * kMaxNormBlocks * 2 * sizeof(double);
+    const size_t n = own > global ? own : global;
+    return (n + 255) & ~(size_t)255;
+}
+
 }  // namespace
 
 extern "C" {
@@ -509,6 +524,104 @@ GQ_API int gq_logq_decode_sum(const signed char* codes_dev, const float* maxabs_
         if ((rc = cuda_status(launch_logq_decode(a, stream)))) return rc;
     }
     return GQ_OK;
+}
+
+GQ_API int gq_bucket_count(long long d, int bucket_log2, long long* nbuckets) {
+    if (!nbuckets || d < 0 || bucket_log2 < kBucketLog2Min || bucket_log2 > kBucketLog2Max)
+        return GQ_ERR_ARG;
+    *nbuckets = count_of(d, bucket_log2);
+    return GQ_OK;
+}
+
+GQ_API int gq_bucket_workspace_bytes(const gq_config* cfg, int W, long long d, int bucket_log2,
+                                     size_t* bytes) {
+    if (!cfg || !bytes || bucket_log2 < kBucketLog2Min || bucket_log2 > kBucketLog2Max)
+        return GQ_ERR_ARG;
+    int rc = check_sizes(W, d);
+    if (rc) return rc;
+    *bytes = bucket_ws_bytes(W, d, bucket_log2);
+    return GQ_OK;
+}
+
+GQ_API int gq_bucket_scales(const float* g_dev, const float* e_dev, int W, long long d,
+                            int bucket_log2, const gq_config* cfg, float* table_dev, void* ws_dev,
+                            cudaStream_t stream) {
+    if (!cfg || bucket_log2 < kBucketLog2Min || bucket_log2 > kBucketLog2Max) return GQ_ERR_ARG;
+    int rc = gq_validate(cfg, W, d);
+    if (rc) return rc;
+    if (cfg->levels == GQ_LOG) return GQ_ERR_ARG;
+    if ((!g_dev && d > 0) || !ws_dev || (!table_dev && d > 0)) return GQ_ERR_ARG;
+    if (cfg->ef && !e_dev && d > 0) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || (cfg->ef && !aligned16(e_dev)) || !aligned16(ws_dev) ||
+        !aligned4(table_dev))
+        return GQ_ERR_ALIGN;
+    if (d == 0) return GQ_OK;
+    BucketArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.g = g_dev;
+    a.e = cfg->ef ? e_dev : nullptr;
+    a.d = d;
+    a.W = W;
+    a.bucket_log2 = bucket_log2;
+    a.chunk_log2 = chunk_log2_of(bucket_log2);
+    a.nbuckets = count_of(d, bucket_log2);
+    a.nchunks = count_of(d, a.chunk_log2);
+    a.kind = cfg->scale_kind;
+    a.levels = cfg->levels;
+    a.smax = (float)cfg->s;
+    a.finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, -(cfg->L - 1)) : 1.0f;
+    a.scales = table_dev;
+    a.mult = table_dev + a.nbuckets;
+    a.unit = table_dev + 2 * a.nbuckets;
+    a.part_sum = reinterpret_cast<double*>(partials_of(ws_dev));
+    a.part_max = reinterpret_cast<unsigned*>(a.part_sum + (size_t)W * a.nchunks);
+    a.hdr = header_of(ws_dev);
+    return cuda_status(launch_bucket_scales(a, sm_count(), stream));
+}
+
+GQ_API int gq_quantize_aggregate_bucketed(const float* g_dev, float* e_dev, int W, long long d,
+                                          int bucket_log2, const gq_config* cfg,
+                                          const float* table_dev, void* codes_dev, void* sum_dev,
+                                          float* out_dev, void* ws_dev, cudaStream_t stream) {
+    if (!cfg || bucket_log2 < kBucketLog2Min || bucket_log2 > kBucketLog2Max) return GQ_ERR_ARG;
+    int rc = gq_validate(cfg, W, d);
+    if (rc) return rc;
+    if (cfg->levels == GQ_LOG) return GQ_ERR_ARG;
+    if (!g_dev || !table_dev || !ws_dev) return GQ_ERR_ARG;
+    const bool ef = cfg->ef != 0;
+    if (ef && !e_dev) return GQ_ERR_ARG;
+    if (!codes_dev && !sum_dev && !out_dev && !ef) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || (ef && !aligned16(e_dev)) || !aligned4(table_dev) ||
+        (codes_dev && !aligned16(codes_dev)) || (sum_dev && !aligned16(sum_dev)) ||
+        (out_dev && !aligned16(out_dev)))
+        return GQ_ERR_ALIGN;
+    if (d == 0) return GQ_OK;
+    const long long K = count_of(d, bucket_log2);
+    QuantArgs a;
+    fill_quant_args(a, cfg, W, d);
+    a.g = g_dev;
+    a.e = ef ? e_dev : nullptr;
+    a.scale = table_dev;  // replaced per 128-coordinate block by the bucket's entries
+    a.bq_mult = table_dev + K;
+    a.bq_unit = table_dev + 2 * K;
+    a.bucket_shift = bucket_log2 - 7;
+    a.codes = reinterpret_cast<unsigned char*>(codes_dev);
+    a.row_bytes = row_bytes_of(cfg->bits, d);
+    a.update_e = ef ? 1 : 0;
+    a.sum = sum_dev;
+    a.out = out_dev;
+    const int bits = codes_dev ? cfg->bits : 0;
+    return cuda_status(launch_fused(a, cfg->levels, bits, ef, ws_dev, d, stream));
+}
+
+GQ_API int gq_step_bucketed(const float* g_dev, float* e_dev, int W, long long d, int bucket_log2,
+                            const gq_config* cfg, float* table_dev, void* codes_dev, void* sum_dev,
+                            float* out_dev, void* ws_dev, cudaStream_t stream) {
+    int rc = gq_bucket_scales(g_dev, cfg && cfg->ef ? e_dev : nullptr, W, d, bucket_log2, cfg,
+                              table_dev, ws_dev, stream);
+    if (rc) return rc;
+    return gq_quantize_aggregate_bucketed(g_dev, e_dev, W, d, bucket_log2, cfg, table_dev,
+                                          codes_dev, sum_dev, out_dev, ws_dev, stream);
 }
 
 }  // extern "C"

@@ -58,6 +58,32 @@ struct QuantArgs {
     float inv_w;       // 1/W when W is a power of two
     int w_pow2;
     WsHeader* hdr;  // flag word for pipeline timeouts
+    // per-bucket scales (null: one global scale): the multiplier and unit of
+    // 128-coordinate block b are bq_mult[b >> bucket_shift], bq_unit[...]
+    const float* bq_mult;
+    const float* bq_unit;
+    int bucket_shift;
+};
+
+struct BucketArgs {
+    const float* g;
+    const float* e;
+    long long d;
+    long long nbuckets;
+    long long nchunks;  // ceil(d / 2^chunk_log2)
+    int W;
+    int bucket_log2;  // bucket = 2^bucket_log2 coordinates, 7 <= bucket_log2 <= 30
+    int chunk_log2;   // min(bucket_log2, 12)
+    int kind;         // 0: L2, 1: max-abs
+    int levels;       // 0: uniform, 1: exponential
+    float smax;
+    float finest;
+    float* scales;  // [nbuckets] S_k
+    float* mult;    // [nbuckets] multiplier of the fused pass
+    float* unit;    // [nbuckets] value of one unit (decode / error feedback)
+    double* part_sum;    // [W][nchunks] per-chunk sums of squares
+    unsigned* part_max;  // [W][nchunks] per-chunk max |v| bits
+    WsHeader* hdr;
 };
 
 struct AggArgs {
@@ -124,6 +150,7 @@ cudaError_t launch_quant_tma(const QuantArgs& a, int levels, int bits, bool ef, 
 // Bounded-wait self-test (raises kFlagPipelineTimeout after limit_ns).
 cudaError_t launch_wait_timeout_selftest(WsHeader* hdr, unsigned long long limit_ns,
                                          cudaStream_t st);
+cudaError_t launch_bucket_scales(const BucketArgs& a, int sms, cudaStream_t st);
 cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st);
 cudaError_t launch_logq_decode(const LogqArgs& a, cudaStream_t st);
 

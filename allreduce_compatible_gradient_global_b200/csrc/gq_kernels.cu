@@ -313,6 +313,10 @@ __global__ void __launch_bounds__(kThreads, GQ_QUANT_MIN_BLOCKS)
 
     for (long long it = wid; it < nblk; it += nwarps) {
         const long long blk = GQ_QUANT_REVERSE ? nblk - 1 - it : it;
+        if (a.bq_mult) {  // per-bucket scale of this block
+            aq = __ldg(a.bq_mult + (blk >> a.bucket_shift));
+            c = __ldg(a.bq_unit + (blk >> a.bucket_shift));
+        }
         const long long j0 = (blk << 7) + (lane << 2);
         const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
         int s0 = 0, s1 = 0, s2 = 0, s3 = 0;

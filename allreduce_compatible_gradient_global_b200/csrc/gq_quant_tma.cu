@@ -121,7 +121,7 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 // WT: the number of workers when known at compile time (the worker loop is
 // then fully unrolled and the Philox chains of all workers interleave), or 0.
-template <int LEVELS, int BITS, bool EF, int WT>
+template <int LEVELS, int BITS, bool EF, int WT, bool BQ>
 __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     quant_tma_kernel(const __grid_constant__ QuantArgs a, int stages) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -205,10 +205,30 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     const long long row_bytes = a.row_bytes;
     int s = 0;
     uint32_t phase = 0;
+    // per-bucket scales: this warp's next block's multiplier and unit, loaded
+    // one tile ahead so that the load's latency hides behind a tile of work
+    float aq_next = 0.f, c_next = 0.f;
+    const long long blk_step = (long long)gridDim.x * kTmaComputeWarps;
+    if (BQ) {
+        const long long b0 = (long long)blockIdx.x * kTmaComputeWarps + warp;
+        if (b0 < nblk) {
+            aq_next = __ldg(a.bq_mult + (b0 >> a.bucket_shift));
+            c_next = __ldg(a.bq_unit + (b0 >> a.bucket_shift));
+        }
+    }
     for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
         if (!mbar_wait_bounded(full0 + 8 * s, phase, a.hdr)) break;
         const long long blk = t * kTmaComputeWarps + warp;
         if (blk < nblk) {
+            if (BQ) {  // per-bucket scale of this block
+                aq = aq_next;
+                c = c_next;
+                const long long bn = blk + blk_step;
+                if (bn < nblk) {
+                    aq_next = __ldg(a.bq_mult + (bn >> a.bucket_shift));
+                    c_next = __ldg(a.bq_unit + (bn >> a.bucket_shift));
+                }
+            }
             const long long j0 = (blk << 7) + (lane << 2);
             const bool in = j0 < a.d;  // d % 4 == 0: all four or none
             const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
@@ -314,9 +334,9 @@ size_t tma_smem_bytes(int W, bool ef, int stages) {
     return (size_t)stages * rows * kTmaTile * sizeof(float) + 2 * stages * sizeof(unsigned long long);
 }
 
-template <int LEVELS, int BITS, bool EF, int WT>
+template <int LEVELS, int BITS, bool EF, int WT, bool BQ>
 static cudaError_t launch_tma_inst(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
-    auto kern = quant_tma_kernel<LEVELS, BITS, EF, WT>;
+    auto kern = quant_tma_kernel<LEVELS, BITS, EF, WT, BQ>;
     const size_t smem = tma_smem_bytes(a.W, EF, stages);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -326,9 +346,16 @@ static cudaError_t launch_tma_inst(const QuantArgs& a, int stages, int grid, cud
 
 template <int LEVELS, int BITS, bool EF>
 static cudaError_t launch_tma_w(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
+    // per-bucket scales get their own instantiations, so the global-scale
+    // kernel keeps one multiplier in a register for the whole launch
+    if (a.bq_mult) {
+        if (GQ_TMA_SPECIALIZE_W8 && a.W == 8)
+            return launch_tma_inst<LEVELS, BITS, EF, 8, true>(a, stages, grid, st);
+        return launch_tma_inst<LEVELS, BITS, EF, 0, true>(a, stages, grid, st);
+    }
     if (GQ_TMA_SPECIALIZE_W8 && a.W == 8)
-        return launch_tma_inst<LEVELS, BITS, EF, 8>(a, stages, grid, st);
-    return launch_tma_inst<LEVELS, BITS, EF, 0>(a, stages, grid, st);
+        return launch_tma_inst<LEVELS, BITS, EF, 8, false>(a, stages, grid, st);
+    return launch_tma_inst<LEVELS, BITS, EF, 0, false>(a, stages, grid, st);
 }
 
 template <int LEVELS, bool EF>

@@ -432,6 +432,89 @@ def run_sweep(args):
             "sweep": rows}
 
 
+def run_buckets(args):
+    """Per-bucket scales on the benchmark workload: the global-scale step against
+    steps with one scale per bucket of 2^b coordinates.  Per variant: median
+    per-launch times of the scale pass (both bucket launches together) and of
+    the fused pass, the step's gradient GB/s, and the relative squared error
+    ||out - mean_w g||^2 / ||mean_w g||^2 of the decoded mean (one draw),
+    which is what the finer scales buy."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = measured_hbm_peak()
+    wl, cfg = workload_config(gq, args.workload)
+    W, d = wl["W"], wl["d"]
+    g = synthetic.workload_gradients(args.workload, device="cuda")
+    e = torch.zeros_like(g) if cfg.ef else None
+    gbar = g.double().mean(dim=0)
+    ref2 = float((gbar * gbar).sum())
+    p1, p2 = algorithmic_bytes(gq, cfg, W, d)
+    K = max(20, min(args.steps, 200))
+    rows = []
+    for b in (None, 10, 12, 14, 17, 20):
+        if b is None:
+            buf = gq.StepBuffers(cfg, W, d)
+            ws = buf.ws
+            table = None
+        else:
+            buf = gq.StepBuffers(cfg, W, d)
+            nk = gq.gq_bucket_count(d, b)
+            table = torch.empty(3 * nk, dtype=torch.float32, device="cuda")
+            ws = torch.empty(gq.gq_bucket_workspace_bytes(cfg, W, d, b), dtype=torch.uint8,
+                             device="cuda")
+            gq.gq_workspace_init(ws)
+
+        def one(i, ev=None):
+            cfg.step = i
+            if ev is not None:
+                ev[0].record(stream)
+            if b is None:
+                gq.gq_global_norm(g, e, cfg, buf.scale, buf.norms, ws, stream)
+            else:
+                gq.gq_bucket_scales(g, e, b, cfg, table, ws, stream)
+            if ev is not None:
+                ev[1].record(stream)
+            if b is None:
+                gq.gq_quantize_aggregate(g, e, cfg, buf.scale, buf.codes, buf.sum, buf.out, ws,
+                                         stream)
+            else:
+                gq.gq_quantize_aggregate_bucketed(g, e, b, cfg, table, buf.codes, buf.sum,
+                                                  buf.out, ws, stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for i in range(5):
+            one(i)
+        torch.cuda.synchronize()
+        if e is not None:
+            e.zero_()
+        one(5)
+        torch.cuda.synchronize()
+        diff = buf.out.double() - gbar
+        rel = float((diff * diff).sum()) / ref2
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        for i in range(K):
+            one(6 + i, evs[i])
+        torch.cuda.synchronize()
+        if gq.gq_get_device_status(ws, stream) != gq.GQ_OK:
+            raise RuntimeError("device flag raised in the bucket comparison")
+        sm = statistics.median(x[0].elapsed_time(x[1]) for x in evs)
+        qm = statistics.median(x[1].elapsed_time(x[2]) for x in evs)
+        step_ms = sum(x[0].elapsed_time(x[2]) for x in evs) / K
+        rows.append({"bucket_log2": b, "buckets": 1 if b is None else gq.gq_bucket_count(d, b),
+                     "scale_ms": round(sm, 5), "quant_ms": round(qm, 5),
+                     "step_ms": round(step_ms, 5),
+                     "grad_gbs": round(4 * W * d / (step_ms * 1e-3) / 1e9, 1),
+                     "scale_frac": round(p1 / (sm * 1e-3) / 1e9 / peak, 4),
+                     "quant_frac": round(p2 / (qm * 1e-3) / 1e9 / peak, 4),
+                     "rel_sq_error": rel})
+        del buf, table, ws
+        torch.cuda.empty_cache()
+    return {"metric": METRIC, "mode": "buckets", "unit": "GB/s", "peak": peak,
+            "peak_source": peak_kind, "workload": args.workload, "W": W, "d": d, "rows": rows}
+
+
 def run_lq(args):
     """The LQ-SGD log quantizer: quantize + decode-sum of 24 factor pairs of
     4096 x r per worker, W = 8, r in {1, 4, 7}."""
@@ -490,6 +573,8 @@ def main():
                     help="one JSON line with the d = 2^16..2^30 sweep instead of the bench line")
     ap.add_argument("--lq", action="store_true",
                     help="one JSON line with the LQ-SGD log-quantizer timings")
+    ap.add_argument("--buckets", action="store_true",
+                    help="one JSON line comparing the global scale with per-bucket scales")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -502,9 +587,10 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
-    if args.sweep or args.lq:
+    if args.sweep or args.lq or args.buckets:
         if rank == 0:
-            print(json.dumps(run_sweep(args) if args.sweep else run_lq(args)), flush=True)
+            fn = run_sweep if args.sweep else (run_lq if args.lq else run_buckets)
+            print(json.dumps(fn(args)), flush=True)
         return
 
     if world > 1:

@@ -247,6 +247,45 @@ GQ_API int gq_step_fused_host(const float* g_host, float* g_dev, float* e_dev, i
                               float* out_host, float* scale_host, void* ws_dev,
                               cudaStream_t stream);
 
+/* Per-bucket scales (no counterpart in the pages; the reading of "one shared
+ * scale" that keeps allreduce compatibility when the scale varies along the
+ * vector).  The d coordinates are cut into K = ceil(d / 2^bucket_log2)
+ * buckets of 2^bucket_log2 consecutive coordinates (the last may be shorter),
+ * 7 <= bucket_log2 <= 30.  Bucket k gets its own scale S_k, computed exactly
+ * like gq_global_norm's S but over the bucket's coordinates only, and shared
+ * by all workers; every coordinate of bucket k is then quantized, summed and
+ * decoded exactly as by gq_quantize_aggregate with S = S_k.  Codes of one
+ * bucket still sum across workers; a real exchange adds a MAX all-reduce of
+ * the K scales.  The bucketed calls need a workspace of
+ * gq_bucket_workspace_bytes() (which is also a valid gq_workspace_bytes()
+ * workspace for the same W and d) and a caller-owned device table of 3*K
+ * floats: [S_0..S_{K-1} | a_0..a_{K-1} | c_0..c_{K-1}] with a_k the
+ * multiplier (s/S_k or 1/S_k rounded toward zero; 0 when S_k is 0 or not
+ * finite) and c_k the value of one code unit (S_k/s or S_k*2^-(L-1)). */
+GQ_API int gq_bucket_count(long long d, int bucket_log2, long long* nbuckets);
+GQ_API int gq_bucket_workspace_bytes(const gq_config* cfg, int W, long long d, int bucket_log2,
+                                     size_t* bytes);
+
+/* Per-bucket step 1: fills table_dev.  Two launches: per-chunk partial sums
+ * of squares and max-abs for every (worker, chunk of min(2^bucket_log2, 4096)
+ * coordinates), then one block per bucket combines them in a fixed order.  A
+ * non-finite S_k raises the NONFINITE flag of the workspace. */
+GQ_API int gq_bucket_scales(const float* g_dev, const float* e_dev, int W, long long d,
+                            int bucket_log2, const gq_config* cfg, float* table_dev, void* ws_dev,
+                            cudaStream_t stream);
+
+/* Per-bucket steps 2-5: gq_quantize_aggregate with each 128-coordinate block
+ * reading its bucket's a_k and c_k from table_dev. */
+GQ_API int gq_quantize_aggregate_bucketed(const float* g_dev, float* e_dev, int W, long long d,
+                                          int bucket_log2, const gq_config* cfg,
+                                          const float* table_dev, void* codes_dev, void* sum_dev,
+                                          float* out_dev, void* ws_dev, cudaStream_t stream);
+
+/* gq_bucket_scales then gq_quantize_aggregate_bucketed. */
+GQ_API int gq_step_bucketed(const float* g_dev, float* e_dev, int W, long long d, int bucket_log2,
+                            const gq_config* cfg, float* table_dev, void* codes_dev, void* sum_dev,
+                            float* out_dev, void* ws_dev, cudaStream_t stream);
+
 /* LQ-SGD log quantizer.  x_dev is [W][n] fp32 with n = sum_m rows[m]*cols[m]:
  * each worker's nmats factor matrices (row-major rows[m] x cols[m]) stored one
  * after another.  Per worker and matrix: m = max|x| (written to

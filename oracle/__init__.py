@@ -201,6 +201,42 @@ def step(g, e=None, *, levels=UNIFORM, s=15, L=8, scale_kind=SCALE_L2, seed=0,
                 e=e_new)
 
 
+def step_bucketed(g, e=None, *, bucket, levels=UNIFORM, s=15, L=8, scale_kind=SCALE_L2,
+                  seed=0, step=0, ef=False, bits=None, S=None):
+    """The whole path with one scale per bucket of `bucket` consecutive
+    coordinates (the last bucket may be shorter).  Per bucket this is exactly
+    the global-scale path of "Quantize Once, Train Fast" (Abstract: global norm
+    scaling) restricted to the bucket's coordinates: the scale over the slice,
+    then quantization at the slice's own coordinate indices (so the uniforms
+    are the same as in the unbucketed path), integer sum, decode and error
+    feedback with that bucket's scale.  No new arithmetic: a composition of the
+    functions above.  S, when given, is the array of K scales to use."""
+    g = _f32(g)
+    e = _f32(e) if ef else None
+    W, d = g.shape
+    K = -(-d // bucket)
+    S_ref = np.zeros(K, np.float32)
+    codes = np.zeros((W, d), np.int32)
+    total = np.zeros(d, np.int32)
+    out = np.zeros(d, np.float32)
+    e_new = np.zeros((W, d), np.float32) if ef else None
+    for k in range(K):
+        lo, hi = k * bucket, min(d, (k + 1) * bucket)
+        gk = g[:, lo:hi]
+        ek = None if e is None else e[:, lo:hi]
+        S_ref[k], _ = global_scale(gk, ek, scale_kind)
+        Sk = S_ref[k] if S is None else np.float32(S[k])
+        ck = quantize(gk, ek, levels=levels, s=s, L=L, seed=seed, step=step, S=Sk,
+                      js=np.arange(lo, hi, dtype=np.int64))
+        codes[:, lo:hi] = ck
+        total[lo:hi] = aggregate(ck, levels=levels, L=L)
+        out[lo:hi] = decode_mean(total[lo:hi], W, levels=levels, s=s, L=L, S=Sk)
+        if ef:
+            e_new[:, lo:hi] = error_feedback(gk, ek, ck, levels=levels, s=s, L=L, S=Sk)
+    packed = pack(codes, bits) if bits else None
+    return dict(S=S_ref, codes=codes, packed=packed, sum=total, out=out, e=e_new)
+
+
 def logq_quantize(x, sizes, *, alpha=10.0, seed=0, step=0):
     """x: [W][sum(sizes)] float32.  Returns (maxabs[W][nmats], codes int8)."""
     x = _f32(x)

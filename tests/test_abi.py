@@ -143,3 +143,44 @@ def test_entry_points_reject_before_launch(gq):
     clog_bad = cfg(gq, levels="log", alpha=-1.0).c()
     assert lib.gq_logq_decode_sum(good, good, 8, 2, rows, cols, ctypes.byref(clog_bad), good,
                                   None) == gq.GQ_ERR_ARG
+
+
+def test_bucket_sizes_and_workspace(gq):
+    assert gq.gq_bucket_count(0, 10) == 0
+    assert gq.gq_bucket_count(1024, 10) == 1
+    assert gq.gq_bucket_count(1025, 10) == 2
+    assert gq.gq_bucket_count(25_557_032, 17) == -(-25_557_032 // (1 << 17))
+    assert gq.gq_bucket_count(1 << 30, 30) == 1
+    for bad in (6, 31, -1):
+        with pytest.raises(gq.GQError):
+            gq.gq_bucket_count(100, bad)
+    c = cfg(gq)
+    for W, d, b in ((8, 25_557_032, 17), (1, 100, 7), (8, 1 << 30, 12), (40, 8192, 10)):
+        n = gq.gq_bucket_workspace_bytes(c, W, d, b)
+        chunks = -(-d // (1 << min(b, 12)))
+        assert n >= 256 + W * chunks * 12
+        assert n >= gq.gq_workspace_bytes(c, W, d)  # also a valid global-path workspace
+        assert n % 256 == 0
+
+
+def test_bucket_entry_points_reject_before_launch(gq):
+    lib = gq.lib()
+    c = cfg(gq, s=15, bits=5, wire="int8").c()
+    P = ctypes.c_void_p
+    good = P(0x10000000)
+    odd = P(0x10000004)
+    assert lib.gq_bucket_scales(good, None, 4, 4096, 6, ctypes.byref(c), good, good, None) == \
+        gq.GQ_ERR_ARG
+    assert lib.gq_bucket_scales(odd, None, 4, 4096, 10, ctypes.byref(c), good, good, None) == \
+        gq.GQ_ERR_ALIGN
+    assert lib.gq_bucket_scales(good, None, 4, 4096, 10, ctypes.byref(c), None, good, None) == \
+        gq.GQ_ERR_ARG
+    assert lib.gq_quantize_aggregate_bucketed(good, None, 9, 4096, 10, ctypes.byref(c), good,
+                                              good, good, good, good, None) == \
+        gq.GQ_ERR_OVERFLOW
+    cef = cfg(gq, s=15, bits=5, wire="int8", ef=True).c()
+    assert lib.gq_step_bucketed(good, None, 4, 4096, 10, ctypes.byref(cef), good, good, good,
+                                good, good, None) == gq.GQ_ERR_ARG
+    clog = cfg(gq, levels="log", alpha=10.0).c()
+    assert lib.gq_step_bucketed(good, None, 4, 4096, 10, ctypes.byref(clog), good, good, good,
+                                good, good, None) == gq.GQ_ERR_ARG

@@ -162,3 +162,59 @@ def check_blocks_one(gq, oracle, cfg, gs, es, buf, b):
     e_ref = oracle.error_feedback(gh, eh, codes, S=S, **kw)
     assert np.array_equal(buf.e[:, j0:j0 + 128].cpu().numpy().view(np.uint32),
                           e_ref.view(np.uint32)), b
+
+
+@pytest.mark.parametrize("b", [12, 17])
+def test_full_size_bucketed(gq, oracle, b):
+    """The benchmark workload with one scale per bucket of 2^b coordinates:
+    sampled whole buckets (first, last (ragged) and a few between) against the
+    oracle's bucket composition on the bucket's coordinates alone."""
+    name = "resnet50_t3_w8"
+    wl = synthetic.WORKLOADS[name]
+    cfg = config_of(gq, wl)
+    g = synthetic.workload_gradients(name, device="cuda")
+    W, d = g.shape
+    nk = gq.gq_bucket_count(d, b)
+    table = torch.empty(3 * nk, dtype=torch.float32, device="cuda")
+    ws = torch.empty(gq.gq_bucket_workspace_bytes(cfg, W, d, b), dtype=torch.uint8,
+                     device="cuda")
+    gq.gq_workspace_init(ws)
+    buf = gq.StepBuffers(cfg, W, d)
+    gq.gq_step_bucketed(g, None, b, cfg, table, buf.codes, buf.sum, buf.out, ws)
+    assert gq.gq_get_device_status(ws) == gq.GQ_OK
+    t = table.cpu().numpy()
+    kw = dict(levels=0 if cfg.levels == "uniform" else 1, s=cfg.s, L=cfg.L,
+              scale_kind=0 if cfg.scale_kind == "l2" else 1)
+    rng = np.random.default_rng(b)
+    picks = sorted(set(rng.integers(0, nk, size=4).tolist()) | {0, nk - 1})
+    B = 1 << b
+    bb = 16 * cfg.bits
+    codes_gpu = buf.codes.view(W, -1, bb)
+    for k in picks:
+        j0, j1 = k * B, min(d, (k + 1) * B)
+        gs = g[:, j0:j1].cpu().numpy()
+        S_k = t[k]
+        ref_S = oracle.step_bucketed(gs, bucket=B, bits=None, **kw)["S"][0]
+        if kw["scale_kind"] == 0:
+            assert abs(float(S_k) - float(ref_S)) <= 1e-5 * float(ref_S), k
+        else:
+            assert S_k == ref_S, k
+        codes = oracle.quantize(gs, seed=cfg.seed, step=cfg.step, S=S_k,
+                                js=np.arange(j0, j1, dtype=np.int64),
+                                levels=kw["levels"], s=cfg.s, L=cfg.L)
+        blk0, blk1 = j0 // 128, -(-j1 // 128)
+        packed = oracle.pack(codes, cfg.bits)
+        got = codes_gpu[:, blk0:blk1, :].cpu().numpy().reshape(W, -1)
+        if not np.array_equal(got, packed):
+            mine = oracle.unpack(got, W, j1 - j0, cfg.bits)
+            w, j = np.nonzero(mine != codes)
+            raise AssertionError(
+                f"bucket {k}: {w.size} codes differ; S_k={S_k!r} a_k={t[nk + k]!r} "
+                f"oracle a={oracle.uniform_multiplier(cfg.s, S_k)!r}; first (w, j, v, gpu, "
+                f"oracle): {[(int(a), int(b) + j0, float(gs[a, b]), int(mine[a, b]), int(codes[a, b])) for a, b in zip(w[:6], j[:6])]}")
+        total = oracle.aggregate(codes, levels=kw["levels"], L=cfg.L)
+        assert np.array_equal(buf.sum[j0:j1].cpu().numpy().astype(np.int32), total), k
+        out = oracle.decode_mean(total, W, levels=kw["levels"], s=cfg.s, L=cfg.L, S=S_k)
+        assert np.array_equal(buf.out[j0:j1].cpu().numpy().view(np.uint32), out.view(np.uint32))
+    del g, buf, table, ws
+    torch.cuda.empty_cache()

@@ -251,3 +251,31 @@ def test_bounded_wait_reports_timeout_and_context_survives(gq):
     g = synthetic.make_gradients(8, 100000, "normal", seed=1, device="cuda")
     gq.gq_step_fused(g, None, cfg, buf.scale, buf.norms, buf.codes, buf.sum, buf.out, buf.ws)
     assert gq.gq_get_device_status(buf.ws) == gq.GQ_OK
+
+
+@pytest.mark.parametrize("d", [4000, 4001])
+def test_rounding_decision_boundaries(gq, oracle, d):
+    """Inputs placed a fraction of an ulp from the round-up boundary u = 1 - p
+    (both sides, and on it), with S = s so the multiplier is exactly 1: the
+    GPU's codes are floor(r + u) exactly, like the oracle's."""
+    s, seed, step = 15, 7, 1
+    cfg = gq.GQConfig(s=s, bits=5, wire="int8", seed=seed, step=step)
+    v = np.zeros(d, np.float32)
+    n = 0
+    for j in range(d):
+        f = oracle.uniform_bits(seed, 0, step, 0, j)
+        if (1 << 20) <= f < (1 << 21):
+            u = f / float(1 << 23)
+            v[j] = -(u + 2.0 ** -26) if n % 3 == 0 else (-(u - 2.0 ** -26) if n % 3 == 1 else -u)
+            n += 1
+    assert n > 300
+    g = torch.from_numpy(v[None, :]).cuda()
+    scale = torch.tensor([float(s)], dtype=torch.float32, device="cuda")
+    codes = torch.empty((1, gq.gq_packed_row_bytes(cfg, d)), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(gq.gq_workspace_bytes(cfg, 1, d), dtype=torch.uint8, device="cuda")
+    gq.gq_workspace_init(ws)
+    gq.gq_quantize_pack(g, None, cfg, scale, codes, ws)
+    assert gq.gq_get_device_status(ws) == gq.GQ_OK
+    ref = oracle.quantize(v[None, :], s=s, seed=seed, step=step, S=np.float32(s))
+    assert (ref == -1).sum() >= 100
+    assert np.array_equal(codes.cpu().numpy(), oracle.pack(ref, 5))
