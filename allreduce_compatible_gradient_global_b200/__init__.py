@@ -107,6 +107,13 @@ def _load():
         "gq_bucket_scales": ([P, P, I, LL, I, CP, P, P, P], I),
         "gq_quantize_aggregate_bucketed": ([P, P, I, LL, I, CP, P, P, P, P, P, P], I),
         "gq_step_bucketed": ([P, P, I, LL, I, CP, P, P, P, P, P, P], I),
+        "gq_psgd_workspace_bytes": ([I, I, P, P, I, ctypes.POINTER(ctypes.c_size_t)], I),
+        "gq_psgd_project": ([P, P, I, I, P, P, I, I, P, P, P, P], I),
+        "gq_psgd_orthonormalize": ([P, I, P, I, P], I),
+        "gq_psgd_back_project": ([P, P, I, I, P, P, I, P, P, P], I),
+        "gq_psgd_mean": ([P, P, LL, I, P], I),
+        "gq_psgd_reconstruct": ([P, P, I, P, P, I, P, P], I),
+        "gq_lqsgd_step": ([P, P, I, I, P, P, I, I, CP, P, P, P, P, P], I),
         "gq_logq_quantize": ([P, I, I, P, P, CP, P, P, P, P], I),
         "gq_logq_decode_sum": ([P, P, I, I, P, P, CP, P, P], I),
     }
@@ -400,6 +407,98 @@ def gq_step_bucketed(g, e, bucket_log2, cfg: GQConfig, table, codes, sum_out, ou
     _check(lib().gq_step_bucketed(_ptr(g), _ptr(e), W, d, int(bucket_log2), ctypes.byref(c),
                                   _ptr(table), _ptr(codes), _ptr(sum_out), _ptr(out), _ptr(ws),
                                   _stream(stream)), "gq_step_bucketed")
+
+
+# ------------------------------------------------------------------ PowerSGD + LQ
+class PsgdShapes:
+    """The matrices of one worker: rows[l] x cols[l], and the rank."""
+
+    def __init__(self, rows, cols, rank):
+        if len(rows) != len(cols):
+            raise ValueError("rows and cols differ in length")
+        self.rows = [int(x) for x in rows]
+        self.cols = [int(x) for x in cols]
+        self.rank = int(rank)
+        self._r = (ctypes.c_int * len(self.rows))(*self.rows)
+        self._c = (ctypes.c_int * len(self.cols))(*self.cols)
+
+    @property
+    def nmats(self):
+        return len(self.rows)
+
+    @property
+    def total(self):
+        return sum(n * m for n, m in zip(self.rows, self.cols))
+
+    @property
+    def ptotal(self):
+        return sum(self.rows) * self.rank
+
+    @property
+    def qtotal(self):
+        return sum(self.cols) * self.rank
+
+
+def gq_psgd_workspace_bytes(W: int, sh: PsgdShapes) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().gq_psgd_workspace_bytes(int(W), sh.nmats, sh._r, sh._c, sh.rank,
+                                         ctypes.byref(out)), "gq_psgd_workspace_bytes")
+    return out.value
+
+
+def gq_psgd_project(g, m, sh: PsgdShapes, have_prev, p_prev, q, pw, stream=None):
+    W = int(g.shape[0])
+    _need(g, torch.float32, (W, sh.total), "g")
+    _need(m, torch.float32, (W, sh.total), "m")
+    _need(p_prev, torch.float32, (sh.ptotal,), "p_prev")
+    _need(q, torch.float32, (sh.qtotal,), "q")
+    _need(pw, torch.float32, (W, sh.ptotal), "pw")
+    _check(lib().gq_psgd_project(_ptr(g), _ptr(m), W, sh.nmats, sh._r, sh._c, sh.rank,
+                                 1 if have_prev else 0, _ptr(p_prev), _ptr(q), _ptr(pw),
+                                 _stream(stream)), "gq_psgd_project")
+
+
+def gq_psgd_orthonormalize(p, sh: PsgdShapes, stream=None):
+    _need(p, torch.float32, (sh.ptotal,), "p")
+    _check(lib().gq_psgd_orthonormalize(_ptr(p), sh.nmats, sh._r, sh.rank, _stream(stream)),
+           "gq_psgd_orthonormalize")
+
+
+def gq_psgd_back_project(m, p, sh: PsgdShapes, qw, ws, stream=None):
+    W = int(m.shape[0])
+    _need(m, torch.float32, (W, sh.total), "m")
+    _need(p, torch.float32, (sh.ptotal,), "p")
+    _need(qw, torch.float32, (W, sh.qtotal), "qw")
+    _check(lib().gq_psgd_back_project(_ptr(m), _ptr(p), W, sh.nmats, sh._r, sh._c, sh.rank,
+                                      _ptr(qw), _ptr(ws), _stream(stream)), "gq_psgd_back_project")
+
+
+def gq_psgd_mean(sum_in, out, W, stream=None):
+    _need(sum_in, torch.float32, None, "sum")
+    _need(out, torch.float32, tuple(sum_in.shape), "out")
+    _check(lib().gq_psgd_mean(_ptr(sum_in), _ptr(out), sum_in.numel(), int(W), _stream(stream)),
+           "gq_psgd_mean")
+
+
+def gq_psgd_reconstruct(p, q, sh: PsgdShapes, ghat, stream=None):
+    _need(p, torch.float32, (sh.ptotal,), "p")
+    _need(q, torch.float32, (sh.qtotal,), "q")
+    _need(ghat, torch.float32, (sh.total,), "ghat")
+    _check(lib().gq_psgd_reconstruct(_ptr(p), _ptr(q), sh.nmats, sh._r, sh._c, sh.rank,
+                                     _ptr(ghat), _stream(stream)), "gq_psgd_reconstruct")
+
+
+def gq_lqsgd_step(g, m, sh: PsgdShapes, have_prev, cfg: GQConfig, p, q, ghat, ws, stream=None):
+    W = int(g.shape[0])
+    _need(g, torch.float32, (W, sh.total), "g")
+    _need(m, torch.float32, (W, sh.total), "m")
+    _need(p, torch.float32, (sh.ptotal,), "p")
+    _need(q, torch.float32, (sh.qtotal,), "q")
+    _need(ghat, torch.float32, (sh.total,), "ghat")
+    c = cfg.c()
+    _check(lib().gq_lqsgd_step(_ptr(g), _ptr(m), W, sh.nmats, sh._r, sh._c, sh.rank,
+                               1 if have_prev else 0, ctypes.byref(c), _ptr(p), _ptr(q),
+                               _ptr(ghat), _ptr(ws), _stream(stream)), "gq_lqsgd_step")
 
 
 # ------------------------------------------------------------------ buffers

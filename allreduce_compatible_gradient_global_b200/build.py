@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libgq.so")
 
-SOURCES = ["gq_api.cu", "gq_kernels.cu", "gq_quant_tma.cu", "gq_bucket.cu", "gq_logq.cu", "gq_noalloc.cu"]
+SOURCES = ["gq_api.cu", "gq_kernels.cu", "gq_quant_tma.cu", "gq_bucket.cu", "gq_psgd.cu", "gq_logq.cu", "gq_noalloc.cu"]
 HEADERS = ["gq_device.cuh", "gq_internal.h"]
 
 NVCC_FLAGS = [

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "gq_api.h"
 #include "gq_internal.h"
@@ -622,6 +623,301 @@ GQ_API int gq_step_bucketed(const float* g_dev, float* e_dev, int W, long long d
     if (rc) return rc;
     return gq_quantize_aggregate_bucketed(g_dev, e_dev, W, d, bucket_log2, cfg, table_dev,
                                           codes_dev, sum_dev, out_dev, ws_dev, stream);
+}
+
+// ---------------------------------------------------------------------------
+// PowerSGD low-rank step (LQ-SGD)
+// ---------------------------------------------------------------------------
+namespace {
+
+// The back projection splits each matrix's rows into chunks so that the whole
+// launch has about this many tiles; a constant (not the SM count) so that the
+// summation order, and hence Q, is the same on every device.
+constexpr long long kBackTargetTiles = 2368;
+
+struct PsgdShape {
+    int nmats = 0, rank = 0, W = 0, max_rows = 0, chunk_rows = 0, chunks_max = 0;
+    const int* rows = nullptr;
+    const int* cols = nullptr;
+    long long total = 0, ptotal = 0, qtotal = 0;
+    bool vec = true;
+};
+
+int psgd_shape(int W, int nmats, const int* rows, const int* cols, int rank, PsgdShape& s) {
+    if (W < 1 || nmats < 1 || nmats > 4096 || !rows || !cols || rank < 1 || rank > 8)
+        return GQ_ERR_ARG;
+    s.W = W;
+    s.nmats = nmats;
+    s.rows = rows;
+    s.cols = cols;
+    s.rank = rank;
+    for (int l = 0; l < nmats; ++l) {
+        if (rows[l] < 1 || cols[l] < 1) return GQ_ERR_ARG;
+        s.total += (long long)rows[l] * cols[l];
+        s.ptotal += (long long)rows[l] * rank;
+        s.qtotal += (long long)cols[l] * rank;
+        if (cols[l] % 4) s.vec = false;
+        if (rows[l] > s.max_rows) s.max_rows = rows[l];
+    }
+    const int ct = s.vec ? 1024 : 256;
+    int chunk = 4096;
+    auto tiles = [&](int ch) {
+        long long t = 0;
+        for (int l = 0; l < nmats; ++l)
+            t += (long long)W * ((cols[l] + ct - 1) / ct) * ((rows[l] + ch - 1) / ch);
+        return t;
+    };
+    while (chunk > 128 && tiles(chunk) < kBackTargetTiles) chunk >>= 1;
+    s.chunk_rows = chunk;
+    s.chunks_max = (s.max_rows + chunk - 1) / chunk;
+    return GQ_OK;
+}
+
+// Workspace of the whole step: header, then each region 256-byte aligned.
+struct PsgdWs {
+    size_t pw, codes_p, max_p, qpart, qw, codes_q, max_q, qsum, end;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+PsgdWs psgd_ws(const PsgdShape& s) {
+    PsgdWs o;
+    size_t at = kWorkspaceHeader;
+    o.pw = at;
+    at = up256(at + (size_t)s.W * s.ptotal * sizeof(float));
+    o.codes_p = at;
+    at = up256(at + (size_t)s.W * s.ptotal);
+    o.max_p = at;
+    at = up256(at + (size_t)s.W * s.nmats * sizeof(float));
+    o.qpart = at;
+    at = up256(at + (size_t)s.chunks_max * s.W * s.qtotal * sizeof(float));
+    o.qw = at;
+    at = up256(at + (size_t)s.W * s.qtotal * sizeof(float));
+    o.codes_q = at;
+    at = up256(at + (size_t)s.W * s.qtotal);
+    o.max_q = at;
+    at = up256(at + (size_t)s.W * s.nmats * sizeof(float));
+    o.qsum = at;
+    at = up256(at + (size_t)s.qtotal * sizeof(float));
+    o.end = at;
+    return o;
+}
+
+enum class PsgdTiles { Project, Back, Reduce, Reconstruct };
+
+// Fill the matrices l0 .. l0 + count - 1 and their work-tile prefix.
+void psgd_group(PsgdArgs& a, const PsgdShape& s, int l0, int count, PsgdTiles kind) {
+    long long goff = 0, poff = 0, qoff = 0;
+    for (int l = 0; l < l0; ++l) {
+        goff += (long long)s.rows[l] * s.cols[l];
+        poff += (long long)s.rows[l] * s.rank;
+        qoff += (long long)s.cols[l] * s.rank;
+    }
+    a.count = count;
+    a.tile0[0] = 0;
+    for (int i = 0; i < count; ++i) {
+        const int n = s.rows[l0 + i], m = s.cols[l0 + i];
+        a.rows[i] = n;
+        a.cols[i] = m;
+        a.goff[i] = goff;
+        a.poff[i] = poff;
+        a.qoff[i] = qoff;
+        goff += (long long)n * m;
+        poff += (long long)n * s.rank;
+        qoff += (long long)m * s.rank;
+        long long tiles = 0;
+        switch (kind) {
+            case PsgdTiles::Project: tiles = (long long)s.W * ((n + 15) / 16); break;
+            case PsgdTiles::Back: {
+                const int ct = s.vec ? 1024 : 256;
+                tiles = (long long)s.W * ((m + ct - 1) / ct) *
+                        ((n + s.chunk_rows - 1) / s.chunk_rows);
+                break;
+            }
+            case PsgdTiles::Reduce:
+                tiles = (long long)s.W * (((long long)m * s.rank + 255) / 256);
+                break;
+            case PsgdTiles::Reconstruct: tiles = (n + 7) / 8; break;
+        }
+        a.tile0[i + 1] = a.tile0[i] + tiles;
+    }
+}
+
+void psgd_common(PsgdArgs& a, const PsgdShape& s) {
+    std::memset(&a, 0, sizeof(a));
+    a.total = s.total;
+    a.ptotal = s.ptotal;
+    a.qtotal = s.qtotal;
+    a.W = s.W;
+    a.rank = s.rank;
+    a.chunk_rows = s.chunk_rows;
+}
+
+}  // namespace
+
+GQ_API int gq_psgd_workspace_bytes(int W, int nmats, const int* rows_host, const int* cols_host,
+                                   int rank, size_t* bytes) {
+    if (!bytes) return GQ_ERR_ARG;
+    PsgdShape s;
+    int rc = psgd_shape(W, nmats, rows_host, cols_host, rank, s);
+    if (rc) return rc;
+    *bytes = psgd_ws(s).end;
+    return GQ_OK;
+}
+
+GQ_API int gq_psgd_project(const float* g_dev, float* m_dev, int W, int nmats,
+                           const int* rows_host, const int* cols_host, int rank, int have_prev,
+                           const float* p_prev_dev, const float* q_dev, float* pw_dev,
+                           cudaStream_t stream) {
+    PsgdShape s;
+    int rc = psgd_shape(W, nmats, rows_host, cols_host, rank, s);
+    if (rc) return rc;
+    if (!g_dev || !m_dev || !q_dev || !pw_dev || (have_prev && !p_prev_dev)) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || !aligned16(m_dev) || !aligned16(q_dev) || !aligned16(pw_dev) ||
+        (have_prev && !aligned16(p_prev_dev)))
+        return GQ_ERR_ALIGN;
+    PsgdArgs a;
+    psgd_common(a, s);
+    a.g = g_dev;
+    a.m = m_dev;
+    a.p = have_prev ? p_prev_dev : nullptr;
+    a.q = q_dev;
+    a.pw = pw_dev;
+    a.have_prev = have_prev ? 1 : 0;
+    for (int l0 = 0; l0 < nmats; l0 += kPsgdGroup) {
+        const int count = nmats - l0 < kPsgdGroup ? nmats - l0 : kPsgdGroup;
+        psgd_group(a, s, l0, count, PsgdTiles::Project);
+        if ((rc = cuda_status(launch_psgd_project(a, s.vec, sm_count(), stream)))) return rc;
+    }
+    return GQ_OK;
+}
+
+GQ_API int gq_psgd_orthonormalize(float* p_dev, int nmats, const int* rows_host, int rank,
+                                  cudaStream_t stream) {
+    if (!rows_host) return GQ_ERR_ARG;
+    std::vector<int> ones((size_t)(nmats > 0 && nmats <= 4096 ? nmats : 1), 4);
+    PsgdShape s;
+    int rc = psgd_shape(1, nmats, rows_host, ones.data(), rank, s);
+    if (rc) return rc;
+    if (!p_dev) return GQ_ERR_ARG;
+    if (!aligned16(p_dev)) return GQ_ERR_ALIGN;
+    PsgdArgs a;
+    psgd_common(a, s);
+    a.psum = p_dev;
+    for (int l0 = 0; l0 < nmats; l0 += kPsgdGroup) {
+        const int count = nmats - l0 < kPsgdGroup ? nmats - l0 : kPsgdGroup;
+        psgd_group(a, s, l0, count, PsgdTiles::Project);
+        if ((rc = cuda_status(launch_psgd_orth(a, stream)))) return rc;
+    }
+    return GQ_OK;
+}
+
+GQ_API int gq_psgd_back_project(const float* m_dev, const float* p_dev, int W, int nmats,
+                                const int* rows_host, const int* cols_host, int rank,
+                                float* qw_dev, void* ws_dev, cudaStream_t stream) {
+    PsgdShape s;
+    int rc = psgd_shape(W, nmats, rows_host, cols_host, rank, s);
+    if (rc) return rc;
+    if (!m_dev || !p_dev || !qw_dev || !ws_dev) return GQ_ERR_ARG;
+    if (!aligned16(m_dev) || !aligned16(p_dev) || !aligned16(qw_dev) || !aligned16(ws_dev))
+        return GQ_ERR_ALIGN;
+    const PsgdWs o = psgd_ws(s);
+    PsgdArgs a;
+    psgd_common(a, s);
+    a.m = const_cast<float*>(m_dev);
+    a.p = p_dev;
+    a.qpart = reinterpret_cast<float*>(static_cast<char*>(ws_dev) + o.qpart);
+    a.qw = qw_dev;
+    for (int l0 = 0; l0 < nmats; l0 += kPsgdGroup) {
+        const int count = nmats - l0 < kPsgdGroup ? nmats - l0 : kPsgdGroup;
+        psgd_group(a, s, l0, count, PsgdTiles::Back);
+        if ((rc = cuda_status(launch_psgd_back(a, s.vec, sm_count(), stream)))) return rc;
+        psgd_group(a, s, l0, count, PsgdTiles::Reduce);
+        if ((rc = cuda_status(launch_psgd_back_reduce(a, sm_count(), stream)))) return rc;
+    }
+    return GQ_OK;
+}
+
+GQ_API int gq_psgd_mean(const float* sum_dev, float* out_dev, long long n, int W,
+                        cudaStream_t stream) {
+    if (!sum_dev || !out_dev || n < 0 || W < 1) return GQ_ERR_ARG;
+    if (!aligned4(sum_dev) || !aligned4(out_dev)) return GQ_ERR_ALIGN;
+    if (n == 0) return GQ_OK;
+    return cuda_status(launch_psgd_mean(sum_dev, out_dev, n, W, sm_count(), stream));
+}
+
+GQ_API int gq_psgd_reconstruct(const float* p_dev, const float* q_dev, int nmats,
+                               const int* rows_host, const int* cols_host, int rank,
+                               float* ghat_dev, cudaStream_t stream) {
+    PsgdShape s;
+    int rc = psgd_shape(1, nmats, rows_host, cols_host, rank, s);
+    if (rc) return rc;
+    if (!p_dev || !q_dev || !ghat_dev) return GQ_ERR_ARG;
+    if (!aligned16(p_dev) || !aligned16(q_dev) || !aligned16(ghat_dev)) return GQ_ERR_ALIGN;
+    PsgdArgs a;
+    psgd_common(a, s);
+    a.p = p_dev;
+    a.q = q_dev;
+    a.out = ghat_dev;
+    for (int l0 = 0; l0 < nmats; l0 += kPsgdGroup) {
+        const int count = nmats - l0 < kPsgdGroup ? nmats - l0 : kPsgdGroup;
+        psgd_group(a, s, l0, count, PsgdTiles::Reconstruct);
+        if ((rc = cuda_status(launch_psgd_reconstruct(a, s.vec, sm_count(), stream)))) return rc;
+    }
+    return GQ_OK;
+}
+
+GQ_API int gq_lqsgd_step(const float* g_dev, float* m_dev, int W, int nmats,
+                         const int* rows_host, const int* cols_host, int rank, int have_prev,
+                         const gq_config* cfg, float* p_dev, float* q_dev, float* ghat_dev,
+                         void* ws_dev, cudaStream_t stream) {
+    if (!cfg || cfg->levels != GQ_LOG || !(cfg->alpha > 0.f) || !(cfg->alpha <= 3.0e38f))
+        return GQ_ERR_ARG;
+    PsgdShape s;
+    int rc = psgd_shape(W, nmats, rows_host, cols_host, rank, s);
+    if (rc) return rc;
+    if (!g_dev || !m_dev || !p_dev || !q_dev || !ws_dev) return GQ_ERR_ARG;
+    if (!aligned16(g_dev) || !aligned16(m_dev) || !aligned16(p_dev) || !aligned16(q_dev) ||
+        !aligned16(ws_dev) || (ghat_dev && !aligned16(ghat_dev)))
+        return GQ_ERR_ALIGN;
+    const PsgdWs o = psgd_ws(s);
+    char* ws = static_cast<char*>(ws_dev);
+    float* pw = reinterpret_cast<float*>(ws + o.pw);
+    float* qw = reinterpret_cast<float*>(ws + o.qw);
+    float* qsum = reinterpret_cast<float*>(ws + o.qsum);
+    signed char* codes_p = reinterpret_cast<signed char*>(ws + o.codes_p);
+    signed char* codes_q = reinterpret_cast<signed char*>(ws + o.codes_q);
+    float* max_p = reinterpret_cast<float*>(ws + o.max_p);
+    float* max_q = reinterpret_cast<float*>(ws + o.max_q);
+    std::vector<int> ranks((size_t)nmats, rank);
+    gq_config c = *cfg;
+    // P_w = M_w Q (with the deferred error), then its log-quantized sum
+    rc = gq_psgd_project(g_dev, m_dev, W, nmats, rows_host, cols_host, rank, have_prev, p_dev,
+                         q_dev, pw, stream);
+    if (rc) return rc;
+    c.step = 2u * cfg->step;
+    rc = gq_logq_quantize(pw, W, nmats, rows_host, ranks.data(), &c, max_p, codes_p, ws_dev,
+                          stream);
+    if (rc) return rc;
+    rc = gq_logq_decode_sum(codes_p, max_p, W, nmats, rows_host, ranks.data(), &c, p_dev, stream);
+    if (rc) return rc;
+    rc = gq_psgd_orthonormalize(p_dev, nmats, rows_host, rank, stream);
+    if (rc) return rc;
+    // Q_w = M_w^T P_hat, its log-quantized sum, and the mean
+    rc = gq_psgd_back_project(m_dev, p_dev, W, nmats, rows_host, cols_host, rank, qw, ws_dev,
+                              stream);
+    if (rc) return rc;
+    c.step = 2u * cfg->step + 1u;
+    rc = gq_logq_quantize(qw, W, nmats, cols_host, ranks.data(), &c, max_q, codes_q, ws_dev,
+                          stream);
+    if (rc) return rc;
+    rc = gq_logq_decode_sum(codes_q, max_q, W, nmats, cols_host, ranks.data(), &c, qsum, stream);
+    if (rc) return rc;
+    rc = gq_psgd_mean(qsum, q_dev, s.qtotal, W, stream);
+    if (rc) return rc;
+    if (ghat_dev)
+        rc = gq_psgd_reconstruct(p_dev, q_dev, nmats, rows_host, cols_host, rank, ghat_dev, stream);
+    return rc;
 }
 
 }  // extern "C"

@@ -515,6 +515,85 @@ def run_buckets(args):
             "peak_source": peak_kind, "workload": args.workload, "W": W, "d": d, "rows": rows}
 
 
+def run_lqsgd(args):
+    """The whole LQ-SGD step (PowerSGD low rank + log quantizer on both
+    factors, error feedback) on W = 8 workers x 24 matrices of 4096 x 4096,
+    ranks 1, 4, 7: step time through gq_lqsgd_step, and the two passes over
+    the matrices (gq_psgd_project, gq_psgd_back_project) timed alone against
+    their algorithmic bytes."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = measured_hbm_peak()
+    wl = synthetic.LQ_WORKLOAD
+    W, L, n, m = wl["W"], wl["pairs"], wl["n"], wl["m"]
+    K = max(5, min(args.steps, 20))
+    rows_out = []
+    g = None
+    for r in wl["ranks"]:
+        sh = gq.PsgdShapes([n] * L, [m] * L, r)
+        if g is None:
+            g = synthetic.make_gradients(W, sh.total, "normal", seed=synthetic.seed_for(5),
+                                         device="cuda")
+            mst = torch.zeros_like(g)
+        else:
+            mst.zero_()
+        p = torch.zeros(sh.ptotal, dtype=torch.float32, device="cuda")
+        q = synthetic.make_gradients(1, sh.qtotal, "normal", seed=r, device="cuda")[0]
+        ghat = torch.empty(sh.total, dtype=torch.float32, device="cuda")
+        pw = torch.empty((W, sh.ptotal), dtype=torch.float32, device="cuda")
+        qw = torch.empty((W, sh.qtotal), dtype=torch.float32, device="cuda")
+        ws = torch.empty(gq.gq_psgd_workspace_bytes(W, sh), dtype=torch.uint8, device="cuda")
+        gq.gq_workspace_init(ws)
+        cfg = gq.GQConfig(levels="log", alpha=wl["alpha"], seed=1)
+        for i in range(3):
+            cfg.step = i
+            gq.gq_lqsgd_step(g, mst, sh, i > 0, cfg, p, q, ghat, ws, stream)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for i in range(K):
+            cfg.step = 3 + i
+            gq.gq_lqsgd_step(g, mst, sh, True, cfg, p, q, ghat, ws, stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        if gq.gq_get_device_status(ws, stream) != gq.GQ_OK:
+            raise RuntimeError("device flag raised in the LQ-SGD step")
+        step_ms = ev[0].elapsed_time(ev[1]) / K
+        pj, bk = [], []
+        for i in range(K):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            gq.gq_psgd_project(g, mst, sh, True, p, q, pw, stream)
+            e[1].record(stream)
+            gq.gq_psgd_back_project(mst, p, sh, qw, ws, stream)
+            e[2].record(stream)
+            pj.append(e)
+        torch.cuda.synchronize()
+        proj_ms = statistics.median(e[0].elapsed_time(e[1]) for e in pj)
+        back_ms = statistics.median(e[1].elapsed_time(e[2]) for e in pj)
+        wt = W * sh.total
+        proj_bytes = 12 * wt + 4 * W * sh.ptotal
+        back_bytes = 4 * wt
+        step_bytes = 16 * wt + 4 * sh.total
+        rows_out.append({
+            "rank": r, "step_ms": round(step_ms, 4),
+            "grad_gbs": round(4 * wt / (step_ms * 1e-3) / 1e9, 1),
+            "step_frac": round(step_bytes / (step_ms * 1e-3) / 1e9 / peak, 4),
+            "project_ms": round(proj_ms, 4),
+            "project_frac": round(proj_bytes / (proj_ms * 1e-3) / 1e9 / peak, 4),
+            "back_project_ms": round(back_ms, 4),
+            "back_project_frac": round(back_bytes / (back_ms * 1e-3) / 1e9 / peak, 4),
+            "wire_bytes_per_worker": (sh.ptotal + sh.qtotal),
+            "fp32_bytes_per_worker": 4 * sh.total})
+        del p, q, ghat, pw, qw, ws
+    del g, mst
+    torch.cuda.empty_cache()
+    return {"metric": "LQ-SGD step: fp32 gradient GB/s", "mode": "lqsgd", "unit": "GB/s",
+            "peak": peak, "peak_source": peak_kind, "W": W,
+            "matrices": f"{L} x {n}x{m} per worker", "rows": rows_out}
+
+
 def run_lq(args):
     """The LQ-SGD log quantizer: quantize + decode-sum of 24 factor pairs of
     4096 x r per worker, W = 8, r in {1, 4, 7}."""
@@ -575,6 +654,8 @@ def main():
                     help="one JSON line with the LQ-SGD log-quantizer timings")
     ap.add_argument("--buckets", action="store_true",
                     help="one JSON line comparing the global scale with per-bucket scales")
+    ap.add_argument("--lqsgd", action="store_true",
+                    help="one JSON line with the PowerSGD + log-quantizer step timings")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -587,9 +668,10 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
-    if args.sweep or args.lq or args.buckets:
+    if args.sweep or args.lq or args.buckets or args.lqsgd:
         if rank == 0:
-            fn = run_sweep if args.sweep else (run_lq if args.lq else run_buckets)
+            fn = (run_sweep if args.sweep else run_lq if args.lq else
+                  run_buckets if args.buckets else run_lqsgd)
             print(json.dumps(fn(args)), flush=True)
         return
 

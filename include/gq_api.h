@@ -305,6 +305,82 @@ GQ_API int gq_logq_decode_sum(const signed char* codes_dev, const float* maxabs_
                               int nmats, const int* rows_host, const int* cols_host,
                               const gq_config* cfg, float* out_dev, cudaStream_t stream);
 
+/* PowerSGD low-rank step with the log quantizer on both factors ("Trustworthy
+ * Efficient Communication for Distributed Learning using LQ-SGD Algorithm",
+ * review, "What carries the argument": G ~ P Q^T, P and Q log-quantized before
+ * their All-Reduce, error E_t = G'_t - Ghat_t added back next step; Desk
+ * Editor's Note, "What is actually new": both factors quantized, with
+ * orthonormalization and error feedback).  The low-rank step itself is
+ * PowerSGD's (Vogels et al., NeurIPS 2019, cited there).
+ *
+ * Shapes: each worker holds nmats matrices, matrix l being rows_host[l] x
+ * cols_host[l] (row-major, each >= 1), stored back to back: g and m are
+ * [W][sum n_l m_l] fp32.  rank r is 1..8; nmats is 1..4096.  P-shaped buffers
+ * hold the n_l x r factors back to back ([sum n_l r]), Q-shaped ones the
+ * m_l x r factors ([sum m_l r]); per-worker factors are [W][...] of those.
+ * All buffers 16-byte aligned.  When every m_l is a multiple of 4 the
+ * kernels use 128-bit accesses; otherwise scalar ones, same results.
+ *
+ * State kept by the caller between steps: m (the previous step's M_w), p
+ * (the previous P_hat) and q (the previous mean Q, also the warm start).
+ * Before the first step m holds the initial error (usually zeros), q a
+ * random start, and have_prev = 0.  The error of step t is never stored:
+ * E_w = M_w - P_hat Q^T is applied when the next step reads m, element by
+ * element as E = fl(M_prev - Ghat), M = fl(G + E) with
+ * Ghat_ij = fma chain over k = 0..r-1 of P_hat[i,k] Q[j,k] starting from 0,
+ * so the result is the same as storing E. */
+
+/* Workspace of gq_psgd_back_project and gq_lqsgd_step (header + factor
+ * scratch + back-projection partials); zero-fill it once (gq_workspace_init). */
+GQ_API int gq_psgd_workspace_bytes(int W, int nmats, const int* rows_host, const int* cols_host,
+                                   int rank, size_t* bytes);
+
+/* Pass 1: per worker and matrix, E = have_prev ? fl(m - Ghat(p_prev, q)) : m,
+ * M = fl(g + E) written back to m, and pw = M q ([W][sum n_l r]; each entry
+ * sums lane-strided fp32 partials in a fixed order).  p_prev is read only
+ * when have_prev. */
+GQ_API int gq_psgd_project(const float* g_dev, float* m_dev, int W, int nmats,
+                           const int* rows_host, const int* cols_host, int rank, int have_prev,
+                           const float* p_prev_dev, const float* q_dev, float* pw_dev,
+                           cudaStream_t stream);
+
+/* Modified Gram-Schmidt on the columns of each n_l x r factor of p_dev, in
+ * place: column k is divided by its norm (unless that is 0), then its
+ * component is removed from every later column; sums in fp64, fixed order. */
+GQ_API int gq_psgd_orthonormalize(float* p_dev, int nmats, const int* rows_host, int rank,
+                                  cudaStream_t stream);
+
+/* Pass 2: qw = M^T p per worker and matrix ([W][sum m_l r]), M read from
+ * m_dev.  Rows are split into chunks whose partial sums are added in chunk
+ * order; the chunking depends only on the shapes, so results are the same on
+ * every device. */
+GQ_API int gq_psgd_back_project(const float* m_dev, const float* p_dev, int W, int nmats,
+                                const int* rows_host, const int* cols_host, int rank,
+                                float* qw_dev, void* ws_dev, cudaStream_t stream);
+
+/* out[x] = fl(sum[x] / W) for x < n: the mean of an All-Reduce sum. */
+GQ_API int gq_psgd_mean(const float* sum_dev, float* out_dev, long long n, int W,
+                        cudaStream_t stream);
+
+/* Ghat = p q^T per matrix ([sum n_l m_l], one copy, not per worker), each
+ * entry the fma chain described above. */
+GQ_API int gq_psgd_reconstruct(const float* p_dev, const float* q_dev, int nmats,
+                               const int* rows_host, const int* cols_host, int rank,
+                               float* ghat_dev, cudaStream_t stream);
+
+/* One LQ-SGD step: gq_psgd_project; gq_logq_quantize of the P_w (uniform
+ * stream step 2*cfg->step) and gq_logq_decode_sum into p_dev (the summed P);
+ * gq_psgd_orthonormalize (p_dev becomes P_hat); gq_psgd_back_project;
+ * gq_logq_quantize of the Q_w (step 2*cfg->step + 1) and gq_logq_decode_sum;
+ * gq_psgd_mean into q_dev; and, if ghat_dev is not NULL,
+ * gq_psgd_reconstruct.  cfg: levels GQ_LOG, alpha, seed, step.  The P and Q
+ * calls draw different uniform streams, so the two factors never share
+ * one. */
+GQ_API int gq_lqsgd_step(const float* g_dev, float* m_dev, int W, int nmats,
+                         const int* rows_host, const int* cols_host, int rank, int have_prev,
+                         const gq_config* cfg, float* p_dev, float* q_dev, float* ghat_dev,
+                         void* ws_dev, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -55,6 +55,8 @@ def lib():
         L.gqo_logq_map.restype = f32
         L.gqo_logq_decode_one.argtypes = [i32, f32, f32]
         L.gqo_logq_decode_one.restype = f32
+        L.gqo_lowrank_fma.argtypes = [P, P, i64, i64, i32, P]
+        L.gqo_lowrank_fma.restype = None
         _lib = L
     return _lib
 
@@ -235,6 +237,17 @@ def step_bucketed(g, e=None, *, bucket, levels=UNIFORM, s=15, L=8, scale_kind=SC
             e_new[:, lo:hi] = error_feedback(gk, ek, ck, levels=levels, s=s, L=L, S=Sk)
     packed = pack(codes, bits) if bits else None
     return dict(S=S_ref, codes=codes, packed=packed, sum=total, out=out, e=e_new)
+
+
+def lowrank_fma(P, Q):
+    """P (n x r) Q^T (m x r) in float32 with the fma chain of gqo_lowrank_fma."""
+    P = _f32(P)
+    Q = _f32(Q)
+    n, r = P.shape
+    m = Q.shape[0]
+    out = np.zeros((n, m), np.float32)
+    lib().gqo_lowrank_fma(_p(P), _p(Q), n, m, r, _p(out))
+    return out
 
 
 def logq_quantize(x, sizes, *, alpha=10.0, seed=0, step=0):

@@ -503,3 +503,17 @@ int gqo_logq_decode_sum(const int8_t* codes, const float* maxabs, int W,
     }
     return 0;
 }
+
+/* PowerSGD's decompression Ghat = P Q^T ("Trustworthy Efficient Communication
+ * for Distributed Learning using LQ-SGD Algorithm", review, "What carries the
+ * argument": G ~ P Q^T), evaluated in the float32 order the library states. */
+void gqo_lowrank_fma(const float* P, const float* Q, int64_t n, int64_t m, int r,
+                     float* out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < m; ++j) {
+            float acc = 0.0f;
+            for (int k = 0; k < r; ++k) acc = fmaf(P[i * r + k], Q[j * r + k], acc);
+            out[i * m + j] = acc;
+        }
+}

@@ -141,6 +141,13 @@ int gqo_logq_decode_sum(const int8_t* codes, const float* maxabs, int W,
 float gqo_logq_map(float xn, float alpha);           /* log1p(a*xn)/log1p(a) */
 float gqo_logq_decode_one(int32_t k, float m, float alpha);
 
+/* The low-rank value P Q^T of one n x m matrix in float32 as the library
+ * states it: out[i*m + j] = acc_r with acc_0 = 0 and
+ * acc_{k+1} = fmaf(P[i*r + k], Q[j*r + k], acc_k) (one rounding per step).
+ * P is n x r, Q is m x r, both row-major. */
+void gqo_lowrank_fma(const float* P, const float* Q, int64_t n, int64_t m, int r,
+                     float* out);
+
 #ifdef __cplusplus
 }
 #endif

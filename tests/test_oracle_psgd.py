@@ -125,3 +125,30 @@ def test_log_quantizer_is_wired_in(psgd, oracle):
     qsizes = np.array([m * r for _, m in shapes])
     mx, codes = oracle.logq_quantize(lq["Qw"].astype(np.float32), qsizes, seed=5, step=7)
     assert np.array_equal(codes, lq["lqQ"]["codes"])
+
+
+def _round_f32(x):
+    """Exact round-to-nearest-even of a Fraction to float32."""
+    from fractions import Fraction
+    f = np.float32(float(x))
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    best = min(cands, key=lambda c: (abs(Fraction(float(c)) - x),
+                                     int(np.frombuffer(np.float32(c).tobytes(), np.uint32)[0]) & 1))
+    return np.float32(best)
+
+
+def test_lowrank_fma_is_a_chain_of_single_roundings(oracle):
+    """Each entry of the float32 low-rank value is acc <- round(p_k q_k + acc)
+    from acc = 0, every step one correct rounding of the exact value."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    P = (rng.standard_normal((6, 5)) * np.exp2(rng.integers(-20, 20, (6, 5)))).astype(np.float32)
+    Q = (rng.standard_normal((7, 5)) * np.exp2(rng.integers(-20, 20, (7, 5)))).astype(np.float32)
+    out = oracle.lowrank_fma(P, Q)
+    for i in range(6):
+        for j in range(7):
+            acc = np.float32(0)
+            for k in range(5):
+                acc = _round_f32(Fraction(float(P[i, k])) * Fraction(float(Q[j, k]))
+                                 + Fraction(float(acc)))
+            assert acc == out[i, j], (i, j)
