@@ -10,6 +10,7 @@
 
 #include "gq_api.h"
 #include "gq_internal.h"
+#include "gq_psgd.h"
 
 using namespace gq;
 

@@ -22,7 +22,7 @@
 // E = fl(M_prev - Ghat_ij), M = fl(G + E).
 #include <cfloat>
 
-#include "gq_internal.h"
+#include "gq_psgd.h"
 
 namespace gq {
 
