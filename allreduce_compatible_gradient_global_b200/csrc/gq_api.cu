@@ -632,9 +632,10 @@ GQ_API int gq_step_bucketed(const float* g_dev, float* e_dev, int W, long long d
 namespace {
 
 // The back projection splits each matrix's rows into chunks so that the whole
-// launch has about this many tiles; a constant (not the SM count) so that the
-// summation order, and hence Q, is the same on every device.
-constexpr long long kBackTargetTiles = 2368;
+// launch has at least this many tiles (about 8 waves of 4 resident blocks on
+// 148 SMs, so the last wave's tail stays small); a constant, not the SM count,
+// so that the summation order, and hence Q, is the same on every device.
+constexpr long long kBackTargetTiles = 4736;
 
 struct PsgdShape {
     int nmats = 0, rank = 0, W = 0, max_rows = 0, chunk_rows = 0, chunks_max = 0;

@@ -42,6 +42,31 @@ __device__ __forceinline__ int matrix_of(const PsgdArgs& a, long long t) {
     return lo;
 }
 
+// Per-lane asynchronous 16-byte copies global -> shared (bypassing L1), so
+// that several loads per lane stay in flight without holding registers.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Projection pass: pipeline depth and resident blocks per SM by rank.  Each
+// stage takes 16 KiB of shared memory per block; what is left of the 256 KiB
+// L1/shared array keeps Q (4r floats per column group, re-read by every row
+// pair) in L1: 64 KiB at r <= 4, 160 KiB at r >= 5.
+template <int R>
+struct ProjCfg {
+    static constexpr int stages = (R >= 3 && R <= 4) ? 4 : 3;
+    static constexpr int min_blocks = R <= 2 ? 4 : (R <= 4 ? 3 : 2);
+};
+constexpr int kBackStages = 8;  // per-thread pipeline depth of the back projection
+
 template <int R>
 __device__ __forceinline__ float lowrank_value(const float (&p)[R], const float* q) {
     float acc = 0.f;
@@ -56,8 +81,10 @@ __device__ __forceinline__ float lowrank_value(const float (&p)[R], const float*
 // P_w[i,k] sums lane-sequential partials, then a xor butterfly over the warp.
 // ---------------------------------------------------------------------------
 template <int R, bool HAVE_PREV, bool VEC>
-__global__ void __launch_bounds__(kPsgdThreads)
+__global__ void __launch_bounds__(kPsgdThreads, ProjCfg<R>::min_blocks)
     psgd_project_kernel(const __grid_constant__ PsgdArgs a) {
+    constexpr int kProjStages = ProjCfg<R>::stages;
+    extern __shared__ float4 psm[];  // VEC: kProjStages x 4 float4 per lane
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (long long t = blockIdx.x; t < a.tile0[a.count]; t += gridDim.x) {
         const int l = matrix_of(a, t);
@@ -86,8 +113,35 @@ __global__ void __launch_bounds__(kPsgdThreads)
 #pragma unroll
         for (int k = 0; k < R; ++k) acc0[k] = acc1[k] = 0.f;
         if (VEC) {
+            // lane-private ring of kProjStages slots, each {G row i0, M row i0,
+            // G row i0+1, M row i0+1} for one float4 column group
+            float4* ring = psm + (size_t)warp * kProjStages * 4 * 32;
+            const float4* gA4 = reinterpret_cast<const float4*>(g0);
+            const float4* mA4 = reinterpret_cast<const float4*>(m0);
+            const float4* gB4 = reinterpret_cast<const float4*>(g0 + m);
+            const float4* mB4 = reinterpret_cast<const float4*>(m0 + m);
             const int m4 = m >> 2;
-            for (int j4 = lane; j4 < m4; j4 += 32) {
+            const int nit = lane < m4 ? (m4 - lane + 31) / 32 : 0;
+            auto issue = [&](int it) {
+                const int j4 = lane + it * 32;
+                float4* d = ring + (it % kProjStages) * 128 + lane;
+                cp_async16(d, gA4 + j4);
+                cp_async16(d + 32, mA4 + j4);
+                if (two) {
+                    cp_async16(d + 64, gB4 + j4);
+                    cp_async16(d + 96, mB4 + j4);
+                }
+            };
+#pragma unroll
+            for (int it = 0; it < kProjStages - 1; ++it) {
+                if (it < nit) issue(it);
+                cp_async_commit();
+            }
+            for (int it = 0; it < nit; ++it) {
+                if (it + kProjStages - 1 < nit) issue(it + kProjStages - 1);
+                cp_async_commit();
+                cp_async_wait<kProjStages - 1>();  // this lane's copies of step `it` landed
+                const int j4 = lane + it * 32;
                 float q[4 * R];  // rows 4 j4 .. 4 j4 + 3 of Q, R values each
                 const float4* q4 = reinterpret_cast<const float4*>(qm + (long long)j4 * 4 * R);
 #pragma unroll
@@ -98,12 +152,12 @@ __global__ void __launch_bounds__(kPsgdThreads)
                     q[4 * k + 2] = v.z;
                     q[4 * k + 3] = v.w;
                 }
-                const float4 ga = __ldcs(reinterpret_cast<const float4*>(g0) + j4);
-                const float4 ma = __ldcs(reinterpret_cast<const float4*>(m0) + j4);
+                const float4* d = ring + (it % kProjStages) * 128 + lane;
+                const float4 ga = d[0], ma = d[32];
                 float4 gb = make_float4(0.f, 0.f, 0.f, 0.f), mb = gb;
                 if (two) {
-                    gb = __ldcs(reinterpret_cast<const float4*>(g0 + m) + j4);
-                    mb = __ldcs(reinterpret_cast<const float4*>(m0 + m) + j4);
+                    gb = d[64];
+                    mb = d[96];
                 }
                 const float gA[4] = {ga.x, ga.y, ga.z, ga.w}, mA[4] = {ma.x, ma.y, ma.z, ma.w};
                 const float gB[4] = {gb.x, gb.y, gb.z, gb.w}, mB[4] = {mb.x, mb.y, mb.z, mb.w};
@@ -130,6 +184,7 @@ __global__ void __launch_bounds__(kPsgdThreads)
                     __stcs(reinterpret_cast<float4*>(m0 + m) + j4,
                            make_float4(outB[0], outB[1], outB[2], outB[3]));
             }
+            cp_async_wait<0>();
         } else {
             for (int j = lane; j < m; j += 32) {
                 float q[R];
@@ -260,47 +315,47 @@ __global__ void __launch_bounds__(kPsgdThreads)
         if (VEC) {
             const int j = ct * kBackColsPerTile + 4 * threadIdx.x;
             if (j < m) {
+                // thread-private ring of kBackStages rows of this thread's float4
+                float4* ring = reinterpret_cast<float4*>(ps + (size_t)a.chunk_rows * RP);
+                const int nrow = r1 - r0;
+                const float* src = mrow + (long long)r0 * m + j;
+                auto issue = [&](int it) {
+                    cp_async16(ring + (it % kBackStages) * kPsgdThreads + threadIdx.x,
+                               src + (long long)it * m);
+                };
+#pragma unroll
+                for (int it = 0; it < kBackStages - 1; ++it) {
+                    if (it < nrow) issue(it);
+                    cp_async_commit();
+                }
                 float acc[4][R];
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
                     for (int k = 0; k < R; ++k) acc[cc][k] = 0.f;
-                int i = r0;
-                for (; i + 4 <= r1; i += 4) {
-                    float4 v[4];
+                for (int it = 0; it < nrow; ++it) {
+                    if (it + kBackStages - 1 < nrow) issue(it + kBackStages - 1);
+                    cp_async_commit();
+                    cp_async_wait<kBackStages - 1>();
+                    const float4 v = ring[(it % kBackStages) * kPsgdThreads + threadIdx.x];
+                    const float* pr = ps + it * RP;
+                    float pk[RP];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        v[u] = __ldcs(reinterpret_cast<const float4*>(mrow + (long long)(i + u) * m + j));
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float* pr = ps + (i + u - r0) * RP;
-                        float pk[RP];
-#pragma unroll
-                        for (int k4 = 0; k4 < RP / 4; ++k4) {
-                            const float4 pv = reinterpret_cast<const float4*>(pr)[k4];
-                            pk[4 * k4] = pv.x;
-                            pk[4 * k4 + 1] = pv.y;
-                            pk[4 * k4 + 2] = pv.z;
-                            pk[4 * k4 + 3] = pv.w;
-                        }
-                        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-                            for (int k = 0; k < R; ++k)
-                                acc[cc][k] = __fmaf_rn(vv[cc], pk[k], acc[cc][k]);
+                    for (int k4 = 0; k4 < RP / 4; ++k4) {
+                        const float4 pv = reinterpret_cast<const float4*>(pr)[k4];
+                        pk[4 * k4] = pv.x;
+                        pk[4 * k4 + 1] = pv.y;
+                        pk[4 * k4 + 2] = pv.z;
+                        pk[4 * k4 + 3] = pv.w;
                     }
-                }
-                for (; i < r1; ++i) {
-                    const float4 v = __ldcs(reinterpret_cast<const float4*>(mrow + (long long)i * m + j));
-                    const float* pr = ps + (i - r0) * RP;
                     const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
                         for (int k = 0; k < R; ++k)
-                            acc[cc][k] = __fmaf_rn(vv[cc], pr[k], acc[cc][k]);
+                            acc[cc][k] = __fmaf_rn(vv[cc], pk[k], acc[cc][k]);
                 }
+                cp_async_wait<0>();
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
@@ -401,27 +456,45 @@ static int grid_for(long long tiles, int sms, int per_sm) {
     return g < 1 ? 1 : (int)g;
 }
 
+// One resident wave of the kernel (grid-stride over its tiles).
+static int resident_grid(const void* fn, size_t smem, long long tiles, int sms) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kPsgdThreads, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    return grid_for(tiles, sms, per_sm);
+}
+
 #define GQ_PSGD_RANKS(X) X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8)
 
+template <int R, bool HP, bool VEC>
+static cudaError_t project_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
+    auto kern = psgd_project_kernel<R, HP, VEC>;
+    const size_t smem = VEC ? (size_t)ProjCfg<R>::stages * 4 * kPsgdThreads * sizeof(float4) : 0;
+    if (VEC) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<resident_grid((const void*)kern, smem, a.tile0[a.count], sms), kPsgdThreads, smem,
+           st>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_psgd_project(const PsgdArgs& a, bool vec, int sms, cudaStream_t st) {
-    const int grid = grid_for(a.tile0[a.count], sms, 8);
     const bool hp = a.have_prev != 0;
-#define GQ_PROJ(RR)                                                                          \
-    case RR:                                                                                 \
-        if (hp) {                                                                            \
-            if (vec) psgd_project_kernel<RR, true, true><<<grid, kPsgdThreads, 0, st>>>(a);  \
-            else psgd_project_kernel<RR, true, false><<<grid, kPsgdThreads, 0, st>>>(a);     \
-        } else {                                                                             \
-            if (vec) psgd_project_kernel<RR, false, true><<<grid, kPsgdThreads, 0, st>>>(a); \
-            else psgd_project_kernel<RR, false, false><<<grid, kPsgdThreads, 0, st>>>(a);    \
-        }                                                                                    \
-        break;
+#define GQ_PROJ(RR)                                                           \
+    case RR:                                                                  \
+        if (hp) return vec ? project_inst<RR, true, true>(a, sms, st)         \
+                           : project_inst<RR, true, false>(a, sms, st);       \
+        return vec ? project_inst<RR, false, true>(a, sms, st)                \
+                   : project_inst<RR, false, false>(a, sms, st);
     switch (a.rank) {
         GQ_PSGD_RANKS(GQ_PROJ)
         default: return cudaErrorInvalidValue;
     }
 #undef GQ_PROJ
-    return cudaGetLastError();
 }
 
 cudaError_t launch_psgd_orth(const PsgdArgs& a, cudaStream_t st) {
@@ -435,33 +508,31 @@ cudaError_t launch_psgd_orth(const PsgdArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-size_t psgd_back_smem(int rank, int chunk_rows) {
-    return (size_t)chunk_rows * (size_t)((rank + 3) & ~3) * sizeof(float);
+size_t psgd_back_smem(int rank, int chunk_rows, bool vec) {
+    return (size_t)chunk_rows * (size_t)((rank + 3) & ~3) * sizeof(float) +
+           (vec ? (size_t)kBackStages * kPsgdThreads * sizeof(float4) : 0);
+}
+
+template <int R, bool VEC>
+static cudaError_t back_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
+    auto kern = psgd_back_kernel<R, VEC>;
+    const size_t smem = psgd_back_smem(R, a.chunk_rows, VEC);
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<resident_grid((const void*)kern, smem, a.tile0[a.count], sms), kPsgdThreads, smem,
+           st>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_psgd_back(const PsgdArgs& a, bool vec, int sms, cudaStream_t st) {
-    const size_t smem = psgd_back_smem(a.rank, a.chunk_rows);
-    const int grid = grid_for(a.tile0[a.count], sms, 4);
-    cudaError_t e = cudaSuccess;
-#define GQ_BACK(RR)                                                                          \
-    case RR:                                                                                 \
-        if (vec) {                                                                           \
-            e = cudaFuncSetAttribute(psgd_back_kernel<RR, true>,                             \
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);\
-            if (e == cudaSuccess) psgd_back_kernel<RR, true><<<grid, kPsgdThreads, smem, st>>>(a); \
-        } else {                                                                             \
-            e = cudaFuncSetAttribute(psgd_back_kernel<RR, false>,                            \
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);\
-            if (e == cudaSuccess) psgd_back_kernel<RR, false><<<grid, kPsgdThreads, smem, st>>>(a); \
-        }                                                                                    \
-        break;
+#define GQ_BACK(RR) \
+    case RR: return vec ? back_inst<RR, true>(a, sms, st) : back_inst<RR, false>(a, sms, st);
     switch (a.rank) {
         GQ_PSGD_RANKS(GQ_BACK)
         default: return cudaErrorInvalidValue;
     }
 #undef GQ_BACK
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
 }
 
 cudaError_t launch_psgd_back_reduce(const PsgdArgs& a, int sms, cudaStream_t st) {

@@ -33,7 +33,7 @@ struct PsgdArgs {
 
 cudaError_t launch_psgd_project(const PsgdArgs& a, bool vec, int sms, cudaStream_t st);
 cudaError_t launch_psgd_orth(const PsgdArgs& a, cudaStream_t st);
-size_t psgd_back_smem(int rank, int chunk_rows);
+size_t psgd_back_smem(int rank, int chunk_rows, bool vec);
 cudaError_t launch_psgd_back(const PsgdArgs& a, bool vec, int sms, cudaStream_t st);
 cudaError_t launch_psgd_back_reduce(const PsgdArgs& a, int sms, cudaStream_t st);
 cudaError_t launch_psgd_mean(const float* qsum, float* q, long long len, int W, int sms,

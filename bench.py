@@ -526,11 +526,12 @@ def run_lqsgd(args):
     stream = torch.cuda.current_stream()
     peak, peak_kind = measured_hbm_peak()
     wl = synthetic.LQ_WORKLOAD
-    W, L, n, m = wl["W"], wl["pairs"], wl["n"], wl["m"]
+    W, L, n, m = wl["W"], args.lqsgd_mats, wl["n"], wl["m"]
     K = max(5, min(args.steps, 20))
     rows_out = []
     g = None
-    for r in wl["ranks"]:
+    ranks = wl["ranks"] if args.lqsgd_rank is None else (args.lqsgd_rank,)
+    for r in ranks:
         sh = gq.PsgdShapes([n] * L, [m] * L, r)
         if g is None:
             g = synthetic.make_gradients(W, sh.total, "normal", seed=synthetic.seed_for(5),
@@ -656,6 +657,10 @@ def main():
                     help="one JSON line comparing the global scale with per-bucket scales")
     ap.add_argument("--lqsgd", action="store_true",
                     help="one JSON line with the PowerSGD + log-quantizer step timings")
+    ap.add_argument("--lqsgd-mats", type=int, default=synthetic.LQ_WORKLOAD["pairs"],
+                    help="matrices per worker for --lqsgd (a smaller case for profiling)")
+    ap.add_argument("--lqsgd-rank", type=int, default=None, choices=range(1, 9),
+                    help="one rank for --lqsgd instead of 1, 4 and 7")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
