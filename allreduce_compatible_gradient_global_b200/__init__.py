@@ -46,7 +46,8 @@ class _Config(ctypes.Structure):
     _fields_ = [("levels", ctypes.c_int), ("s", ctypes.c_int), ("L", ctypes.c_int),
                 ("bits", ctypes.c_int), ("scale_kind", ctypes.c_int), ("wire", ctypes.c_int),
                 ("ef", ctypes.c_int), ("alpha", ctypes.c_float),
-                ("seed", ctypes.c_ulonglong), ("step", ctypes.c_uint)]
+                ("seed", ctypes.c_ulonglong), ("step", ctypes.c_uint),
+                ("worker0", ctypes.c_uint)]
 
 
 @dataclass
@@ -62,6 +63,7 @@ class GQConfig:
     alpha: float = 10.0
     seed: int = 0
     step: int = 0
+    worker0: int = 0
 
     def c(self) -> _Config:
         lv = _LEVELS.get(self.levels, self.levels)
@@ -69,7 +71,8 @@ class GQConfig:
         wr = _WIRES.get(self.wire, self.wire)
         return _Config(int(lv), int(self.s), int(self.L), int(self.bits), int(sk), int(wr),
                        1 if self.ef else 0, float(self.alpha),
-                       int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.step) & 0xFFFFFFFF)
+                       int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.step) & 0xFFFFFFFF,
+                       int(self.worker0) & 0xFFFFFFFF)
 
     @property
     def wire_dtype(self):

@@ -176,6 +176,7 @@ void fill_quant_args(QuantArgs& a, const gq_config* cfg, int W, long long d) {
     a.W = W;
     a.wire = cfg->wire;
     a.step = cfg->step;
+    a.worker0 = cfg->worker0;
     a.L = cfg->L;
     a.smax = (float)cfg->s;
     a.finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, -(cfg->L - 1)) : 1.0f;

@@ -51,6 +51,7 @@ struct QuantArgs {
     int W;
     int wire;  // bytes per sum element
     unsigned int step;
+    unsigned int worker0;  // Philox worker index of row 0
     int L;
     float smax;        // (float)s
     float finest;      // 2^-(L-1)

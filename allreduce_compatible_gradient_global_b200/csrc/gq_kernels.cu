@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, GQ_QUANT_MIN_BLOCKS)
                 if (wb + i < a.W) {
                     const int w = wb + i;
                     const float4 v = EF ? add4(gv[i], ev[i]) : gv[i];
-                    const uint4 rnd = philox10(philox_counter(q, a.step, (uint32_t)w), a.rk);
+                    const uint4 rnd = philox10(philox_counter(q, a.step, a.worker0 + (uint32_t)w), a.rk);
                     const int c0 = quantize_one<LEVELS>(v.x, aq, a, rnd.x);
                     const int c1 = quantize_one<LEVELS>(v.y, aq, a, rnd.y);
                     const int c2 = quantize_one<LEVELS>(v.z, aq, a, rnd.z);

@@ -121,7 +121,7 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 // WT: the number of workers when known at compile time (the worker loop is
 // then fully unrolled and the Philox chains of all workers interleave), or 0.
-template <int LEVELS, int BITS, bool EF, int WT, bool BQ>
+template <int LEVELS, int BITS, bool EF, int WT, bool BQ, bool WOFF>
 __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     quant_tma_kernel(const __grid_constant__ QuantArgs a, int stages) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -249,7 +249,9 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                     v = make_float4(__fadd_rn(v.x, ev.x), __fadd_rn(v.y, ev.y),
                                     __fadd_rn(v.z, ev.z), __fadd_rn(v.w, ev.w));
                 }
-                const uint4 rnd = philox10(philox_counter(q, a.step, (uint32_t)w), a.rk);
+                // WOFF = 0: the worker word is the loop constant w (the common case)
+                const uint32_t wid = WOFF ? a.worker0 + (uint32_t)w : (uint32_t)w;
+                const uint4 rnd = philox10(philox_counter(q, a.step, wid), a.rk);
                 unsigned char* cdst = codes_blk + (long long)w * row_bytes;
                 float4 qv;  // the values Q(v) in units of c, as floats
                 if (LEVELS == 0) {
@@ -334,9 +336,9 @@ size_t tma_smem_bytes(int W, bool ef, int stages) {
     return (size_t)stages * rows * kTmaTile * sizeof(float) + 2 * stages * sizeof(unsigned long long);
 }
 
-template <int LEVELS, int BITS, bool EF, int WT, bool BQ>
+template <int LEVELS, int BITS, bool EF, int WT, bool BQ, bool WOFF>
 static cudaError_t launch_tma_inst(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
-    auto kern = quant_tma_kernel<LEVELS, BITS, EF, WT, BQ>;
+    auto kern = quant_tma_kernel<LEVELS, BITS, EF, WT, BQ, WOFF>;
     const size_t smem = tma_smem_bytes(a.W, EF, stages);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -348,14 +350,19 @@ template <int LEVELS, int BITS, bool EF>
 static cudaError_t launch_tma_w(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
     // per-bucket scales get their own instantiations, so the global-scale
     // kernel keeps one multiplier in a register for the whole launch
+    // The unrolled W = 8 kernel gets the worker offset of a data-parallel rank
+    // as a separate instantiation; the general one always adds it.
+    const bool woff = a.worker0 != 0;
     if (a.bq_mult) {
         if (GQ_TMA_SPECIALIZE_W8 && a.W == 8)
-            return launch_tma_inst<LEVELS, BITS, EF, 8, true>(a, stages, grid, st);
-        return launch_tma_inst<LEVELS, BITS, EF, 0, true>(a, stages, grid, st);
+            return woff ? launch_tma_inst<LEVELS, BITS, EF, 8, true, true>(a, stages, grid, st)
+                        : launch_tma_inst<LEVELS, BITS, EF, 8, true, false>(a, stages, grid, st);
+        return launch_tma_inst<LEVELS, BITS, EF, 0, true, true>(a, stages, grid, st);
     }
     if (GQ_TMA_SPECIALIZE_W8 && a.W == 8)
-        return launch_tma_inst<LEVELS, BITS, EF, 8, false>(a, stages, grid, st);
-    return launch_tma_inst<LEVELS, BITS, EF, 0, false>(a, stages, grid, st);
+        return woff ? launch_tma_inst<LEVELS, BITS, EF, 8, false, true>(a, stages, grid, st)
+                    : launch_tma_inst<LEVELS, BITS, EF, 8, false, false>(a, stages, grid, st);
+    return launch_tma_inst<LEVELS, BITS, EF, 0, false, true>(a, stages, grid, st);
 }
 
 template <int LEVELS, bool EF>

@@ -188,8 +188,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl, cfg = workload_config(gq, args.workload)
-    W, d = wl["W"], wl["d"]
-    g = synthetic.workload_gradients(args.workload, device=dev)
+    W, d = wl["W"], (args.coords or wl["d"])
+    g = synthetic.workload_gradients(args.workload, device=dev, d=d)
     buf = gq.StepBuffers(cfg, W, d, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -239,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
     n_avg = sum(norm_ms) / K
     peak, peak_kind = measured_hbm_peak()
     achieved = p2 / (q_avg * 1e-3) / 1e9
-    traffic = recorded_traffic(args.workload)
+    traffic = None if args.coords else recorded_traffic(args.workload)
     roofline = {"bound": "hbm", "kernel": "fused pass of gq_quantize_aggregate "
                                           "(quant_tma_kernel when d % 4 == 0 and the rows fit)",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -265,6 +265,7 @@ def run_ours(args, rank, world, local_rank):
         config={"workload": args.workload, "W": W, "d": d, "levels": cfg.levels, "s": cfg.s,
                 "L": cfg.L, "bits": cfg.bits, "wire": cfg.wire, "scale": cfg.scale_kind,
                 "ef": cfg.ef, "parallelism": f"replicas x{world}",
+                "truncated_to_coords": args.coords,
                 "l2": f"inputs exceed L2: {grad_bytes / 1e6:.1f} MB of gradient per read "
                       f"vs {L2_BYTES / 1e6:.0f} MB L2"},
         roofline=roofline, gpu_launches=2 * K, clocks=sampler.summary(), e2e=e2e)
@@ -595,6 +596,47 @@ def run_lqsgd(args):
             "matrices": f"{L} x {n}x{m} per worker", "rows": rows_out}
 
 
+def run_dp(args, rank, world, local_rank):
+    """The real data-parallel exchange (one worker per rank, NCCL): per step
+    gq_global_norm + MAX all-reduce of the scale + gq_quantize_aggregate + SUM
+    all-reduce of the int8 sums + decode, against a plain fp32 SUM all-reduce of
+    the same gradient.  Times are the max over ranks of CUDA-event times."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    wl, cfg = workload_config(gq, args.workload)
+    d = args.coords or wl["d"]
+    g = synthetic.make_gradients(1, d, wl["recipe"], seed=synthetic.seed_for(wl["seed_index"])
+                                 + rank, device=dev, seg=wl.get("seg", 0), lo=wl.get("lo", 0.0),
+                                 hi=wl.get("hi", 0.0))
+    stepper = DataParallelStep(cfg, d, w_local=1, device=dev)
+    flat = g[0].clone()
+    K = args.steps
+
+    def timed(fn):
+        for i in range(args.warmup):
+            fn(i)
+        torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(K):
+            fn(args.warmup + i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return job_time_ms(t0.elapsed_time(t1), world, dev) / K
+
+    q_ms = timed(lambda i: stepper(g, None, step=i))
+    f_ms = timed(lambda i: torch.distributed.all_reduce(flat))
+    return {"metric": "data-parallel exchange: compressed step vs fp32 all-reduce",
+            "mode": "dp", "n_gpus": world, "workload": args.workload, "d": d,
+            "wire": "int8 sums via NCCL", "compressed_step_ms": round(q_ms, 5),
+            "fp32_allreduce_ms": round(f_ms, 5), "speedup": round(f_ms / q_ms, 3),
+            "bytes_on_wire_per_rank": {"compressed": d + 4, "fp32": 4 * d}}
+
+
 def run_lq(args):
     """The LQ-SGD log quantizer: quantize + decode-sum of 24 factor pairs of
     4096 x r per worker, W = 8, r in {1, 4, 7}."""
@@ -639,6 +681,13 @@ def run_lq(args):
             "W": W, "rows": rows}
 
 
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -649,12 +698,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--reference-coords", type=int, default=1 << 21)
+    ap.add_argument("--coords", type=int, default=None,
+                    help="truncate the workload to this many coordinates (a smaller case "
+                         "of the same recipe, for profiling; not a bench line)")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line with the d = 2^16..2^30 sweep instead of the bench line")
     ap.add_argument("--lq", action="store_true",
                     help="one JSON line with the LQ-SGD log-quantizer timings")
     ap.add_argument("--buckets", action="store_true",
                     help="one JSON line comparing the global scale with per-bucket scales")
+    ap.add_argument("--dp", action="store_true",
+                    help="one JSON line timing the real data-parallel exchange (one worker per "
+                         "rank over NCCL) against an fp32 all-reduce; run under torchrun")
     ap.add_argument("--lqsgd", action="store_true",
                     help="one JSON line with the PowerSGD + log-quantizer step timings")
     ap.add_argument("--lqsgd-mats", type=int, default=synthetic.LQ_WORKLOAD["pairs"],
@@ -685,6 +740,22 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    if args.dp:
+        if world == 1:
+            import datetime
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group(
+                "nccl", rank=0, world_size=1, init_method="tcp://127.0.0.1:%d" % _free_port(),
+                timeout=datetime.timedelta(seconds=120),
+                device_id=torch.device("cuda", local_rank))
+        try:
+            res = run_dp(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+        finally:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     try:
         result = run_ours(args, rank, world, local_rank)
         if rank == 0:

@@ -98,6 +98,10 @@ typedef struct {
     float alpha;      /* LOG: curvature a > 0 of the log map */
     unsigned long long seed; /* Philox key */
     unsigned int step;       /* step counter (part of the Philox counter) */
+    unsigned int worker0;    /* Philox worker index of row 0 (row w draws as worker
+                                worker0 + w): 0 when all W workers are on this GPU;
+                                the rank's first worker in a real data-parallel
+                                exchange, so that every worker keeps its own stream */
 } gq_config;
 
 /* Library version (major*10000 + minor*100 + patch). */

@@ -38,6 +38,8 @@ def lib():
         L.gqo_maxabs.restype = f32
         L.gqo_global_scale.argtypes = [P, P, i32, i64, i32, P, P]
         L.gqo_quantize.argtypes = [P, P, i32, i64, P, i32, i32, i32, u64, u32, f32, P]
+        L.gqo_quantize_workers.argtypes = [P, P, i32, i64, P, u32, i32, i32, i32, u64, u32,
+                                           f32, P]
         L.gqo_code_value.argtypes = [i32, i32, i32]
         L.gqo_code_value.restype = i32
         L.gqo_uniform_multiplier.argtypes = [i32, f32]
@@ -116,15 +118,16 @@ def global_scale(g, e=None, scale_kind=SCALE_L2):
     return np.float32(S[0]), norms
 
 
-def quantize(g, e=None, *, levels=UNIFORM, s=15, L=8, seed=0, step=0, S, js=None):
-    """Codes [W][n] int32 for v = g + e at coordinates js (default 0..n-1)."""
+def quantize(g, e=None, *, levels=UNIFORM, s=15, L=8, seed=0, step=0, S, js=None, worker0=0):
+    """Codes [W][n] int32 for v = g + e at coordinates js (default 0..n-1); row w
+    draws its uniforms as worker worker0 + w."""
     g = _f32(g)
     e = _f32(e)
     W, n = g.shape
     jsa = None if js is None else np.ascontiguousarray(js, dtype=np.int64)
     out = np.zeros((W, n), np.int32)
-    _check(lib().gqo_quantize(_p(g), _p(e), W, n, _p(jsa), levels, s, L, seed, step,
-                              float(S), _p(out)), "quantize")
+    _check(lib().gqo_quantize_workers(_p(g), _p(e), W, n, _p(jsa), int(worker0), levels, s, L,
+                                      seed, step, float(S), _p(out)), "quantize")
     return out
 
 

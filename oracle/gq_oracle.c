@@ -230,6 +230,15 @@ int gqo_quantize(const float* g, const float* e, int W, int64_t n,
                  const int64_t* js, int levels, int s, int L,
                  uint64_t seed, uint32_t step, float S, int32_t* codes_out)
 {
+    return gqo_quantize_workers(g, e, W, n, js, 0u, levels, s, L, seed, step, S,
+                                codes_out);
+}
+
+int gqo_quantize_workers(const float* g, const float* e, int W, int64_t n,
+                         const int64_t* js, uint32_t worker0, int levels, int s,
+                         int L, uint64_t seed, uint32_t step, float S,
+                         int32_t* codes_out)
+{
     if (!g || !codes_out || W < 1 || n < 0) return -1;
     if (levels == GQO_UNIFORM) {
         if (s < 1) return -1;
@@ -245,7 +254,7 @@ int gqo_quantize(const float* g, const float* e, int W, int64_t n,
             int64_t at = (int64_t)w * n + i;
             float v = e ? g[at] + e[at] : g[at];
             uint64_t j = js ? (uint64_t)js[i] : (uint64_t)i;
-            uint32_t f = gqo_uniform_bits(seed, 0u, step, (uint32_t)w, j);
+            uint32_t f = gqo_uniform_bits(seed, 0u, step, worker0 + (uint32_t)w, j);
             codes_out[at] = (levels == GQO_UNIFORM)
                                 ? quantize_uniform(v, a, s, f)
                                 : quantize_exp(v, a, L, f);

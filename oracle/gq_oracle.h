@@ -86,6 +86,13 @@ int gqo_quantize(const float* g, const float* e, int W, int64_t n,
                  const int64_t* js, int levels, int s, int L,
                  uint64_t seed, uint32_t step, float S, int32_t* codes_out);
 
+/* The same with row w drawing its uniforms as worker worker0 + w (the rows of
+ * one rank in a data-parallel exchange). */
+int gqo_quantize_workers(const float* g, const float* e, int W, int64_t n,
+                         const int64_t* js, uint32_t worker0, int levels, int s,
+                         int L, uint64_t seed, uint32_t step, float S,
+                         int32_t* codes_out);
+
 /* The integer each code contributes to the sum: the code itself (UNIFORM) or
  * sign * 2^(idx-1) units of the finest level 2^-(L-1) (EXP, idx = |code|). */
 int32_t gqo_code_value(int32_t code, int levels, int L);

@@ -1,0 +1,150 @@
+"""The data-parallel exchange's host orchestration, on CPU with gloo ranks.
+
+Each rank holds its own rows and runs ``DataParallelStep``; the kernels are
+stood in for by the oracle (test-only ``ops``), so what is checked is the
+exchange itself: the MAX all-reduce of the scale, worker indices rank * W_local
++ w for the uniforms, the SUM all-reduce of the integer sums, the decode over
+all W workers, and local error feedback.  The result must equal the oracle's
+single-process step on all W rows, bit for bit (the oracle's per-worker norms do
+not depend on how rows are grouped).
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import synthetic
+
+
+class OracleOps:
+    """The oracle in place of the kernels, for host-side tests only."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    def _kw(self, cfg):
+        return dict(levels=0 if cfg.levels == "uniform" else 1, s=cfg.s, L=cfg.L)
+
+    def global_norm(self, g, e, cfg, scale, ws):
+        kind = 0 if cfg.scale_kind == "l2" else 1
+        S, _ = self.o.global_scale(g.numpy(), None if e is None else e.numpy(), kind)
+        scale[0] = float(S)
+
+    def quantize_sum(self, g, e, cfg, scale, sum_out, ws):
+        S = np.float32(scale[0].item())
+        ev = e.numpy() if (cfg.ef and e is not None) else None
+        codes = self.o.quantize(g.numpy(), ev, seed=cfg.seed, step=cfg.step, S=S,
+                                worker0=cfg.worker0, **self._kw(cfg))
+        sum_out.copy_(torch.from_numpy(self.o.aggregate(codes, levels=self._kw(cfg)["levels"],
+                                                        L=cfg.L)))
+        if cfg.ef and e is not None:
+            e.copy_(torch.from_numpy(self.o.error_feedback(g.numpy(), ev, codes, S=S,
+                                                           **self._kw(cfg))))
+
+    def decode(self, sum_in, W, cfg, scale, out, ws):
+        S = np.float32(scale[0].item())
+        out.copy_(torch.from_numpy(self.o.decode_mean(sum_in.numpy().astype(np.int32), W, S=S,
+                                                      **self._kw(cfg))))
+
+    def status(self, ws):
+        return 0
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+CASES = {
+    "uniform": dict(levels="uniform", s=15, bits=5, wire="int8", seed=3, step=2),
+    "exp_ef": dict(levels="exp", L=5, bits=4, wire="int8", scale_kind="maxabs", ef=True,
+                   seed=5, step=1),
+}
+
+
+def _rank_main(rank, world, port, case, w_local, d, outdir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import allreduce_compatible_gradient_global_b200 as gq
+        from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
+        cfg = gq.GQConfig(**CASES[case])
+        W = world * w_local
+        g_all = synthetic.make_gradients(W, d, "student_t3", seed=11, seg=100, lo=-3, hi=0)
+        e_all = synthetic.make_gradients(W, d, "normal", seed=12) * 1e-3
+        rows = slice(rank * w_local, (rank + 1) * w_local)
+        g = g_all[rows].clone()
+        e = e_all[rows].clone()
+        stepper = DataParallelStep(cfg, d, w_local=w_local, device="cpu", ops=OracleOps(oracle))
+        outs = []
+        for t in range(2):
+            outs.append(stepper(g, e, step=cfg.step + t).clone().numpy())
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"), out0=outs[0], out1=outs[1],
+                 e=e.numpy(), scale=stepper.scale.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("case,w_local", [("uniform", 1), ("uniform", 3), ("exp_ef", 2)])
+def test_two_ranks_equal_the_single_process_step(oracle, tmp_path, case, w_local):
+    world, d = 2, 700
+    mp.start_processes(_rank_main, args=(world, _free_port(), case, w_local, d, str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
+    import allreduce_compatible_gradient_global_b200 as gq
+    cfg = gq.GQConfig(**CASES[case])
+    W = world * w_local
+    g_all = synthetic.make_gradients(W, d, "student_t3", seed=11, seg=100, lo=-3, hi=0).numpy()
+    e = (synthetic.make_gradients(W, d, "normal", seed=12) * 1e-3).numpy()
+    kw = dict(levels=0 if cfg.levels == "uniform" else 1, s=cfg.s, L=cfg.L,
+              scale_kind=0 if cfg.scale_kind == "l2" else 1)
+    res = [np.load(tmp_path / f"rank{r}.npz") for r in range(world)]
+    for t in range(2):
+        ref = oracle.step(g_all, e if cfg.ef else None, seed=cfg.seed, step=cfg.step + t,
+                          ef=cfg.ef, **kw)
+        for r in range(world):
+            got = res[r][f"out{t}"]
+            assert np.array_equal(got.view(np.uint32), ref["out"].view(np.uint32)), (t, r)
+        if cfg.ef:
+            e = ref["e"]
+    if cfg.ef:
+        for r in range(world):
+            rows = slice(r * w_local, (r + 1) * w_local)
+            assert np.array_equal(res[r]["e"].view(np.uint32), e[rows].view(np.uint32))
+    assert res[0]["scale"][0] == res[1]["scale"][0]
+
+
+def test_overflow_rule_uses_the_total_worker_count(oracle):
+    """W = world * W_local decides the wire type: 9 workers of s = 15 overflow int8."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    assert gq.gq_validate(gq.GQConfig(s=15, bits=5, wire="int8"), 8, 100) == gq.GQ_OK
+    assert gq.gq_validate(gq.GQConfig(s=15, bits=5, wire="int8"), 9, 100) == gq.GQ_ERR_OVERFLOW
+
+
+def test_worker0_offsets_the_uniform_streams(oracle):
+    """Rows quantized as workers k.. equal rows k.. of a quantization of all rows."""
+    g = synthetic.make_gradients(5, 300, "normal", seed=2).numpy()
+    full = oracle.quantize(g, s=7, seed=9, step=4, S=np.float32(40.0))
+    part = oracle.quantize(g[2:4], s=7, seed=9, step=4, S=np.float32(40.0), worker0=2)
+    assert np.array_equal(full[2:4], part)
+    assert not np.array_equal(full[0:2], part)
+
+
+def test_int16_wire_is_refused():
+    """NCCL cannot reduce 16-bit integers: the exchange refuses int16 sums up front."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        with pytest.raises(ValueError):
+            DataParallelStep(gq.GQConfig(s=127, bits=8, wire="int16"), 100, device="cpu")
+    finally:
+        dist.destroy_process_group()
