@@ -184,3 +184,38 @@ def test_bucket_entry_points_reject_before_launch(gq):
     clog = cfg(gq, levels="log", alpha=10.0).c()
     assert lib.gq_step_bucketed(good, None, 4, 4096, 10, ctypes.byref(clog), good, good, good,
                                 good, good, None) == gq.GQ_ERR_ARG
+
+
+def test_psgd_entry_points_reject_before_launch(gq):
+    lib = gq.lib()
+    P = ctypes.c_void_p
+    good = P(0x10000000)
+    odd = P(0x10000004)
+    rows = (ctypes.c_int * 2)(64, 32)
+    cols = (ctypes.c_int * 2)(48, 32)
+    n = ctypes.c_size_t()
+    assert lib.gq_psgd_workspace_bytes(2, 2, rows, cols, 4, ctypes.byref(n)) == gq.GQ_OK
+    assert n.value > 256
+    for bad_rank in (0, 9):
+        assert lib.gq_psgd_workspace_bytes(2, 2, rows, cols, bad_rank, ctypes.byref(n)) == \
+            gq.GQ_ERR_ARG
+    assert lib.gq_psgd_workspace_bytes(0, 2, rows, cols, 4, ctypes.byref(n)) == gq.GQ_ERR_ARG
+    zero = (ctypes.c_int * 1)(0)
+    assert lib.gq_psgd_workspace_bytes(2, 1, zero, cols, 4, ctypes.byref(n)) == gq.GQ_ERR_ARG
+    # have_prev without a previous P
+    assert lib.gq_psgd_project(good, good, 2, 2, rows, cols, 4, 1, None, good, good, None) == \
+        gq.GQ_ERR_ARG
+    assert lib.gq_psgd_project(odd, good, 2, 2, rows, cols, 4, 0, None, good, good, None) == \
+        gq.GQ_ERR_ALIGN
+    assert lib.gq_psgd_back_project(good, good, 2, 2, rows, cols, 4, good, None, None) == \
+        gq.GQ_ERR_ARG
+    assert lib.gq_psgd_mean(good, good, 10, 0, None) == gq.GQ_ERR_ARG
+    c = cfg(gq).c()  # not the log level set
+    assert lib.gq_lqsgd_step(good, good, 2, 2, rows, cols, 4, 0, ctypes.byref(c), good, good,
+                             None, good, None) == gq.GQ_ERR_ARG
+
+
+def test_workspace_and_config_layout(gq):
+    """gq_config carries worker0 after step (the C struct and the binding agree)."""
+    assert ctypes.sizeof(gq._Config) == 48
+    assert gq._Config.worker0.offset == 44
