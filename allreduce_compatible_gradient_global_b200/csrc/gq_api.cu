@@ -797,10 +797,12 @@ GQ_API int gq_psgd_project(const float* g_dev, float* m_dev, int W, int nmats,
 
 GQ_API int gq_psgd_orthonormalize(float* p_dev, int nmats, const int* rows_host, int rank,
                                   cudaStream_t stream) {
-    if (!rows_host) return GQ_ERR_ARG;
-    std::vector<int> ones((size_t)(nmats > 0 && nmats <= 4096 ? nmats : 1), 4);
+    if (!rows_host || nmats < 1 || nmats > 4096) return GQ_ERR_ARG;
+    // only the row counts matter here; the column counts are set to a valid
+    // placeholder so that the shared shape check and offsets apply
+    const std::vector<int> any_cols((size_t)nmats, 4);
     PsgdShape s;
-    int rc = psgd_shape(1, nmats, rows_host, ones.data(), rank, s);
+    int rc = psgd_shape(1, nmats, rows_host, any_cols.data(), rank, s);
     if (rc) return rc;
     if (!p_dev) return GQ_ERR_ARG;
     if (!aligned16(p_dev)) return GQ_ERR_ALIGN;
