@@ -218,3 +218,26 @@ def test_full_size_bucketed(gq, oracle, b):
         assert np.array_equal(buf.out[j0:j1].cpu().numpy().view(np.uint32), out.view(np.uint32))
     del g, buf, table, ws
     torch.cuda.empty_cache()
+
+
+def test_beyond_2_31_coordinates(gq, oracle):
+    """One worker with d = 2^31 + 4 (8.6 GB of gradient): coordinate indices
+    pass 2^31, so a 32-bit index anywhere would show.  The scale is checked
+    against the oracle's streamed fp64 norm, and sampled blocks on both sides
+    of 2^31 (and the last one) bit for bit."""
+    W, d = 1, (1 << 31) + 4
+    cfg = gq.GQConfig(levels="uniform", s=15, bits=5, wire="int8", seed=77, step=1)
+    g = torch.empty((W, d), dtype=torch.float32, device="cuda")
+    synthetic.fill_gradients(g, "normal", seed=31)
+    buf = gq.StepBuffers(cfg, W, d)
+    run_bench_launches(gq, g, None, cfg, buf)
+    S_ref, _ = streamed_scale(oracle, g, None, "l2")
+    S = np.float32(buf.scale.item())
+    assert abs(float(S) - float(S_ref)) <= 1e-5 * float(S_ref)
+    nblk = (d + 127) // 128
+    edge = (1 << 31) // 128  # the last block: coordinates 2^31 .. 2^31 + 3
+    assert edge == nblk - 1
+    blocks = sorted({0, 12345, edge - 3, edge - 2, edge - 1, edge})
+    check_blocks(gq, oracle, cfg, g, None, buf, None, blocks)
+    del g, buf
+    torch.cuda.empty_cache()
