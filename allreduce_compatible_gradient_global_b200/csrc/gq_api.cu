@@ -8,6 +8,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "gq_api.h"
 #include "gq_internal.h"
 #include "gq_psgd.h"
@@ -15,6 +17,15 @@
 using namespace gq;
 
 namespace {
+
+// An NVTX range around each compute call of the ABI (free when no tool is
+// attached), so that timelines and profiles show the library's calls.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kVersion = 100;  // 0.1.0
 
@@ -273,6 +284,7 @@ GQ_API int gq_selftest_wait_timeout(void* ws_dev, unsigned int limit_ms, cudaStr
 GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long long d,
                           const gq_config* cfg, float* scale_dev, double* norms_dev, void* ws_dev,
                           cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_global_norm");
     if (!cfg || (!g_dev && d > 0) || !scale_dev || !ws_dev) return GQ_ERR_ARG;
     int rc = check_sizes(W, d);
     if (rc) return rc;
@@ -326,6 +338,7 @@ static int quant_common(const float* g_dev, float* e_dev, int W, long long d, co
 GQ_API int gq_quantize_pack(const float* g_dev, const float* e_dev, int W, long long d,
                             const gq_config* cfg, const float* scale_dev, void* codes_dev,
                             void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_quantize_pack");
     if (!codes_dev) return GQ_ERR_ARG;
     // v = g + e is read but e is not updated here: the update belongs to step 5
     gq_config c;
@@ -351,6 +364,7 @@ GQ_API int gq_quantize_pack(const float* g_dev, const float* e_dev, int W, long 
 
 GQ_API int gq_aggregate(const void* codes_dev, int W, long long d, const gq_config* cfg,
                         void* sum_dev, void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_aggregate");
     (void)ws_dev;
     int rc = gq_validate(cfg, W, d);
     if (rc) return rc;
@@ -371,6 +385,7 @@ GQ_API int gq_dequantize_ef(const void* sum_dev, const void* codes_dev, const fl
                             float* e_dev, int W, long long d, const gq_config* cfg,
                             const float* scale_dev, float* out_dev, void* ws_dev,
                             cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_dequantize_ef");
     (void)ws_dev;
     int rc = gq_validate(cfg, W, d);
     if (rc) return rc;
@@ -406,6 +421,7 @@ GQ_API int gq_dequantize_ef(const void* sum_dev, const void* codes_dev, const fl
 GQ_API int gq_quantize_aggregate(const float* g_dev, float* e_dev, int W, long long d,
                                  const gq_config* cfg, const float* scale_dev, void* codes_dev,
                                  void* sum_dev, float* out_dev, void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_quantize_aggregate");
     return quant_common(g_dev, e_dev, W, d, cfg, scale_dev, codes_dev, sum_dev, out_dev, ws_dev,
                         true, stream);
 }
@@ -414,6 +430,7 @@ GQ_API int gq_step_fused(const float* g_dev, float* e_dev, int W, long long d,
                          const gq_config* cfg, float* scale_dev, double* norms_dev,
                          void* codes_dev, void* sum_dev, float* out_dev, void* ws_dev,
                          cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_step_fused");
     int rc = gq_validate(cfg, W, d);
     if (rc) return rc;
     if (cfg->ef && !e_dev) return GQ_ERR_ARG;
@@ -433,6 +450,7 @@ GQ_API int gq_step_fused_host(const float* g_host, float* g_dev, float* e_dev, i
                               const gq_config* cfg, float* scale_dev, void* codes_dev,
                               void* sum_dev, float* out_dev, float* out_host, float* scale_host,
                               void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_step_fused_host");
     int rc = gq_validate(cfg, W, d);
     if (rc) return rc;
     if (!g_host || !g_dev || !out_dev || !out_host) return GQ_ERR_ARG;
@@ -474,6 +492,7 @@ static void logq_group(LogqArgs& a, int m0, int count, const int* rows, const in
 GQ_API int gq_logq_quantize(const float* x_dev, int W, int nmats, const int* rows_host,
                             const int* cols_host, const gq_config* cfg, float* maxabs_dev,
                             signed char* codes_dev, void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_logq_quantize");
     if (!cfg || cfg->levels != GQ_LOG || !(cfg->alpha > 0.f) || !(cfg->alpha <= 3.0e38f))
         return GQ_ERR_ARG;
     if (!x_dev || !maxabs_dev || !codes_dev || !ws_dev || W < 1) return GQ_ERR_ARG;
@@ -505,6 +524,7 @@ GQ_API int gq_logq_quantize(const float* x_dev, int W, int nmats, const int* row
 GQ_API int gq_logq_decode_sum(const signed char* codes_dev, const float* maxabs_dev, int W,
                               int nmats, const int* rows_host, const int* cols_host,
                               const gq_config* cfg, float* out_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_logq_decode_sum");
     if (!cfg || cfg->levels != GQ_LOG || !(cfg->alpha > 0.f) || !(cfg->alpha <= 3.0e38f))
         return GQ_ERR_ARG;
     if (!codes_dev || !maxabs_dev || !out_dev || W < 1) return GQ_ERR_ARG;
@@ -549,6 +569,7 @@ GQ_API int gq_bucket_workspace_bytes(const gq_config* cfg, int W, long long d, i
 GQ_API int gq_bucket_scales(const float* g_dev, const float* e_dev, int W, long long d,
                             int bucket_log2, const gq_config* cfg, float* table_dev, void* ws_dev,
                             cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_bucket_scales");
     if (!cfg || bucket_log2 < kBucketLog2Min || bucket_log2 > kBucketLog2Max) return GQ_ERR_ARG;
     int rc = gq_validate(cfg, W, d);
     if (rc) return rc;
@@ -586,6 +607,7 @@ GQ_API int gq_quantize_aggregate_bucketed(const float* g_dev, float* e_dev, int 
                                           int bucket_log2, const gq_config* cfg,
                                           const float* table_dev, void* codes_dev, void* sum_dev,
                                           float* out_dev, void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_quantize_aggregate_bucketed");
     if (!cfg || bucket_log2 < kBucketLog2Min || bucket_log2 > kBucketLog2Max) return GQ_ERR_ARG;
     int rc = gq_validate(cfg, W, d);
     if (rc) return rc;
@@ -620,6 +642,7 @@ GQ_API int gq_quantize_aggregate_bucketed(const float* g_dev, float* e_dev, int 
 GQ_API int gq_step_bucketed(const float* g_dev, float* e_dev, int W, long long d, int bucket_log2,
                             const gq_config* cfg, float* table_dev, void* codes_dev, void* sum_dev,
                             float* out_dev, void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_step_bucketed");
     int rc = gq_bucket_scales(g_dev, cfg && cfg->ef ? e_dev : nullptr, W, d, bucket_log2, cfg,
                               table_dev, ws_dev, stream);
     if (rc) return rc;
@@ -772,6 +795,7 @@ GQ_API int gq_psgd_project(const float* g_dev, float* m_dev, int W, int nmats,
                            const int* rows_host, const int* cols_host, int rank, int have_prev,
                            const float* p_prev_dev, const float* q_dev, float* pw_dev,
                            cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_psgd_project");
     PsgdShape s;
     int rc = psgd_shape(W, nmats, rows_host, cols_host, rank, s);
     if (rc) return rc;
@@ -797,6 +821,7 @@ GQ_API int gq_psgd_project(const float* g_dev, float* m_dev, int W, int nmats,
 
 GQ_API int gq_psgd_orthonormalize(float* p_dev, int nmats, const int* rows_host, int rank,
                                   cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_psgd_orthonormalize");
     if (!rows_host || nmats < 1 || nmats > 4096) return GQ_ERR_ARG;
     // only the row counts matter here; the column counts are set to a valid
     // placeholder so that the shared shape check and offsets apply
@@ -820,6 +845,7 @@ GQ_API int gq_psgd_orthonormalize(float* p_dev, int nmats, const int* rows_host,
 GQ_API int gq_psgd_back_project(const float* m_dev, const float* p_dev, int W, int nmats,
                                 const int* rows_host, const int* cols_host, int rank,
                                 float* qw_dev, void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_psgd_back_project");
     PsgdShape s;
     int rc = psgd_shape(W, nmats, rows_host, cols_host, rank, s);
     if (rc) return rc;
@@ -845,6 +871,7 @@ GQ_API int gq_psgd_back_project(const float* m_dev, const float* p_dev, int W, i
 
 GQ_API int gq_psgd_mean(const float* sum_dev, float* out_dev, long long n, int W,
                         cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_psgd_mean");
     if (!sum_dev || !out_dev || n < 0 || W < 1) return GQ_ERR_ARG;
     if (!aligned4(sum_dev) || !aligned4(out_dev)) return GQ_ERR_ALIGN;
     if (n == 0) return GQ_OK;
@@ -854,6 +881,7 @@ GQ_API int gq_psgd_mean(const float* sum_dev, float* out_dev, long long n, int W
 GQ_API int gq_psgd_reconstruct(const float* p_dev, const float* q_dev, int nmats,
                                const int* rows_host, const int* cols_host, int rank,
                                float* ghat_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_psgd_reconstruct");
     PsgdShape s;
     int rc = psgd_shape(1, nmats, rows_host, cols_host, rank, s);
     if (rc) return rc;
@@ -876,6 +904,7 @@ GQ_API int gq_lqsgd_step(const float* g_dev, float* m_dev, int W, int nmats,
                          const int* rows_host, const int* cols_host, int rank, int have_prev,
                          const gq_config* cfg, float* p_dev, float* q_dev, float* ghat_dev,
                          void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_lqsgd_step");
     if (!cfg || cfg->levels != GQ_LOG || !(cfg->alpha > 0.f) || !(cfg->alpha <= 3.0e38f))
         return GQ_ERR_ARG;
     PsgdShape s;
