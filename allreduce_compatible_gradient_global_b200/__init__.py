@@ -29,11 +29,11 @@ GQ_ERR_TIMEOUT = -7
 
 UNIFORM, EXP, LOG = 0, 1, 2
 SCALE_L2, SCALE_MAXABS = 0, 1
-WIRE_INT8, WIRE_INT16 = 1, 2
+WIRE_INT8, WIRE_INT16, WIRE_F16 = 1, 2, 3
 
 _LEVELS = {"uniform": UNIFORM, "exp": EXP, "log": LOG}
 _SCALES = {"l2": SCALE_L2, "maxabs": SCALE_MAXABS}
-_WIRES = {"int8": WIRE_INT8, "int16": WIRE_INT16}
+_WIRES = {"int8": WIRE_INT8, "int16": WIRE_INT16, "f16": WIRE_F16}
 
 
 class GQError(RuntimeError):
@@ -76,7 +76,8 @@ class GQConfig:
 
     @property
     def wire_dtype(self):
-        return torch.int8 if _WIRES.get(self.wire, self.wire) == WIRE_INT8 else torch.int16
+        wr = _WIRES.get(self.wire, self.wire)
+        return {WIRE_INT8: torch.int8, WIRE_INT16: torch.int16, WIRE_F16: torch.float16}[wr]
 
 
 def _load():

@@ -80,8 +80,9 @@ int check_bits(const gq_config* c) {
 }
 
 int check_wire(const gq_config* c, int W) {
-    if (c->wire != GQ_WIRE_INT8 && c->wire != GQ_WIRE_INT16) return GQ_ERR_ARG;
-    const long long lim = c->wire == GQ_WIRE_INT8 ? 127 : 32767;
+    if (c->wire != GQ_WIRE_INT8 && c->wire != GQ_WIRE_INT16 && c->wire != GQ_WIRE_F16)
+        return GQ_ERR_ARG;
+    const long long lim = c->wire == GQ_WIRE_INT8 ? 127 : c->wire == GQ_WIRE_INT16 ? 32767 : 2048;
     if ((long long)W * max_value(*c) > lim) return GQ_ERR_OVERFLOW;
     return GQ_OK;
 }

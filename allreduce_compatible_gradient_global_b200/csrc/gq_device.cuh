@@ -6,6 +6,8 @@
 // compiler can neither contract nor reorder it.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include <cstdint>
 
 namespace gq {
@@ -330,10 +332,40 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
                        __fadd_rn(a.w, b.w));
 }
 
+// The fp16 wire type holds the integer sum itself: every integer of magnitude
+// at most 2048 is an fp16 value, so int -> float -> fp16 and back are exact.
+__device__ __forceinline__ uint32_t int_to_f16_bits(int x) {
+    return (uint32_t)__half_as_ushort(__float2half_rn((float)x));
+}
+__device__ __forceinline__ int f16_bits_to_int(uint32_t h) {
+    return (int)__half2float(__ushort_as_half((unsigned short)h));
+}
+
 // The [d] outputs (sum, mean) are vectors of their own: j0 is a multiple of 4,
 // so a 4-wide store is aligned whenever all 4 coordinates are in range.
+// wire: 1 int8, 2 int16, 3 fp16 holding the integer.
+__device__ __forceinline__ void store_sum_16(void* sum, long long j0, long long d, uint32_t s0,
+                                             uint32_t s1, uint32_t s2, uint32_t s3) {
+    unsigned short* p = reinterpret_cast<unsigned short*>(sum) + j0;
+    if (j0 + 3 < d) {
+        uint2 x;
+        x.x = (s0 & 0xFFFFu) | (s1 << 16);
+        x.y = (s2 & 0xFFFFu) | (s3 << 16);
+        __stcs(reinterpret_cast<uint2*>(p), x);
+    } else {
+        if (j0 < d) p[0] = (unsigned short)s0;
+        if (j0 + 1 < d) p[1] = (unsigned short)s1;
+        if (j0 + 2 < d) p[2] = (unsigned short)s2;
+    }
+}
+
 __device__ __forceinline__ void store_sum(void* sum, int wire, long long j0, long long d, int s0,
                                           int s1, int s2, int s3) {
+    if (wire == 3) {
+        store_sum_16(sum, j0, d, int_to_f16_bits(s0), int_to_f16_bits(s1), int_to_f16_bits(s2),
+                     int_to_f16_bits(s3));
+        return;
+    }
     if (wire == 1) {
         signed char* p = reinterpret_cast<signed char*>(sum) + j0;
         if (j0 + 3 < d) {
@@ -346,17 +378,7 @@ __device__ __forceinline__ void store_sum(void* sum, int wire, long long j0, lon
             if (j0 + 2 < d) p[2] = (signed char)s2;
         }
     } else {
-        short* p = reinterpret_cast<short*>(sum) + j0;
-        if (j0 + 3 < d) {
-            uint2 x;
-            x.x = (uint32_t)(s0 & 0xFFFF) | ((uint32_t)s1 << 16);
-            x.y = (uint32_t)(s2 & 0xFFFF) | ((uint32_t)s3 << 16);
-            __stcs(reinterpret_cast<uint2*>(p), x);
-        } else {
-            if (j0 < d) p[0] = (short)s0;
-            if (j0 + 1 < d) p[1] = (short)s1;
-            if (j0 + 2 < d) p[2] = (short)s2;
-        }
+        store_sum_16(sum, j0, d, (uint32_t)s0, (uint32_t)s1, (uint32_t)s2, (uint32_t)s3);
     }
 }
 
@@ -389,6 +411,12 @@ __device__ __forceinline__ void load_sum(const void* sum, int wire, long long j0
             s1 = j0 + 1 < d ? p[1] : 0;
             s2 = j0 + 2 < d ? p[2] : 0;
             s3 = 0;
+        }
+        if (wire == 3) {
+            s0 = f16_bits_to_int((uint32_t)s0 & 0xFFFFu);
+            s1 = f16_bits_to_int((uint32_t)s1 & 0xFFFFu);
+            s2 = f16_bits_to_int((uint32_t)s2 & 0xFFFFu);
+            s3 = f16_bits_to_int((uint32_t)s3 & 0xFFFFu);
         }
     }
 }

@@ -11,8 +11,8 @@ real collectives of ``torch.distributed`` (NCCL across GPUs):
    fp32 scale;
 2. ``gq_quantize_aggregate`` of the rank's rows with that scale (codes drawn as
    workers rank * W_local + w, error feedback applied locally), writing the
-   rank's integer sum as int8;
-3. an all-reduce SUM of those integers (d bytes instead of 4d of fp32);
+   rank's integer sum as int8, or as fp16 holding the integer;
+3. an all-reduce SUM of those sums (d or 2d bytes instead of 4d of fp32);
 4. ``gq_dequantize_ef`` of the total into the mean over all W = world * W_local
    workers.
 
@@ -21,7 +21,9 @@ the same scale; the scale itself is the max of per-rank scales, each within
 1e-5 of its fp64 norm.  Packed sub-byte codes cannot be summed by NCCL, so the
 exchange carries the unpacked integer sums.  NCCL reduces 8-, 32- and 64-bit
 integers but not 16-bit ones, so the exchange takes the int8 wire type (W
-times the largest code value at most 127); int16 configurations are refused.
+times the largest code value at most 127) or the fp16 one (at most 2048: every
+partial sum of such integers is an exact fp16 value, in any order); int16
+configurations are refused.
 
 The library calls are reached through an ``ops`` object (``GpuOps`` by
 default) so that the host-side orchestration can be exercised with other
@@ -71,9 +73,9 @@ class DataParallelStep:
         rc = gq_validate(cfg, self.W, self.d)
         if rc != GQ_OK:
             raise GQError(rc, "DataParallelStep")
-        if cfg.wire_dtype != torch.int8:
-            raise ValueError("the exchange sums int8 integers: NCCL has no 16-bit integer "
-                             "reduction, so use wire='int8' (W * max code value <= 127)")
+        if cfg.wire_dtype not in (torch.int8, torch.float16):
+            raise ValueError("NCCL has no 16-bit integer reduction: use wire='int8' (W * max "
+                             "code value <= 127) or wire='f16' (<= 2048)")
         self.cfg = replace(cfg, worker0=self.rank * self.w_local)
         self.ops = ops if ops is not None else GpuOps()
         dev = torch.device(device) if device is not None else torch.device("cuda")

@@ -86,6 +86,8 @@ extern "C" {
 /* Sum (wire) types of the aggregated codes. */
 #define GQ_WIRE_INT8 1
 #define GQ_WIRE_INT16 2
+#define GQ_WIRE_F16 3 /* fp16 holding the integer sum, exact for |sum| <= 2048: for
+                          collectives that reduce fp16 but not 16-bit integers (NCCL) */
 
 typedef struct {
     int levels;       /* GQ_UNIFORM, GQ_EXP or GQ_LOG */
@@ -93,7 +95,7 @@ typedef struct {
     int L;            /* EXP: 1 <= L <= 15, levels 0 and 2^-(L-1) ... 1 */
     int bits;         /* packed code width: 4, 5, 8 or 16; must hold 2*max+1 codes */
     int scale_kind;   /* GQ_SCALE_L2 or GQ_SCALE_MAXABS */
-    int wire;         /* GQ_WIRE_INT8 or GQ_WIRE_INT16: element type of the sum */
+    int wire;         /* GQ_WIRE_INT8, GQ_WIRE_INT16 or GQ_WIRE_F16: type of the sum */
     int ef;           /* 1: error feedback on (e buffer given), 0: off */
     float alpha;      /* LOG: curvature a > 0 of the log map */
     unsigned long long seed; /* Philox key */
@@ -112,7 +114,8 @@ GQ_API const char* gq_status_string(int status);
 
 /* Host-side check of a configuration for W workers and d coordinates:
  * level parameters in range, `bits` wide enough for the codes, and the
- * overflow rule: W * max|value| <= 127 (INT8) or <= 32767 (INT16), where the
+ * overflow rule: W * max|value| <= 127 (INT8), <= 32767 (INT16) or <= 2048 (F16,
+ * where every partial sum of such values is an exact fp16 integer), where the
  * per-worker max value is s (UNIFORM) or 2^(L-1) units of the finest level
  * (EXP, whose sums count in those units).  Returns GQ_OK, GQ_ERR_ARG or
  * GQ_ERR_OVERFLOW. */

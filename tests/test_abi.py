@@ -94,7 +94,8 @@ def test_bad_levels_and_sizes(gq):
         gq.GQ_ERR_ARG
     assert gq.gq_validate(cfg(gq, levels=7), 1, 10) == gq.GQ_ERR_ARG
     assert gq.gq_validate(cfg(gq, scale_kind=5), 1, 10) == gq.GQ_ERR_ARG
-    assert gq.gq_validate(cfg(gq, wire=3), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, wire=4), 1, 10) == gq.GQ_ERR_ARG
+    assert gq.gq_validate(cfg(gq, wire=0), 1, 10) == gq.GQ_ERR_ARG
     assert gq.gq_validate(cfg(gq), 0, 10) == gq.GQ_ERR_ARG
     assert gq.gq_validate(cfg(gq), 1, -1) == gq.GQ_ERR_ARG
     assert gq.gq_validate(cfg(gq), 1, 0) == gq.GQ_OK

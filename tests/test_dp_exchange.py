@@ -40,7 +40,7 @@ class OracleOps:
         codes = self.o.quantize(g.numpy(), ev, seed=cfg.seed, step=cfg.step, S=S,
                                 worker0=cfg.worker0, **self._kw(cfg))
         sum_out.copy_(torch.from_numpy(self.o.aggregate(codes, levels=self._kw(cfg)["levels"],
-                                                        L=cfg.L)))
+                                                        L=cfg.L)).to(sum_out.dtype))
         if cfg.ef and e is not None:
             e.copy_(torch.from_numpy(self.o.error_feedback(g.numpy(), ev, codes, S=S,
                                                            **self._kw(cfg))))
@@ -64,6 +64,8 @@ CASES = {
     "uniform": dict(levels="uniform", s=15, bits=5, wire="int8", seed=3, step=2),
     "exp_ef": dict(levels="exp", L=5, bits=4, wire="int8", scale_kind="maxabs", ef=True,
                    seed=5, step=1),
+    "exp_f16": dict(levels="exp", L=8, bits=5, wire="f16", seed=6, step=0),
+    "u127_f16": dict(s=127, bits=8, wire="f16", ef=True, seed=7, step=3),
 }
 
 
@@ -93,7 +95,8 @@ def _rank_main(rank, world, port, case, w_local, d, outdir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("case,w_local", [("uniform", 1), ("uniform", 3), ("exp_ef", 2)])
+@pytest.mark.parametrize("case,w_local", [("uniform", 1), ("uniform", 3), ("exp_ef", 2),
+                                           ("exp_f16", 2), ("u127_f16", 4)])
 def test_two_ranks_equal_the_single_process_step(oracle, tmp_path, case, w_local):
     world, d = 2, 700
     mp.start_processes(_rank_main, args=(world, _free_port(), case, w_local, d, str(tmp_path)),
@@ -122,10 +125,18 @@ def test_two_ranks_equal_the_single_process_step(oracle, tmp_path, case, w_local
 
 
 def test_overflow_rule_uses_the_total_worker_count(oracle):
-    """W = world * W_local decides the wire type: 9 workers of s = 15 overflow int8."""
+    """W = world * W_local decides the wire type: 9 workers of s = 15 overflow int8;
+    the fp16 sums hold integers up to 2048."""
     import allreduce_compatible_gradient_global_b200 as gq
     assert gq.gq_validate(gq.GQConfig(s=15, bits=5, wire="int8"), 8, 100) == gq.GQ_OK
     assert gq.gq_validate(gq.GQConfig(s=15, bits=5, wire="int8"), 9, 100) == gq.GQ_ERR_OVERFLOW
+    assert gq.gq_validate(gq.GQConfig(s=127, bits=8, wire="f16"), 16, 100) == gq.GQ_OK
+    assert gq.gq_validate(gq.GQConfig(s=127, bits=8, wire="f16"), 17, 100) == \
+        gq.GQ_ERR_OVERFLOW
+    assert gq.gq_validate(gq.GQConfig(levels="exp", L=8, bits=5, wire="f16"), 16, 100) == \
+        gq.GQ_OK
+    assert gq.gq_validate(gq.GQConfig(levels="exp", L=8, bits=5, wire="f16"), 17, 100) == \
+        gq.GQ_ERR_OVERFLOW
 
 
 def test_worker0_offsets_the_uniform_streams(oracle):

@@ -36,7 +36,9 @@ def gq():
 
 @pytest.mark.parametrize("kw,ef", [(dict(s=15, bits=5, wire="int8"), False),
                                    (dict(levels="exp", L=5, bits=4, wire="int8",
-                                         scale_kind="maxabs"), True)])
+                                         scale_kind="maxabs"), True),
+                                   (dict(levels="exp", L=8, bits=5, wire="f16"), False),
+                                   (dict(s=127, bits=8, wire="f16"), True)])
 def test_nccl_single_rank_equals_fused_step(gq, kw, ef):
     from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))

@@ -100,6 +100,9 @@ CASES = [
     (40, 8192, dict(s=3, bits=4, wire="int8")),           # rows too many to stage: register path
     (16, 50000, dict(s=7, bits=4, wire="int8", seed=8)),  # 16 staged rows
     (8, 1 << 20, dict(s=15, bits=5, wire="int8", seed=9)),  # many tiles per block
+    (8, 30001, dict(s=127, bits=8, wire="f16", seed=12)),   # fp16 sums, ragged tail
+    (8, 40000, dict(levels="exp", L=8, bits=5, wire="f16", scale_kind="maxabs")),
+    (16, 5003, dict(s=127, bits=8, wire="f16")),            # |sum| up to 2032
 ]
 
 
@@ -112,7 +115,7 @@ def test_fused_step_matches_oracle(gq, oracle, W, d, kw):
     check_against_oracle(oracle, cfg, g.cpu().numpy(), None, r)
 
 
-@pytest.mark.parametrize("W,d,kw", [c for c in CASES if c[1] in (33, 4099, 65580, 40000, 7777)])
+@pytest.mark.parametrize("W,d,kw", [c for c in CASES if c[1] in (33, 4099, 65580, 40000, 7777, 30001)])
 def test_split_pipeline_equals_fused(gq, oracle, W, d, kw):
     cfg = gq.GQConfig(**{"seed": 99, **kw})
     g = synthetic.make_gradients(W, d, "laplace", seed=d, device="cuda", seg=512, lo=-5, hi=-2)
@@ -128,6 +131,7 @@ def test_split_pipeline_equals_fused(gq, oracle, W, d, kw):
     (8, 30000, dict(s=127, bits=8, wire="int16")),
     (4, 4097, dict(s=15, bits=5, wire="int8")),
     (8, 20000, dict(levels="exp", L=8, bits=5, wire="int16", scale_kind="maxabs")),
+    (16, 5003, dict(s=127, bits=8, wire="f16")),
 ])
 def test_error_feedback_steps_match_oracle(gq, oracle, W, d, kw, split):
     cfg = gq.GQConfig(**{"ef": True, "seed": 77, **kw})
