@@ -510,6 +510,7 @@ GQ_API int gq_logq_quantize(const float* x_dev, int W, int nmats, const int* row
     a.W = W;
     a.nmats = nmats;
     a.step = cfg->step;
+    a.worker0 = cfg->worker0;
     a.seed_lo = (uint32_t)cfg->seed;
     a.seed_hi = (uint32_t)(cfg->seed >> 32);
     a.alpha = cfg->alpha;

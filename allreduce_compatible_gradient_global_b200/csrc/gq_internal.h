@@ -129,6 +129,7 @@ struct LogqArgs {
     int count;  // matrices in this launch
     long long off[kLogqGroup + 1];
     unsigned int step;
+    unsigned int worker0;  // Philox worker index of row 0
     unsigned int seed_lo, seed_hi;
     float alpha;
     WsHeader* hdr;

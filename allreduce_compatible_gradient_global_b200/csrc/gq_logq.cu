@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kLogqThreads) logq_quantize_kernel(const __gri
 
     // four consecutive entries per thread share one Philox block
     for (long long q = threadIdx.x; 4 * q < n; q += kLogqThreads) {
-        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, a.step, (uint32_t)w), k0, k1);
+        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, a.step, a.worker0 + (uint32_t)w), k0, k1);
         const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {

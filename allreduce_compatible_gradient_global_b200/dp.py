@@ -103,3 +103,89 @@ class DataParallelStep:
             if rc != GQ_OK:
                 raise GQError(rc, "DataParallelStep")
         return self.out
+
+
+def gather_rows(local, out, group=None):
+    """All-gather each rank's [w_local][n] rows into out [world * w_local][n],
+    rank-major, so that row i of out is global worker i."""
+    world = dist.get_world_size(group)
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(out, local, group=group)
+    else:
+        dist.all_gather(list(out.chunk(world)), local, group=group)
+
+
+class DataParallelLqsgdStep:
+    """LQ-SGD ("Trustworthy Efficient Communication for Distributed Learning
+    using LQ-SGD Algorithm", review, "What carries the argument": P and Q
+    log-quantized before they are exchanged, error fed back) with each rank
+    holding W_local workers' matrices.
+
+    Log codes are not additive, so the exchange of a factor is an all-gather of
+    every worker's int8 codes and per-matrix max-abs values; every rank then
+    decodes and sums all W workers in ascending worker order, exactly as the
+    single-GPU step does, so P_hat, Q and Ghat are the same on every rank and
+    equal the single-GPU step's.  Per step: gq_psgd_project (local) ->
+    gq_logq_quantize (local, worker offset) -> all-gather -> gq_logq_decode_sum
+    -> gq_psgd_orthonormalize -> gq_psgd_back_project (local) ->
+    gq_logq_quantize -> all-gather -> gq_logq_decode_sum -> gq_psgd_mean ->
+    gq_psgd_reconstruct."""
+
+    def __init__(self, shapes, w_local=1, alpha=10.0, seed=0, group=None, device=None):
+        from . import gq_psgd_workspace_bytes
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.sh = shapes
+        self.w_local = int(w_local)
+        self.W = self.world * self.w_local
+        self.alpha, self.seed = float(alpha), int(seed)
+        dev = torch.device(device) if device is not None else torch.device("cuda")
+        sh, wl, W = shapes, self.w_local, self.W
+        f32, i8 = torch.float32, torch.int8
+        self.pw = torch.empty((wl, sh.ptotal), dtype=f32, device=dev)
+        self.qw = torch.empty((wl, sh.qtotal), dtype=f32, device=dev)
+        self.codes_p_l = torch.empty((wl, sh.ptotal), dtype=i8, device=dev)
+        self.codes_q_l = torch.empty((wl, sh.qtotal), dtype=i8, device=dev)
+        self.max_p_l = torch.empty((wl, sh.nmats), dtype=f32, device=dev)
+        self.max_q_l = torch.empty((wl, sh.nmats), dtype=f32, device=dev)
+        self.codes_p = torch.empty((W, sh.ptotal), dtype=i8, device=dev)
+        self.codes_q = torch.empty((W, sh.qtotal), dtype=i8, device=dev)
+        self.max_p = torch.empty((W, sh.nmats), dtype=f32, device=dev)
+        self.max_q = torch.empty((W, sh.nmats), dtype=f32, device=dev)
+        self.qsum = torch.empty(sh.qtotal, dtype=f32, device=dev)
+        self.ws = torch.zeros(gq_psgd_workspace_bytes(wl, sh), dtype=torch.uint8, device=dev)
+        if dev.type == "cuda":
+            gq_workspace_init(self.ws)
+        self.ranks = [sh.rank] * sh.nmats
+
+    def __call__(self, g, m, p, q, ghat, have_prev, step, check=False):
+        """g, m: this rank's [w_local][sum n m] rows (m is the state, updated);
+        p, q: P_hat and the mean Q (the same on every rank, updated); ghat:
+        [sum n m] output, or None."""
+        from . import (gq_logq_decode_sum, gq_logq_quantize, gq_psgd_back_project,
+                       gq_psgd_mean, gq_psgd_orthonormalize, gq_psgd_project,
+                       gq_psgd_reconstruct)
+        sh = self.sh
+        cfg = GQConfig(levels="log", alpha=self.alpha, seed=self.seed, step=2 * int(step),
+                       worker0=self.rank * self.w_local)
+        gq_psgd_project(g, m, sh, have_prev, p, q, self.pw)
+        gq_logq_quantize(self.pw, sh.rows, self.ranks, cfg, self.max_p_l, self.codes_p_l, self.ws)
+        gather_rows(self.codes_p_l, self.codes_p, self.group)
+        gather_rows(self.max_p_l, self.max_p, self.group)
+        gq_logq_decode_sum(self.codes_p, self.max_p, sh.rows, self.ranks, cfg, p)
+        gq_psgd_orthonormalize(p, sh)
+        gq_psgd_back_project(m, p, sh, self.qw, self.ws)
+        cfg.step = 2 * int(step) + 1
+        gq_logq_quantize(self.qw, sh.cols, self.ranks, cfg, self.max_q_l, self.codes_q_l, self.ws)
+        gather_rows(self.codes_q_l, self.codes_q, self.group)
+        gather_rows(self.max_q_l, self.max_q, self.group)
+        gq_logq_decode_sum(self.codes_q, self.max_q, sh.cols, self.ranks, cfg, self.qsum)
+        gq_psgd_mean(self.qsum, q, self.W)
+        if ghat is not None:
+            gq_psgd_reconstruct(p, q, sh, ghat)
+        if check:
+            rc = gq_get_device_status(self.ws)
+            if rc != GQ_OK:
+                raise GQError(rc, "DataParallelLqsgdStep")
+        return ghat

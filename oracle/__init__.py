@@ -52,6 +52,7 @@ def lib():
         L.gqo_decode_mean.argtypes = [P, i64, i32, i32, i32, i32, f32, P]
         L.gqo_error_feedback.argtypes = [P, P, P, i32, i64, i32, i32, i32, f32, P]
         L.gqo_logq_quantize.argtypes = [P, i32, i32, P, f32, u64, u32, P, P]
+        L.gqo_logq_quantize_workers.argtypes = [P, i32, i32, P, f32, u64, u32, u32, P, P]
         L.gqo_logq_decode_sum.argtypes = [P, P, i32, i32, P, f32, P]
         L.gqo_logq_map.argtypes = [f32, f32]
         L.gqo_logq_map.restype = f32
@@ -253,15 +254,15 @@ def lowrank_fma(P, Q):
     return out
 
 
-def logq_quantize(x, sizes, *, alpha=10.0, seed=0, step=0):
+def logq_quantize(x, sizes, *, alpha=10.0, seed=0, step=0, worker0=0):
     """x: [W][sum(sizes)] float32.  Returns (maxabs[W][nmats], codes int8)."""
     x = _f32(x)
     W = x.shape[0]
     sz = np.ascontiguousarray(sizes, dtype=np.int64)
     mx = np.zeros((W, sz.size), np.float32)
     codes = np.zeros(x.shape, np.int8)
-    _check(lib().gqo_logq_quantize(_p(x), W, sz.size, _p(sz), alpha, seed, step, _p(mx),
-                                   _p(codes)), "logq_quantize")
+    _check(lib().gqo_logq_quantize_workers(_p(x), W, sz.size, _p(sz), alpha, seed, step,
+                                           int(worker0), _p(mx), _p(codes)), "logq_quantize")
     return mx, codes
 
 

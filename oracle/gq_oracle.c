@@ -444,6 +444,15 @@ int gqo_logq_quantize(const float* x, int W, int nmats, const int64_t* sizes,
                       float alpha, uint64_t seed, uint32_t step,
                       float* maxabs_out, int8_t* codes_out)
 {
+    return gqo_logq_quantize_workers(x, W, nmats, sizes, alpha, seed, step, 0u,
+                                     maxabs_out, codes_out);
+}
+
+int gqo_logq_quantize_workers(const float* x, int W, int nmats,
+                              const int64_t* sizes, float alpha, uint64_t seed,
+                              uint32_t step, uint32_t worker0,
+                              float* maxabs_out, int8_t* codes_out)
+{
     if (!x || !sizes || !maxabs_out || !codes_out || W < 1 || nmats < 1)
         return -1;
     if (!(alpha > 0.0f) || !isfinite(alpha)) return -1;
@@ -479,7 +488,7 @@ int gqo_logq_quantize(const float* x, int W, int nmats, const int64_t* sizes,
                 if (!(y <= 127.0f)) y = 127.0f;
                 float l = floorf(y);
                 float p = y - l;
-                uint32_t f = gqo_uniform_bits(seed, tag, step, (uint32_t)w,
+                uint32_t f = gqo_uniform_bits(seed, tag, step, worker0 + (uint32_t)w,
                                               (uint64_t)i);
                 int32_t k = (int32_t)l + round_up(p, f);
                 cm[i] = (int8_t)(sign_negative(xm[i]) ? -k : k);

@@ -138,6 +138,12 @@ int gqo_logq_quantize(const float* x, int W, int nmats, const int64_t* sizes,
                       float alpha, uint64_t seed, uint32_t step,
                       float* maxabs_out, int8_t* codes_out);
 
+/* The same with row w drawing its uniforms as worker worker0 + w. */
+int gqo_logq_quantize_workers(const float* x, int W, int nmats,
+                              const int64_t* sizes, float alpha, uint64_t seed,
+                              uint32_t step, uint32_t worker0,
+                              float* maxabs_out, int8_t* codes_out);
+
 /* [LQ] Eq. (6) decode of every worker's codes, fp32 sum over workers in
  * ascending order.  out is [total]. */
 int gqo_logq_decode_sum(const int8_t* codes, const float* maxabs, int W,

@@ -159,3 +159,41 @@ def test_int16_wire_is_refused():
             DataParallelStep(gq.GQConfig(s=127, bits=8, wire="int16"), 100, device="cpu")
     finally:
         dist.destroy_process_group()
+
+
+def _gather_main(rank, world, port, outdir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from allreduce_compatible_gradient_global_b200.dp import gather_rows
+        w_local, sizes = 2, np.array([300, 120], np.int64)
+        W = world * w_local
+        x = synthetic.make_gradients(W, int(sizes.sum()), "normal", seed=4).numpy()
+        rows = slice(rank * w_local, (rank + 1) * w_local)
+        mx_l, codes_l = oracle.logq_quantize(x[rows], sizes, seed=9, step=2,
+                                             worker0=rank * w_local)
+        codes = torch.empty((W, int(sizes.sum())), dtype=torch.int8)
+        mx = torch.empty((W, sizes.size), dtype=torch.float32)
+        gather_rows(torch.from_numpy(codes_l), codes)
+        gather_rows(torch.from_numpy(mx_l), mx)
+        total = oracle.logq_decode_sum(codes.numpy(), mx.numpy(), sizes)
+        np.save(os.path.join(outdir, f"lq{rank}.npy"), total)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gathered_log_codes_decode_like_one_process(oracle, tmp_path):
+    """Each rank log-quantizes its own workers (worker offset rank * W_local),
+    the codes and max-abs values are all-gathered rank-major, and every rank's
+    decoded sum equals the single-process decode of all workers, bit for bit."""
+    world = 2
+    mp.start_processes(_gather_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    sizes = np.array([300, 120], np.int64)
+    x = synthetic.make_gradients(4, int(sizes.sum()), "normal", seed=4).numpy()
+    mx, codes = oracle.logq_quantize(x, sizes, seed=9, step=2)
+    ref = oracle.logq_decode_sum(codes, mx, sizes)
+    for r in range(world):
+        got = np.load(tmp_path / f"lq{r}.npy")
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), r

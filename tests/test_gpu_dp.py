@@ -67,3 +67,38 @@ def test_nccl_single_rank_equals_fused_step(gq, kw, ef):
                 assert torch.equal(e1, e2), t
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("r", [1, 5])
+def test_nccl_single_rank_lqsgd_equals_whole_step(gq, r):
+    """The LQ-SGD exchange (all-gather of the factor codes) on one NCCL rank
+    holding all W workers equals gq_lqsgd_step bit for bit, state included."""
+    from allreduce_compatible_gradient_global_b200.dp import DataParallelLqsgdStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        W = 4
+        sh = gq.PsgdShapes([256, 100], [128, 64], r)
+
+        def state():
+            m = torch.zeros((W, sh.total), dtype=torch.float32, device="cuda")
+            p = torch.zeros(sh.ptotal, dtype=torch.float32, device="cuda")
+            q = synthetic.make_gradients(1, sh.qtotal, "normal", seed=3, device="cuda")[0]
+            return m, p, q, torch.empty(sh.total, dtype=torch.float32, device="cuda")
+
+        a, b = state(), state()
+        ws = torch.empty(gq.gq_psgd_workspace_bytes(W, sh), dtype=torch.uint8, device="cuda")
+        gq.gq_workspace_init(ws)
+        dp = DataParallelLqsgdStep(sh, w_local=W, alpha=10.0, seed=12)
+        for t in range(3):
+            g = synthetic.make_gradients(W, sh.total, "normal", seed=40 + t, device="cuda")
+            dp(g, a[0], a[1], a[2], a[3], t > 0, t, check=True)
+            gq.gq_lqsgd_step(g, b[0], sh, t > 0, gq.GQConfig(levels="log", alpha=10.0, seed=12,
+                                                             step=t), b[1], b[2], b[3], ws)
+            torch.cuda.synchronize()
+            for x, y in zip(a, b):
+                assert torch.equal(x, y), t
+    finally:
+        dist.destroy_process_group()
