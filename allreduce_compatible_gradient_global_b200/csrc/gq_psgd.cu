@@ -226,6 +226,152 @@ __global__ void __launch_bounds__(kPsgdThreads, ProjCfg<R>::min_blocks)
 }
 
 // ---------------------------------------------------------------------------
+// project, ranks 5..8 (every m a multiple of 4): the same arithmetic and
+// summation order as psgd_project_kernel, but the Q slice of each column step
+// is staged once per block.  All 8 warps of a block walk the same column
+// groups (j4 = lane + 32 it) of their own two rows, so one copy of Q's rows
+// 4 j4 .. 4 j4 + 3 serves the block instead of being re-read by every row
+// pair through L1.  Ring of kQStages slots: per warp the lane-private G / M
+// vectors, per block the shared Q slice; one block barrier per step makes the
+// step's copies visible and frees the slot the previous step read.
+// ---------------------------------------------------------------------------
+constexpr int kQStages = 3;
+
+template <int R, bool HAVE_PREV>
+__global__ void __launch_bounds__(kPsgdThreads, ProjCfg<R>::min_blocks)
+    psgd_project_q_kernel(const __grid_constant__ PsgdArgs a) {
+    extern __shared__ float4 qsm[];
+    float4* qring = qsm;                                    // [kQStages][32 * R]
+    float4* vring = qsm + kQStages * 32 * R;                // [8 warps][kQStages][4][32]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float4* ring = vring + (size_t)warp * kQStages * 4 * 32;
+    for (long long t = blockIdx.x; t < a.tile0[a.count]; t += gridDim.x) {
+        const int l = matrix_of(a, t);
+        const long long lt = t - a.tile0[l];
+        const int n = a.rows[l], m = a.cols[l];
+        const long long row_tiles = (n + kProjRowsPerTile - 1) / kProjRowsPerTile;
+        const int w = (int)(lt / row_tiles);
+        const int i0 = (int)(lt - (long long)w * row_tiles) * kProjRowsPerTile +
+                       warp * kProjRowsPerWarp;
+        const bool row0 = i0 < n, two = i0 + 1 < n;  // warp-uniform
+        const long long base = (long long)w * a.total + a.goff[l];
+        const float* g0 = a.g + base + (long long)(row0 ? i0 : 0) * m;
+        float* m0 = a.m + base + (long long)(row0 ? i0 : 0) * m;
+        const float* qm = a.q + a.qoff[l];
+        float p0[R], p1[R];
+        if (HAVE_PREV) {
+            const float* pr = a.p + a.poff[l] + (long long)(row0 ? i0 : 0) * R;
+#pragma unroll
+            for (int k = 0; k < R; ++k) {
+                p0[k] = row0 ? __ldg(pr + k) : 0.f;
+                p1[k] = two ? __ldg(pr + R + k) : 0.f;
+            }
+        }
+        float acc0[R], acc1[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) acc0[k] = acc1[k] = 0.f;
+        const float4* gA4 = reinterpret_cast<const float4*>(g0);
+        const float4* mA4 = reinterpret_cast<const float4*>(m0);
+        const float4* gB4 = reinterpret_cast<const float4*>(g0 + m);
+        const float4* mB4 = reinterpret_cast<const float4*>(m0 + m);
+        const int m4 = m >> 2;
+        const int nit = (m4 + 31) / 32;  // the same for every warp of the block
+        // thread x < 32 R copies float4 k = x % R of the Q rows of lane x / R
+        const int qx = threadIdx.x, ql = qx / R, qk = qx - ql * R;
+        auto issue = [&](int it) {
+            const int slot = it % kQStages;
+            const int j4 = lane + it * 32;
+            if (row0 && j4 < m4) {
+                float4* d = ring + slot * 128 + lane;
+                cp_async16(d, gA4 + j4);
+                cp_async16(d + 32, mA4 + j4);
+                if (two) {
+                    cp_async16(d + 64, gB4 + j4);
+                    cp_async16(d + 96, mB4 + j4);
+                }
+            }
+            const int qj4 = ql + it * 32;
+            if (qx < 32 * R && qj4 < m4)
+                cp_async16(qring + slot * 32 * R + qx,
+                           reinterpret_cast<const float4*>(qm + (long long)qj4 * 4 * R) + qk);
+        };
+        __syncthreads();  // the previous tile's reads of the rings are done
+#pragma unroll
+        for (int it = 0; it < kQStages - 1; ++it) {
+            if (it < nit) issue(it);
+            cp_async_commit();
+        }
+        for (int it = 0; it < nit; ++it) {
+            cp_async_wait<kQStages - 2>();  // this thread's copies of step `it` landed
+            __syncthreads();                // ... and every thread's; slot (it - 1) is free
+            if (it + kQStages - 1 < nit) issue(it + kQStages - 1);
+            cp_async_commit();
+            const int j4 = lane + it * 32;
+            if (!row0 || j4 >= m4) continue;
+            const int slot = it % kQStages;
+            float q[4 * R];  // rows 4 j4 .. 4 j4 + 3 of Q, R values each
+            const float4* qs = qring + slot * 32 * R + lane * R;
+#pragma unroll
+            for (int k = 0; k < R; ++k) {
+                const float4 v = qs[k];
+                q[4 * k] = v.x;
+                q[4 * k + 1] = v.y;
+                q[4 * k + 2] = v.z;
+                q[4 * k + 3] = v.w;
+            }
+            const float4* d = ring + slot * 128 + lane;
+            const float4 ga = d[0], ma = d[32];
+            float4 gb = make_float4(0.f, 0.f, 0.f, 0.f), mb = gb;
+            if (two) {
+                gb = d[64];
+                mb = d[96];
+            }
+            const float gA[4] = {ga.x, ga.y, ga.z, ga.w}, mA[4] = {ma.x, ma.y, ma.z, ma.w};
+            const float gB[4] = {gb.x, gb.y, gb.z, gb.w}, mB[4] = {mb.x, mb.y, mb.z, mb.w};
+            float outA[4], outB[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float* qc = q + c * R;
+                float eA = mA[c], eB = mB[c];
+                if (HAVE_PREV) {
+                    eA = __fsub_rn(eA, lowrank_value<R>(p0, qc));
+                    eB = __fsub_rn(eB, lowrank_value<R>(p1, qc));
+                }
+                outA[c] = __fadd_rn(gA[c], eA);
+                outB[c] = __fadd_rn(gB[c], eB);
+#pragma unroll
+                for (int k = 0; k < R; ++k) {
+                    acc0[k] = __fmaf_rn(outA[c], qc[k], acc0[k]);
+                    acc1[k] = __fmaf_rn(outB[c], qc[k], acc1[k]);
+                }
+            }
+            __stcs(reinterpret_cast<float4*>(m0) + j4, make_float4(outA[0], outA[1], outA[2], outA[3]));
+            if (two)
+                __stcs(reinterpret_cast<float4*>(m0 + m) + j4,
+                       make_float4(outB[0], outB[1], outB[2], outB[3]));
+        }
+        cp_async_wait<0>();
+        if (!row0) continue;  // warp-uniform; no barrier follows before the next tile's
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+            for (int k = 0; k < R; ++k) {
+                acc0[k] = __fadd_rn(acc0[k], __shfl_xor_sync(kFull, acc0[k], o));
+                acc1[k] = __fadd_rn(acc1[k], __shfl_xor_sync(kFull, acc1[k], o));
+            }
+        }
+        if (lane == 0) {
+            float* pw = a.pw + (long long)w * a.ptotal + a.poff[l] + (long long)i0 * R;
+#pragma unroll
+            for (int k = 0; k < R; ++k) {
+                pw[k] = acc0[k];
+                if (two) pw[R + k] = acc1[k];
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // orthonormalize: one block per matrix, modified Gram-Schmidt over the columns
 // in order, fp64 sums in a fixed order, fp32 storage.  A column whose
 // remaining norm is 0 stays 0.
@@ -482,8 +628,39 @@ static cudaError_t project_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <int R, bool HP>
+static cudaError_t project_q_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
+    auto kern = psgd_project_q_kernel<R, HP>;
+    const size_t smem = (size_t)kQStages * (32 * R + 8 * 4 * 32) * sizeof(float4);
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<resident_grid((const void*)kern, smem, a.tile0[a.count], sms), kPsgdThreads, smem,
+           st>>>(a);
+    return cudaGetLastError();
+}
+
+#ifndef GQ_PSGD_SHARED_Q
+#define GQ_PSGD_SHARED_Q 1
+#endif
+#ifndef GQ_PSGD_SHARED_Q_MIN_RANK
+#define GQ_PSGD_SHARED_Q_MIN_RANK 1
+#endif
+
 cudaError_t launch_psgd_project(const PsgdArgs& a, bool vec, int sms, cudaStream_t st) {
     const bool hp = a.have_prev != 0;
+    if (GQ_PSGD_SHARED_Q && vec && a.rank >= GQ_PSGD_SHARED_Q_MIN_RANK) {
+        switch (a.rank) {
+            case 1: return hp ? project_q_inst<1, true>(a, sms, st) : project_q_inst<1, false>(a, sms, st);
+            case 2: return hp ? project_q_inst<2, true>(a, sms, st) : project_q_inst<2, false>(a, sms, st);
+            case 3: return hp ? project_q_inst<3, true>(a, sms, st) : project_q_inst<3, false>(a, sms, st);
+            case 4: return hp ? project_q_inst<4, true>(a, sms, st) : project_q_inst<4, false>(a, sms, st);
+            case 5: return hp ? project_q_inst<5, true>(a, sms, st) : project_q_inst<5, false>(a, sms, st);
+            case 6: return hp ? project_q_inst<6, true>(a, sms, st) : project_q_inst<6, false>(a, sms, st);
+            case 7: return hp ? project_q_inst<7, true>(a, sms, st) : project_q_inst<7, false>(a, sms, st);
+            default: return hp ? project_q_inst<8, true>(a, sms, st) : project_q_inst<8, false>(a, sms, st);
+        }
+    }
 #define GQ_PROJ(RR)                                                           \
     case RR:                                                                  \
         if (hp) return vec ? project_inst<RR, true, true>(a, sms, st)         \
