@@ -731,7 +731,7 @@ PsgdWs psgd_ws(const PsgdShape& s) {
     return o;
 }
 
-enum class PsgdTiles { Project, Back, Reduce, Reconstruct };
+enum class PsgdTiles { Project, Back, Reduce, Reconstruct, ReconstructCols };
 
 // Fill the matrices l0 .. l0 + count - 1 and their work-tile prefix.
 void psgd_group(PsgdArgs& a, const PsgdShape& s, int l0, int count, PsgdTiles kind) {
@@ -766,6 +766,9 @@ void psgd_group(PsgdArgs& a, const PsgdShape& s, int l0, int count, PsgdTiles ki
                 tiles = (long long)s.W * (((long long)m * s.rank + 255) / 256);
                 break;
             case PsgdTiles::Reconstruct: tiles = (n + 7) / 8; break;
+            case PsgdTiles::ReconstructCols:
+                tiles = (long long)((m + 1023) / 1024) * ((n + 127) / 128);
+                break;
         }
         a.tile0[i + 1] = a.tile0[i] + tiles;
     }
@@ -896,8 +899,14 @@ GQ_API int gq_psgd_reconstruct(const float* p_dev, const float* q_dev, int nmats
     a.out = ghat_dev;
     for (int l0 = 0; l0 < nmats; l0 += kPsgdGroup) {
         const int count = nmats - l0 < kPsgdGroup ? nmats - l0 : kPsgdGroup;
-        psgd_group(a, s, l0, count, PsgdTiles::Reconstruct);
-        if ((rc = cuda_status(launch_psgd_reconstruct(a, s.vec, sm_count(), stream)))) return rc;
+        if (s.vec) {
+            psgd_group(a, s, l0, count, PsgdTiles::ReconstructCols);
+            rc = cuda_status(launch_psgd_reconstruct_cols(a, sm_count(), stream));
+        } else {
+            psgd_group(a, s, l0, count, PsgdTiles::Reconstruct);
+            rc = cuda_status(launch_psgd_reconstruct(a, s.vec, sm_count(), stream));
+        }
+        if (rc) return rc;
     }
     return GQ_OK;
 }

@@ -594,6 +594,58 @@ __global__ void __launch_bounds__(kPsgdThreads)
 }
 
 // ---------------------------------------------------------------------------
+// reconstruct, every m a multiple of 4: tiles of (matrix, 1024 columns, 128
+// rows).  A thread keeps the Q rows of its 4 columns in registers and runs
+// down the tile's rows, whose P_hat rows are staged in shared memory; each
+// row is one coalesced 16-byte store per thread.  Same fma chain as above.
+// ---------------------------------------------------------------------------
+constexpr int kRecRows = 128;
+
+template <int R>
+__global__ void __launch_bounds__(kPsgdThreads)
+    psgd_reconstruct_cols_kernel(const __grid_constant__ PsgdArgs a) {
+    constexpr int RP = Padded<R>::value;
+    __shared__ __align__(16) float ps[kRecRows * RP];
+    for (long long t = blockIdx.x; t < a.tile0[a.count]; t += gridDim.x) {
+        const int l = matrix_of(a, t);
+        const long long lt = t - a.tile0[l];
+        const int n = a.rows[l], m = a.cols[l];
+        const int rtiles = (n + kRecRows - 1) / kRecRows;
+        const int ct = (int)(lt / rtiles);
+        const int r0 = (int)(lt - (long long)ct * rtiles) * kRecRows;
+        const int r1 = min(n, r0 + kRecRows);
+        __syncthreads();  // the previous tile's reads of ps are done
+        for (int x = threadIdx.x; x < (r1 - r0) * RP; x += kPsgdThreads) {
+            const int i = x / RP, k = x - i * RP;
+            ps[x] = k < R ? __ldg(a.p + a.poff[l] + (long long)(r0 + i) * R + k) : 0.f;
+        }
+        __syncthreads();
+        const int j = ct * kBackColsPerTile + 4 * threadIdx.x;
+        if (j >= m) continue;
+        float q[4 * R];
+        const float4* q4 = reinterpret_cast<const float4*>(a.q + a.qoff[l] + (long long)j * R);
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const float4 v = __ldg(q4 + k);
+            q[4 * k] = v.x;
+            q[4 * k + 1] = v.y;
+            q[4 * k + 2] = v.z;
+            q[4 * k + 3] = v.w;
+        }
+        float* out = a.out + a.goff[l] + (long long)r0 * m + j;
+        for (int i = 0; i < r1 - r0; ++i) {
+            float p[R];
+            const float* pr = ps + i * RP;
+#pragma unroll
+            for (int k = 0; k < R; ++k) p[k] = pr[k];
+            __stcs(reinterpret_cast<float4*>(out + (long long)i * m),
+                   make_float4(lowrank_value<R>(p, q), lowrank_value<R>(p, q + R),
+                               lowrank_value<R>(p, q + 2 * R), lowrank_value<R>(p, q + 3 * R)));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
 static int grid_for(long long tiles, int sms, int per_sm) {
@@ -721,6 +773,22 @@ cudaError_t launch_psgd_mean(const float* qsum, float* q, long long len, int W, 
                              cudaStream_t st) {
     const long long blocks = (len + 255) / 256;
     psgd_mean_kernel<<<grid_for(blocks, sms, 8), 256, 0, st>>>(qsum, q, len, (float)W);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_psgd_reconstruct_cols(const PsgdArgs& a, int sms, cudaStream_t st) {
+#define GQ_RECC(RR)                                                                    \
+    case RR: {                                                                         \
+        auto kern = psgd_reconstruct_cols_kernel<RR>;                                  \
+        kern<<<resident_grid((const void*)kern, 0, a.tile0[a.count], sms), kPsgdThreads, 0, \
+               st>>>(a);                                                               \
+        break;                                                                         \
+    }
+    switch (a.rank) {
+        GQ_PSGD_RANKS(GQ_RECC)
+        default: return cudaErrorInvalidValue;
+    }
+#undef GQ_RECC
     return cudaGetLastError();
 }
 

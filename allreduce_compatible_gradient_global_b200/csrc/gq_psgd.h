@@ -39,6 +39,8 @@ cudaError_t launch_psgd_back_reduce(const PsgdArgs& a, int sms, cudaStream_t st)
 cudaError_t launch_psgd_mean(const float* qsum, float* q, long long len, int W, int sms,
                              cudaStream_t st);
 cudaError_t launch_psgd_reconstruct(const PsgdArgs& a, bool vec, int sms, cudaStream_t st);
+// Every m a multiple of 4; tiles of (matrix, 1024 columns, 128 rows).
+cudaError_t launch_psgd_reconstruct_cols(const PsgdArgs& a, int sms, cudaStream_t st);
 
 }  // namespace gq
 
