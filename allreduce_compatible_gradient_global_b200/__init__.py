@@ -47,7 +47,7 @@ class _Config(ctypes.Structure):
                 ("bits", ctypes.c_int), ("scale_kind", ctypes.c_int), ("wire", ctypes.c_int),
                 ("ef", ctypes.c_int), ("alpha", ctypes.c_float),
                 ("seed", ctypes.c_ulonglong), ("step", ctypes.c_uint),
-                ("worker0", ctypes.c_uint)]
+                ("worker0", ctypes.c_uint), ("coord0", ctypes.c_ulonglong)]
 
 
 @dataclass
@@ -64,6 +64,7 @@ class GQConfig:
     seed: int = 0
     step: int = 0
     worker0: int = 0
+    coord0: int = 0
 
     def c(self) -> _Config:
         lv = _LEVELS.get(self.levels, self.levels)
@@ -72,7 +73,7 @@ class GQConfig:
         return _Config(int(lv), int(self.s), int(self.L), int(self.bits), int(sk), int(wr),
                        1 if self.ef else 0, float(self.alpha),
                        int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.step) & 0xFFFFFFFF,
-                       int(self.worker0) & 0xFFFFFFFF)
+                       int(self.worker0) & 0xFFFFFFFF, int(self.coord0) & 0xFFFFFFFFFFFFFFFF)
 
     @property
     def wire_dtype(self):

@@ -189,6 +189,7 @@ void fill_quant_args(QuantArgs& a, const gq_config* cfg, int W, long long d) {
     a.wire = cfg->wire;
     a.step = cfg->step;
     a.worker0 = cfg->worker0;
+    a.q0 = cfg->coord0 >> 2;
     a.L = cfg->L;
     a.smax = (float)cfg->s;
     a.finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, -(cfg->L - 1)) : 1.0f;
@@ -233,6 +234,7 @@ GQ_API const char* gq_status_string(int status) {
 }
 
 GQ_API int gq_validate(const gq_config* cfg, int W, long long d) {
+    if (!cfg || (cfg->coord0 & 3ull) != 0) return GQ_ERR_ARG;
     int rc = check_levels(cfg);
     if (rc) return rc;
     if ((rc = check_sizes(W, d))) return rc;

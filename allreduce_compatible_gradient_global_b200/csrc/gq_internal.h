@@ -52,6 +52,7 @@ struct QuantArgs {
     int wire;  // bytes per sum element
     unsigned int step;
     unsigned int worker0;  // Philox worker index of row 0
+    unsigned long long q0;  // coord0 / 4: Philox block counter of column 0
     int L;
     float smax;        // (float)s
     float finest;      // 2^-(L-1)

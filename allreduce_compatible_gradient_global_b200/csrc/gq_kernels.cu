@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, GQ_QUANT_MIN_BLOCKS)
             c = __ldg(a.bq_unit + (blk >> a.bucket_shift));
         }
         const long long j0 = (blk << 7) + (lane << 2);
-        const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
+        const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane + a.q0;
         int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
         for (int wb = 0; wb < a.W; wb += kWorkerBatch) {
             float4 gv[kWorkerBatch], ev[kWorkerBatch];

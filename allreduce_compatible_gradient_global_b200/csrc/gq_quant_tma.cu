@@ -231,7 +231,9 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
             }
             const long long j0 = (blk << 7) + (lane << 2);
             const bool in = j0 < a.d;  // d % 4 == 0: all four or none
-            const unsigned long long q = (unsigned long long)(blk << 5) + (unsigned)lane;
+            // WOFF = 0: no worker or coordinate offset (the common case)
+            const unsigned long long q =
+                (unsigned long long)(blk << 5) + (unsigned)lane + (WOFF ? a.q0 : 0ull);
             const float* stage = buf + (size_t)s * rows * kTmaTile + warp * 128 + lane * 4;
             unsigned char* codes_blk = a.codes + blk * (16 * BITS);
             // uniform levels accumulate the biased patterns (code + kCodeBias);
@@ -350,9 +352,10 @@ template <int LEVELS, int BITS, bool EF>
 static cudaError_t launch_tma_w(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
     // per-bucket scales get their own instantiations, so the global-scale
     // kernel keeps one multiplier in a register for the whole launch
-    // The unrolled W = 8 kernel gets the worker offset of a data-parallel rank
-    // as a separate instantiation; the general one always adds it.
-    const bool woff = a.worker0 != 0;
+    // The unrolled W = 8 kernel gets the worker and coordinate offsets of a
+    // data-parallel rank or chunk as a separate instantiation; the general one
+    // always adds them.
+    const bool woff = a.worker0 != 0 || a.q0 != 0;
     if (a.bq_mult) {
         if (GQ_TMA_SPECIALIZE_W8 && a.W == 8)
             return woff ? launch_tma_inst<LEVELS, BITS, EF, 8, true, true>(a, stages, grid, st)

@@ -25,6 +25,12 @@ times the largest code value at most 127) or the fp16 one (at most 2048: every
 partial sum of such integers is an exact fp16 value, in any order); int16
 configurations are refused.
 
+With ``chunks > 1`` (one worker per rank) the quantization of chunk k + 1
+overlaps the all-reduce of chunk k: each chunk is quantized with
+``gq_config.coord0`` set to its first coordinate, so it draws exactly the
+uniforms it would draw in the whole vector, and the result is bit-identical
+to the unchunked exchange.
+
 The library calls are reached through an ``ops`` object (``GpuOps`` by
 default) so that the host-side orchestration can be exercised with other
 backends in tests; the product path always uses ``GpuOps``.
@@ -63,7 +69,7 @@ class DataParallelStep:
     rule is checked for the total W = world * w_local."""
 
     def __init__(self, cfg: GQConfig, d: int, w_local: int = 1, group=None, device=None,
-                 ops=None):
+                 ops=None, chunks: int = 1):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -76,6 +82,14 @@ class DataParallelStep:
         if cfg.wire_dtype not in (torch.int8, torch.float16):
             raise ValueError("NCCL has no 16-bit integer reduction: use wire='int8' (W * max "
                              "code value <= 127) or wire='f16' (<= 2048)")
+        self.chunks = max(1, int(chunks))
+        if self.chunks > 1 and self.w_local != 1:
+            raise ValueError("chunked exchange: one worker per rank (the rows of a chunk must "
+                             "be contiguous)")
+        # chunk boundaries on 128-coordinate blocks (keeps every chunk's sum,
+        # mean and gradient pointers 16-byte aligned)
+        step_c = -(-self.d // (self.chunks * 128)) * 128 if self.chunks > 1 else self.d
+        self.bounds = [(c0, min(self.d, c0 + step_c)) for c0 in range(0, self.d, max(1, step_c))]
         self.cfg = replace(cfg, worker0=self.rank * self.w_local)
         self.ops = ops if ops is not None else GpuOps()
         dev = torch.device(device) if device is not None else torch.device("cuda")
@@ -95,9 +109,24 @@ class DataParallelStep:
         ef = e if self.cfg.ef else None
         self.ops.global_norm(g, ef, self.cfg, self.scale, self.ws)
         dist.all_reduce(self.scale, op=dist.ReduceOp.MAX, group=self.group)
-        self.ops.quantize_sum(g, e, self.cfg, self.scale, self.sum, self.ws)
-        dist.all_reduce(self.sum, op=dist.ReduceOp.SUM, group=self.group)
-        self.ops.decode(self.sum, self.W, self.cfg, self.scale, self.out, self.ws)
+        if self.chunks == 1:
+            self.ops.quantize_sum(g, e, self.cfg, self.scale, self.sum, self.ws)
+            dist.all_reduce(self.sum, op=dist.ReduceOp.SUM, group=self.group)
+            self.ops.decode(self.sum, self.W, self.cfg, self.scale, self.out, self.ws)
+        else:
+            # quantize chunk k + 1 while the all-reduce of chunk k runs on the
+            # collective's own stream; decode each chunk once its sum is in
+            works = []
+            for c0, c1 in self.bounds:
+                cfg_k = replace(self.cfg, coord0=c0)
+                self.ops.quantize_sum(g[:, c0:c1], None if e is None else e[:, c0:c1], cfg_k,
+                                      self.scale, self.sum[c0:c1], self.ws)
+                works.append(dist.all_reduce(self.sum[c0:c1], op=dist.ReduceOp.SUM,
+                                             group=self.group, async_op=True))
+            for (c0, c1), work in zip(self.bounds, works):
+                work.wait()
+                self.ops.decode(self.sum[c0:c1], self.W, self.cfg, self.scale,
+                                self.out[c0:c1], self.ws)
         if check:
             rc = self.ops.status(self.ws)
             if rc != GQ_OK:

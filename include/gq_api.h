@@ -104,6 +104,11 @@ typedef struct {
                                 worker0 + w): 0 when all W workers are on this GPU;
                                 the rank's first worker in a real data-parallel
                                 exchange, so that every worker keeps its own stream */
+    unsigned long long coord0; /* coordinate index of column 0: column j draws the
+                                  uniforms of coordinate coord0 + j, so a chunk of a
+                                  longer vector quantizes exactly as in the whole
+                                  vector; a multiple of 4 (else GQ_ERR_ARG); 0 for a
+                                  whole vector */
 } gq_config;
 
 /* Library version (major*10000 + minor*100 + patch). */

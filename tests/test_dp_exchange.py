@@ -37,8 +37,11 @@ class OracleOps:
     def quantize_sum(self, g, e, cfg, scale, sum_out, ws):
         S = np.float32(scale[0].item())
         ev = e.numpy() if (cfg.ef and e is not None) else None
+        n = g.shape[1]
         codes = self.o.quantize(g.numpy(), ev, seed=cfg.seed, step=cfg.step, S=S,
-                                worker0=cfg.worker0, **self._kw(cfg))
+                                worker0=cfg.worker0,
+                                js=np.arange(cfg.coord0, cfg.coord0 + n, dtype=np.int64),
+                                **self._kw(cfg))
         sum_out.copy_(torch.from_numpy(self.o.aggregate(codes, levels=self._kw(cfg)["levels"],
                                                         L=cfg.L)).to(sum_out.dtype))
         if cfg.ef and e is not None:
@@ -69,7 +72,7 @@ CASES = {
 }
 
 
-def _rank_main(rank, world, port, case, w_local, d, outdir):
+def _rank_main(rank, world, port, case, w_local, d, outdir, chunks=1):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
     dist.init_process_group("gloo", rank=rank, world_size=world,
@@ -85,7 +88,8 @@ def _rank_main(rank, world, port, case, w_local, d, outdir):
         rows = slice(rank * w_local, (rank + 1) * w_local)
         g = g_all[rows].clone()
         e = e_all[rows].clone()
-        stepper = DataParallelStep(cfg, d, w_local=w_local, device="cpu", ops=OracleOps(oracle))
+        stepper = DataParallelStep(cfg, d, w_local=w_local, device="cpu", ops=OracleOps(oracle),
+                                   chunks=chunks)
         outs = []
         for t in range(2):
             outs.append(stepper(g, e, step=cfg.step + t).clone().numpy())
@@ -95,11 +99,16 @@ def _rank_main(rank, world, port, case, w_local, d, outdir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("case,w_local", [("uniform", 1), ("uniform", 3), ("exp_ef", 2),
-                                           ("exp_f16", 2), ("u127_f16", 4)])
-def test_two_ranks_equal_the_single_process_step(oracle, tmp_path, case, w_local):
+@pytest.mark.parametrize("case,w_local,chunks", [("uniform", 1, 1), ("uniform", 3, 1),
+                                                  ("exp_ef", 2, 1), ("exp_f16", 2, 1),
+                                                  ("u127_f16", 4, 1), ("uniform", 1, 3),
+                                                  ("exp_ef", 1, 2)])
+def test_two_ranks_equal_the_single_process_step(oracle, tmp_path, case, w_local, chunks):
+    """chunks > 1: chunk k + 1 is quantized while chunk k is all-reduced; each
+    chunk draws the uniforms of its own coordinates (coord0)."""
     world, d = 2, 700
-    mp.start_processes(_rank_main, args=(world, _free_port(), case, w_local, d, str(tmp_path)),
+    mp.start_processes(_rank_main, args=(world, _free_port(), case, w_local, d, str(tmp_path),
+                                         chunks),
                        nprocs=world, join=True, start_method="spawn")
     import allreduce_compatible_gradient_global_b200 as gq
     cfg = gq.GQConfig(**CASES[case])

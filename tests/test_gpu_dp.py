@@ -102,3 +102,34 @@ def test_nccl_single_rank_lqsgd_equals_whole_step(gq, r):
                 assert torch.equal(x, y), t
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("chunks,kw", [(4, dict(s=15, bits=5, wire="int8", ef=True)),
+                                       (3, dict(levels="exp", L=8, bits=5, wire="f16"))])
+def test_nccl_chunked_exchange_equals_unchunked(gq, chunks, kw):
+    """Chunk k + 1 is quantized while chunk k is all-reduced (NCCL, async);
+    with each chunk drawing the uniforms of its own coordinates the mean and
+    the error buffer are bit-identical to the unchunked exchange."""
+    from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        d = 1_000_003 - 3  # a multiple of 4, not of 128
+        cfg = gq.GQConfig(seed=5, **kw)
+        g = synthetic.make_gradients(1, d, "student_t3", seed=2, device="cuda", seg=4096,
+                                     lo=-4, hi=0)
+        e1, e2 = torch.zeros_like(g), torch.zeros_like(g)
+        whole = DataParallelStep(cfg, d)
+        parts = DataParallelStep(cfg, d, chunks=chunks)
+        assert len(parts.bounds) == chunks
+        for t in range(2):
+            a = whole(g, e1, step=t, check=True).clone()
+            b = parts(g, e2, step=t, check=True).clone()
+            torch.cuda.synchronize()
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32)), t
+            if cfg.ef:
+                assert torch.equal(e1, e2), t
+    finally:
+        dist.destroy_process_group()

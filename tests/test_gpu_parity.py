@@ -283,3 +283,25 @@ def test_rounding_decision_boundaries(gq, oracle, d):
     ref = oracle.quantize(v[None, :], s=s, seed=seed, step=step, S=np.float32(s))
     assert (ref == -1).sum() >= 100
     assert np.array_equal(codes.cpu().numpy(), oracle.pack(ref, 5))
+
+
+@pytest.mark.parametrize("W,d,c0,n", [(4, 10000, 4096, 3000), (8, 65536, 1024, 40000),
+                                      (3, 20001, 4, 999)])
+def test_coordinate_offset_equals_the_whole_vector(gq, W, d, c0, n):
+    """A chunk quantized with coord0 = its first coordinate (and the whole
+    vector's scale) gives the same integer sums and means as those columns of
+    the whole vector."""
+    cfg = gq.GQConfig(s=15, bits=5, wire="int8", seed=31, step=2)
+    g = synthetic.make_gradients(W, d, "normal", seed=d, device="cuda")
+    whole = gq.StepBuffers(cfg, W, d)
+    gq.gq_step_fused(g, None, cfg, whole.scale, whole.norms, whole.codes, whole.sum, whole.out,
+                     whole.ws)
+    chunk = g[:, c0:c0 + n].contiguous()
+    part = gq.StepBuffers(cfg, W, n)
+    cfgc = gq.GQConfig(s=15, bits=5, wire="int8", seed=31, step=2, coord0=c0)
+    gq.gq_quantize_aggregate(chunk, None, cfgc, whole.scale, part.codes, part.sum, part.out,
+                             part.ws)
+    assert gq.gq_get_device_status(part.ws) == gq.GQ_OK
+    torch.cuda.synchronize()
+    assert torch.equal(part.sum, whole.sum[c0:c0 + n])
+    assert torch.equal(part.out.view(torch.int32), whole.out[c0:c0 + n].view(torch.int32))
