@@ -70,19 +70,27 @@ class Machine:
     pass2_efficiency: float = 0.76  # measured fraction of hbm the fused pass reaches
 
 
-def dp_step_seconds(d, ranks, bits=8, sum_bytes=1, m=Machine(), compressed=True):
+def dp_step_seconds(d, ranks, bits=8, sum_bytes=1, m=Machine(), compressed=True, chunks=1):
     """One data-parallel gradient exchange with one worker per GPU.
 
     compressed: norm pass + MAX all-reduce of 4 bytes + quantize pass + SUM
     all-reduce of d * sum_bytes + decode pass (read the sum, write the mean).
-    Otherwise: a SUM all-reduce of 4 * d bytes."""
+    Otherwise: a SUM all-reduce of 4 * d bytes.  chunks > 1: the quantize pass
+    and the SUM all-reduce run as a K-stage pipeline (chunk k + 1 quantized
+    while chunk k is summed), each chunk paying its own launch and alpha."""
     if not compressed:
         return ring_allreduce_seconds(4.0 * d, ranks, m.link, m.allreduce_alpha)
     norm = m.launch + 4.0 * d / m.hbm
-    quant = m.launch + (4.0 * d + d * bits / 8.0) / (m.hbm * m.pass2_efficiency)
+    scale = ring_allreduce_seconds(4.0, ranks, m.link, m.allreduce_alpha)
     decode = m.launch + (sum_bytes * d + 4.0 * d) / m.hbm
-    return (norm + ring_allreduce_seconds(4.0, ranks, m.link, m.allreduce_alpha) + quant
-            + ring_allreduce_seconds(sum_bytes * d, ranks, m.link, m.allreduce_alpha) + decode)
+    K = max(1, int(chunks))
+    dk = d / K
+    quant = m.launch + (4.0 * dk + dk * bits / 8.0) / (m.hbm * m.pass2_efficiency)
+    summ = ring_allreduce_seconds(sum_bytes * dk, ranks, m.link, m.allreduce_alpha)
+    # a K-stage two-resource pipeline: first quantize, then the slower of the
+    # two stages K - 1 times, then the last all-reduce
+    pipelined = quant + (K - 1) * max(quant, summ) + summ
+    return norm + scale + pipelined + decode
 
 
 def crossover_d(ranks, bits=8, sum_bytes=1, m=Machine(), lo=1, hi=1 << 40):

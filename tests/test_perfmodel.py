@@ -60,3 +60,23 @@ def test_large_d_ratio_follows_the_byte_counts():
                       + 2 * (n - 1) / n / m.link)
     per_coord_slow = 2 * (n - 1) / n * 4 / m.link
     assert math.isclose(slow / fast, per_coord_slow / per_coord_fast, rel_tol=1e-3)
+
+
+def test_chunked_pipeline_model():
+    """One chunk is the unpipelined step; many chunks hide the shorter of the
+    two stages, down to the launch and alpha each chunk pays."""
+    from allreduce_compatible_gradient_global_b200 import perfmodel as pm
+    m = pm.Machine()
+    d, N = 25_557_032, 8
+    one = pm.dp_step_seconds(d, N, m=m, chunks=1)
+    four = pm.dp_step_seconds(d, N, m=m, chunks=4)
+    assert four < one
+    # the lower bound: norm + scale + decode + the slower stage over all of d
+    norm = m.launch + 4.0 * d / m.hbm
+    scale = pm.ring_allreduce_seconds(4.0, N, m.link, m.allreduce_alpha)
+    decode = m.launch + (d + 4.0 * d) / m.hbm
+    slow = max(m.launch + 5.0 * d / (m.hbm * m.pass2_efficiency),
+               pm.ring_allreduce_seconds(float(d), N, m.link, m.allreduce_alpha))
+    assert four > norm + scale + decode + slow * 0.99
+    # too many chunks pay alpha and launches again
+    assert pm.dp_step_seconds(d, N, m=m, chunks=4096) > four
