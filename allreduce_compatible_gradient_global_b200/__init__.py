@@ -47,7 +47,8 @@ class _Config(ctypes.Structure):
                 ("bits", ctypes.c_int), ("scale_kind", ctypes.c_int), ("wire", ctypes.c_int),
                 ("ef", ctypes.c_int), ("alpha", ctypes.c_float),
                 ("seed", ctypes.c_ulonglong), ("step", ctypes.c_uint),
-                ("worker0", ctypes.c_uint), ("coord0", ctypes.c_ulonglong)]
+                ("worker0", ctypes.c_uint), ("coord0", ctypes.c_ulonglong),
+                ("step_dev", ctypes.c_void_p)]
 
 
 @dataclass
@@ -65,6 +66,7 @@ class GQConfig:
     step: int = 0
     worker0: int = 0
     coord0: int = 0
+    step_dev: object = None  # a CUDA uint32 / int32 tensor of one element, or None
 
     def c(self) -> _Config:
         lv = _LEVELS.get(self.levels, self.levels)
@@ -73,7 +75,8 @@ class GQConfig:
         return _Config(int(lv), int(self.s), int(self.L), int(self.bits), int(sk), int(wr),
                        1 if self.ef else 0, float(self.alpha),
                        int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.step) & 0xFFFFFFFF,
-                       int(self.worker0) & 0xFFFFFFFF, int(self.coord0) & 0xFFFFFFFFFFFFFFFF)
+                       int(self.worker0) & 0xFFFFFFFF, int(self.coord0) & 0xFFFFFFFFFFFFFFFF,
+                       None if self.step_dev is None else self.step_dev.data_ptr())
 
     @property
     def wire_dtype(self):
@@ -107,6 +110,7 @@ def _load():
         "gq_quantize_aggregate": ([P, P, I, LL, CP, P, P, P, P, P, P], I),
         "gq_step_fused": ([P, P, I, LL, CP, P, P, P, P, P, P, P], I),
         "gq_step_fused_host": ([P, P, P, I, LL, CP, P, P, P, P, P, P, P, P], I),
+        "gq_advance_step": ([P, ctypes.c_uint, P], I),
         "gq_bucket_count": ([LL, I, ctypes.POINTER(LL)], I),
         "gq_bucket_workspace_bytes": ([CP, I, LL, I, ctypes.POINTER(ctypes.c_size_t)], I),
         "gq_bucket_scales": ([P, P, I, LL, I, CP, P, P, P], I),
@@ -225,6 +229,15 @@ def gq_selftest_wait_timeout(ws, limit_ms=50, stream=None):
     _check(lib().gq_selftest_wait_timeout(_ptr(ws), int(limit_ms), _stream(stream)),
            "gq_selftest_wait_timeout")
     return lib().gq_get_device_status(_ptr(ws), _stream(stream))
+
+
+def gq_advance_step(step_dev, by=1, stream=None):
+    """step_dev[0] += by on the stream (the device step counter of a captured
+    step graph; see GQConfig.step_dev)."""
+    _need(step_dev, step_dev.dtype, (1,), "step_dev")
+    if step_dev.element_size() != 4:
+        raise TypeError("step_dev: a 32-bit integer tensor")
+    _check(lib().gq_advance_step(_ptr(step_dev), int(by), _stream(stream)), "gq_advance_step")
 
 
 # ------------------------------------------------------------------ the path

@@ -190,6 +190,7 @@ void fill_quant_args(QuantArgs& a, const gq_config* cfg, int W, long long d) {
     a.step = cfg->step;
     a.worker0 = cfg->worker0;
     a.q0 = cfg->coord0 >> 2;
+    a.step_dev = cfg->step_dev;
     a.L = cfg->L;
     a.smax = (float)cfg->s;
     a.finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, -(cfg->L - 1)) : 1.0f;
@@ -233,8 +234,15 @@ GQ_API const char* gq_status_string(int status) {
     }
 }
 
+GQ_API int gq_advance_step(unsigned int* step_dev, unsigned int by, cudaStream_t stream) {
+    if (!step_dev) return GQ_ERR_ARG;
+    if (!aligned4(step_dev)) return GQ_ERR_ALIGN;
+    return cuda_status(launch_advance_step(step_dev, by, stream));
+}
+
 GQ_API int gq_validate(const gq_config* cfg, int W, long long d) {
     if (!cfg || (cfg->coord0 & 3ull) != 0) return GQ_ERR_ARG;
+    if (cfg->step_dev && !aligned4(cfg->step_dev)) return GQ_ERR_ALIGN;
     int rc = check_levels(cfg);
     if (rc) return rc;
     if ((rc = check_sizes(W, d))) return rc;
@@ -513,6 +521,7 @@ GQ_API int gq_logq_quantize(const float* x_dev, int W, int nmats, const int* row
     a.nmats = nmats;
     a.step = cfg->step;
     a.worker0 = cfg->worker0;
+    a.step_dev = cfg->step_dev;
     a.seed_lo = (uint32_t)cfg->seed;
     a.seed_hi = (uint32_t)(cfg->seed >> 32);
     a.alpha = cfg->alpha;
@@ -920,6 +929,8 @@ GQ_API int gq_lqsgd_step(const float* g_dev, float* m_dev, int W, int nmats,
     const NvtxRange nvtx_range("gq_lqsgd_step");
     if (!cfg || cfg->levels != GQ_LOG || !(cfg->alpha > 0.f) || !(cfg->alpha <= 3.0e38f))
         return GQ_ERR_ARG;
+    // the step derives two streams (2t, 2t + 1) on the host: no device step word
+    if (cfg->step_dev) return GQ_ERR_ARG;
     PsgdShape s;
     int rc = psgd_shape(W, nmats, rows_host, cols_host, rank, s);
     if (rc) return rc;

@@ -53,6 +53,7 @@ struct QuantArgs {
     unsigned int step;
     unsigned int worker0;  // Philox worker index of row 0
     unsigned long long q0;  // coord0 / 4: Philox block counter of column 0
+    const unsigned int* step_dev;  // non-null: the step is read here, not from `step`
     int L;
     float smax;        // (float)s
     float finest;      // 2^-(L-1)
@@ -131,10 +132,25 @@ struct LogqArgs {
     long long off[kLogqGroup + 1];
     unsigned int step;
     unsigned int worker0;  // Philox worker index of row 0
+    const unsigned int* step_dev;  // non-null: the step is read here, not from `step`
     unsigned int seed_lo, seed_hi;
     float alpha;
     WsHeader* hdr;
 };
+
+// Raise a kernel's dynamic shared-memory limit only when a larger size is
+// needed on this device: `limits` is the caller's per-kernel record (one
+// static array per kernel instantiation).  Later calls, including calls made
+// while a stream is being captured into a graph, then make no runtime call.
+inline cudaError_t ensure_dynamic_smem(const void* kern, size_t smem, int* limits) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if ((int)smem <= __atomic_load_n(&limits[dev], __ATOMIC_ACQUIRE)) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) __atomic_store_n(&limits[dev], (int)smem, __ATOMIC_RELEASE);
+    return e;
+}
 
 // Launchers (return the cudaGetLastError() of the launch).
 cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st);
@@ -154,6 +170,7 @@ cudaError_t launch_quant_tma(const QuantArgs& a, int levels, int bits, bool ef, 
 cudaError_t launch_wait_timeout_selftest(WsHeader* hdr, unsigned long long limit_ns,
                                          cudaStream_t st);
 cudaError_t launch_bucket_scales(const BucketArgs& a, int sms, cudaStream_t st);
+cudaError_t launch_advance_step(unsigned int* step_dev, unsigned int by, cudaStream_t st);
 cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st);
 cudaError_t launch_logq_decode(const LogqArgs& a, cudaStream_t st);
 

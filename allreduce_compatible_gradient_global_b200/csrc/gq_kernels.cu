@@ -308,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, GQ_QUANT_MIN_BLOCKS)
     const long long nwarps = ((long long)gridDim.x * kThreads) >> 5;
     float aq, c;
     scale_constants<LEVELS>(__ldg(a.scale), a.smax, a.finest, aq, c);
+    const uint32_t step = a.step_dev ? __ldg(a.step_dev) : a.step;
     Packer<BITS> pk;
     pk.init(lane);
 
@@ -334,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, GQ_QUANT_MIN_BLOCKS)
                 if (wb + i < a.W) {
                     const int w = wb + i;
                     const float4 v = EF ? add4(gv[i], ev[i]) : gv[i];
-                    const uint4 rnd = philox10(philox_counter(q, a.step, a.worker0 + (uint32_t)w), a.rk);
+                    const uint4 rnd = philox10(philox_counter(q, step, a.worker0 + (uint32_t)w), a.rk);
                     const int c0 = quantize_one<LEVELS>(v.x, aq, a, rnd.x);
                     const int c1 = quantize_one<LEVELS>(v.y, aq, a, rnd.y);
                     const int c2 = quantize_one<LEVELS>(v.z, aq, a, rnd.z);
@@ -516,6 +517,14 @@ cudaError_t launch_dequant(const DequantArgs& a, int levels, int bits, bool vec,
         }
     }
 #undef GQ_DQ
+    return cudaGetLastError();
+}
+
+// The device step counter of captured step graphs.
+__global__ void advance_step_kernel(unsigned int* step_dev, unsigned int by) { *step_dev += by; }
+
+cudaError_t launch_advance_step(unsigned int* step_dev, unsigned int by, cudaStream_t st) {
+    advance_step_kernel<<<1, 1, 0, st>>>(step_dev, by);
     return cudaGetLastError();
 }
 

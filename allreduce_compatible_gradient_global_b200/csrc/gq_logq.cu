@@ -60,10 +60,11 @@ __global__ void __launch_bounds__(kLogqThreads) logq_quantize_kernel(const __gri
     const float alpha = a.alpha;
     const float lam = log1pf(alpha);
     const uint32_t k0 = a.seed_lo, k1 = a.seed_hi ^ (0x4C510000u | (uint32_t)m);
+    const uint32_t step = a.step_dev ? __ldg(a.step_dev) : a.step;
 
     // four consecutive entries per thread share one Philox block
     for (long long q = threadIdx.x; 4 * q < n; q += kLogqThreads) {
-        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, a.step, a.worker0 + (uint32_t)w), k0, k1);
+        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, step, a.worker0 + (uint32_t)w), k0, k1);
         const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {

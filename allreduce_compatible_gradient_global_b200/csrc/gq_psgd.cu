@@ -671,8 +671,8 @@ static cudaError_t project_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
     auto kern = psgd_project_kernel<R, HP, VEC>;
     const size_t smem = VEC ? (size_t)ProjCfg<R>::stages * 4 * kPsgdThreads * sizeof(float4) : 0;
     if (VEC) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static int limits[64] = {};
+        const cudaError_t e = ensure_dynamic_smem((const void*)kern, smem, limits);
         if (e != cudaSuccess) return e;
     }
     kern<<<resident_grid((const void*)kern, smem, a.tile0[a.count], sms), kPsgdThreads, smem,
@@ -684,8 +684,8 @@ template <int R, bool HP>
 static cudaError_t project_q_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
     auto kern = psgd_project_q_kernel<R, HP>;
     const size_t smem = (size_t)kQStages * (32 * R + 8 * 4 * 32) * sizeof(float4);
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int limits[64] = {};
+    const cudaError_t e = ensure_dynamic_smem((const void*)kern, smem, limits);
     if (e != cudaSuccess) return e;
     kern<<<resident_grid((const void*)kern, smem, a.tile0[a.count], sms), kPsgdThreads, smem,
            st>>>(a);
@@ -746,8 +746,8 @@ template <int R, bool VEC>
 static cudaError_t back_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
     auto kern = psgd_back_kernel<R, VEC>;
     const size_t smem = psgd_back_smem(R, a.chunk_rows, VEC);
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int limits[64] = {};
+    const cudaError_t e = ensure_dynamic_smem((const void*)kern, smem, limits);
     if (e != cudaSuccess) return e;
     kern<<<resident_grid((const void*)kern, smem, a.tile0[a.count], sms), kPsgdThreads, smem,
            st>>>(a);

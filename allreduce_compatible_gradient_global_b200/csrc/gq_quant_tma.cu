@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
             c = __fmul_rn(S, a.finest);
         }
     }
+    const uint32_t step = a.step_dev ? __ldg(a.step_dev) : a.step;
     Packer<BITS> pk;
     pk.init(lane);
     const long long row_bytes = a.row_bytes;
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 }
                 // WOFF = 0: the worker word is the loop constant w (the common case)
                 const uint32_t wid = WOFF ? a.worker0 + (uint32_t)w : (uint32_t)w;
-                const uint4 rnd = philox10(philox_counter(q, a.step, wid), a.rk);
+                const uint4 rnd = philox10(philox_counter(q, step, wid), a.rk);
                 unsigned char* cdst = codes_blk + (long long)w * row_bytes;
                 float4 qv;  // the values Q(v) in units of c, as floats
                 if (LEVELS == 0) {
@@ -342,7 +343,8 @@ template <int LEVELS, int BITS, bool EF, int WT, bool BQ, bool WOFF>
 static cudaError_t launch_tma_inst(const QuantArgs& a, int stages, int grid, cudaStream_t st) {
     auto kern = quant_tma_kernel<LEVELS, BITS, EF, WT, BQ, WOFF>;
     const size_t smem = tma_smem_bytes(a.W, EF, stages);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int limits[64] = {};
+    cudaError_t e = ensure_dynamic_smem((const void*)kern, smem, limits);
     if (e != cudaSuccess) return e;
     kern<<<grid, kTmaThreads, smem, st>>>(a, stages);
     return cudaGetLastError();

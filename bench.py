@@ -400,10 +400,44 @@ def time_step_pair(gq, g, e, cfg, buf, K, warmup, stream):
     return n, q, step
 
 
+def time_step_graph(gq, g, cfg, W, d, K):
+    """Mean step time (ms) of the step captured once in a CUDA graph (norm pass,
+    fused pass, device step counter advanced in the graph) and replayed K times."""
+    step_dev = torch.zeros(1, dtype=torch.int32, device=g.device)
+    gcfg = gq.GQConfig(levels=cfg.levels, s=cfg.s, L=cfg.L, bits=cfg.bits,
+                       scale_kind=cfg.scale_kind, wire=cfg.wire, ef=cfg.ef, seed=cfg.seed,
+                       step_dev=step_dev)
+    buf = gq.StepBuffers(gcfg, W, d)
+    gq.gq_step_fused(g, buf.e, gcfg, buf.scale, buf.norms, buf.codes, buf.sum, buf.out, buf.ws)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        gq.gq_step_fused(g, buf.e, gcfg, buf.scale, buf.norms, buf.codes, buf.sum, buf.out,
+                         buf.ws)
+        gq.gq_advance_step(step_dev)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(K):
+        graph.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    if gq.gq_get_device_status(buf.ws) != gq.GQ_OK:
+        raise RuntimeError("device flag raised in the graph replay")
+    ms = t0.elapsed_time(t1) / K
+    del graph, buf
+    return ms
+
+
 def run_sweep(args):
     """Step throughput over d = 2^16 ... 2^30 at W = 8 (uniform s = 15, 5-bit
     codes, int8 sums, L2 scale), error feedback off and on.  Below ~2^22 the
-    second read can hit L2; the fraction is reported but not targeted there."""
+    second read can hit L2; the fraction is reported but not targeted there.
+    Each row also times the step captured in a CUDA graph and replayed, which
+    removes the host's per-call cost where the step is launch-bound."""
     import allreduce_compatible_gradient_global_b200 as gq
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
@@ -419,13 +453,16 @@ def run_sweep(args):
             buf = gq.StepBuffers(cfg, W, d)
             K = max(20, min(400, int(2e9 // (4 * W * d))))
             n_ms, q_ms, step_ms = time_step_pair(gq, g, buf.e, cfg, buf, K, 5, stream)
+            graph_ms = time_step_graph(gq, g, cfg, W, d, K)
             p1, p2 = algorithmic_bytes(gq, cfg, W, d)
             rows.append({"d": d, "log2_d": lg, "ef": ef, "steps": K,
                          "step_ms": round(step_ms, 5), "norm_ms": round(n_ms, 5),
                          "quant_ms": round(q_ms, 5),
                          "grad_gbs": round(4 * W * d / (step_ms * 1e-3) / 1e9, 1),
                          "step_frac": round((p1 + p2) / (step_ms * 1e-3) / 1e9 / peak, 4),
-                         "quant_frac": round(p2 / (q_ms * 1e-3) / 1e9 / peak, 4)})
+                         "quant_frac": round(p2 / (q_ms * 1e-3) / 1e9 / peak, 4),
+                         "graph_step_ms": round(graph_ms, 5),
+                         "graph_grad_gbs": round(4 * W * d / (graph_ms * 1e-3) / 1e9, 1)})
             del g, buf
             torch.cuda.empty_cache()
     return {"metric": METRIC, "mode": "sweep", "unit": "GB/s", "peak": peak,

@@ -109,10 +109,18 @@ typedef struct {
                                   longer vector quantizes exactly as in the whole
                                   vector; a multiple of 4 (else GQ_ERR_ARG); 0 for a
                                   whole vector */
+    const unsigned int* step_dev; /* NULL, or a device word holding the step: the
+                                     kernels then read the step there instead of
+                                     `step`, so a captured CUDA graph can replay
+                                     steps (advance it with gq_advance_step) */
 } gq_config;
 
 /* Library version (major*10000 + minor*100 + patch). */
 GQ_API int gq_version(void);
+
+/* *step_dev += by, on `stream` (one thread): the device step counter that
+ * gq_config.step_dev points to, advanced inside a captured step graph. */
+GQ_API int gq_advance_step(unsigned int* step_dev, unsigned int by, cudaStream_t stream);
 
 /* Static text for a status code. */
 GQ_API const char* gq_status_string(int status);
@@ -385,7 +393,8 @@ GQ_API int gq_psgd_reconstruct(const float* p_dev, const float* q_dev, int nmats
  * gq_psgd_orthonormalize (p_dev becomes P_hat); gq_psgd_back_project;
  * gq_logq_quantize of the Q_w (step 2*cfg->step + 1) and gq_logq_decode_sum;
  * gq_psgd_mean into q_dev; and, if ghat_dev is not NULL,
- * gq_psgd_reconstruct.  cfg: levels GQ_LOG, alpha, seed, step.  The P and Q
+ * gq_psgd_reconstruct.  cfg: levels GQ_LOG, alpha, seed, step (step_dev must
+ * be NULL: the two streams are derived from `step` on the host).  The P and Q
  * calls draw different uniform streams, so the two factors never share
  * one. */
 GQ_API int gq_lqsgd_step(const float* g_dev, float* m_dev, int W, int nmats,

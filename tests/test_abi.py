@@ -219,7 +219,8 @@ def test_psgd_entry_points_reject_before_launch(gq):
 def test_workspace_and_config_layout(gq):
     """gq_config carries worker0 and coord0 after step (the C struct and the
     binding agree); coord0 must be a multiple of 4."""
-    assert ctypes.sizeof(gq._Config) == 56
+    assert ctypes.sizeof(gq._Config) == 64
+    assert gq._Config.step_dev.offset == 56
     assert gq._Config.worker0.offset == 44
     assert gq._Config.coord0.offset == 48
     assert gq.gq_validate(cfg(gq, coord0=4096), 1, 10) == gq.GQ_OK
