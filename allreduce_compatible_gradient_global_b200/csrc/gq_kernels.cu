@@ -241,9 +241,11 @@ __global__ void __launch_bounds__(kThreads, 8) norm_kernel(const __grid_constant
 
 int norm_resident_blocks(int kind, bool has_e, bool vec) {
     // resident blocks per SM of the instantiation that will run (cached)
+    // (atomic: calls from several host threads may race on the first query)
     static int cache[2][2][2] = {};
-    int& c = cache[kind != 0][has_e][vec];
-    if (c == 0) {
+    int* c = &cache[kind != 0][has_e][vec];
+    int n = __atomic_load_n(c, __ATOMIC_ACQUIRE);
+    if (n == 0) {
         const void* fn;
         if (kind == 0) {
             fn = has_e ? (vec ? (const void*)norm_kernel<0, true, true> : (const void*)norm_kernel<0, true, false>)
@@ -252,12 +254,11 @@ int norm_resident_blocks(int kind, bool has_e, bool vec) {
             fn = has_e ? (vec ? (const void*)norm_kernel<1, true, true> : (const void*)norm_kernel<1, true, false>)
                        : (vec ? (const void*)norm_kernel<1, false, true> : (const void*)norm_kernel<1, false, false>);
         }
-        int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, 0) != cudaSuccess || n < 1)
             n = 1;
-        c = n;
+        __atomic_store_n(c, n, __ATOMIC_RELEASE);
     }
-    return c;
+    return n;
 }
 
 cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st) {

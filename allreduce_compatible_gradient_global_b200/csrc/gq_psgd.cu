@@ -56,13 +56,10 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Projection pass: pipeline depth and resident blocks per SM by rank.  Each
-// stage takes 16 KiB of shared memory per block; what is left of the 256 KiB
-// L1/shared array keeps Q (4r floats per column group, re-read by every row
-// pair) in L1: 64 KiB at r <= 4, 160 KiB at r >= 5.
+// Projection pass: resident blocks per SM by rank (the register budget the
+// kernels are cut for; the 4r-float Q slice per column group grows with r).
 template <int R>
 struct ProjCfg {
-    static constexpr int stages = (R >= 3 && R <= 4) ? 4 : 3;
     static constexpr int min_blocks = R <= 2 ? 4 : (R <= 4 ? 3 : 2);
 };
 constexpr int kBackStages = 8;  // per-thread pipeline depth of the back projection
@@ -76,15 +73,14 @@ __device__ __forceinline__ float lowrank_value(const float (&p)[R], const float*
 }
 
 // ---------------------------------------------------------------------------
-// project: tiles of (matrix, worker, 16 rows); each warp takes two rows and its
-// lanes stride over the columns (float4 when every m is a multiple of 4).
-// P_w[i,k] sums lane-sequential partials, then a xor butterfly over the warp.
+// project, any m: tiles of (matrix, worker, 16 rows); each warp takes two rows
+// and its lanes stride over the columns one float at a time.  P_w[i,k] sums
+// lane-sequential partials, then a xor butterfly over the warp.  (When every m
+// is a multiple of 4, psgd_project_q_kernel below takes the pass.)
 // ---------------------------------------------------------------------------
-template <int R, bool HAVE_PREV, bool VEC>
+template <int R, bool HAVE_PREV>
 __global__ void __launch_bounds__(kPsgdThreads, ProjCfg<R>::min_blocks)
     psgd_project_kernel(const __grid_constant__ PsgdArgs a) {
-    constexpr int kProjStages = ProjCfg<R>::stages;
-    extern __shared__ float4 psm[];  // VEC: kProjStages x 4 float4 per lane
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (long long t = blockIdx.x; t < a.tile0[a.count]; t += gridDim.x) {
         const int l = matrix_of(a, t);
@@ -112,98 +108,23 @@ __global__ void __launch_bounds__(kPsgdThreads, ProjCfg<R>::min_blocks)
         float acc0[R], acc1[R];
 #pragma unroll
         for (int k = 0; k < R; ++k) acc0[k] = acc1[k] = 0.f;
-        if (VEC) {
-            // lane-private ring of kProjStages slots, each {G row i0, M row i0,
-            // G row i0+1, M row i0+1} for one float4 column group
-            float4* ring = psm + (size_t)warp * kProjStages * 4 * 32;
-            const float4* gA4 = reinterpret_cast<const float4*>(g0);
-            const float4* mA4 = reinterpret_cast<const float4*>(m0);
-            const float4* gB4 = reinterpret_cast<const float4*>(g0 + m);
-            const float4* mB4 = reinterpret_cast<const float4*>(m0 + m);
-            const int m4 = m >> 2;
-            const int nit = lane < m4 ? (m4 - lane + 31) / 32 : 0;
-            auto issue = [&](int it) {
-                const int j4 = lane + it * 32;
-                float4* d = ring + (it % kProjStages) * 128 + lane;
-                cp_async16(d, gA4 + j4);
-                cp_async16(d + 32, mA4 + j4);
-                if (two) {
-                    cp_async16(d + 64, gB4 + j4);
-                    cp_async16(d + 96, mB4 + j4);
-                }
-            };
+        for (int j = lane; j < m; j += 32) {
+            float q[R];
 #pragma unroll
-            for (int it = 0; it < kProjStages - 1; ++it) {
-                if (it < nit) issue(it);
-                cp_async_commit();
+            for (int k = 0; k < R; ++k) q[k] = __ldg(qm + (long long)j * R + k);
+            float eA = m0[j], eB = two ? m0[m + j] : 0.f;
+            if (HAVE_PREV) {
+                eA = __fsub_rn(eA, lowrank_value<R>(p0, q));
+                eB = __fsub_rn(eB, lowrank_value<R>(p1, q));
             }
-            for (int it = 0; it < nit; ++it) {
-                if (it + kProjStages - 1 < nit) issue(it + kProjStages - 1);
-                cp_async_commit();
-                cp_async_wait<kProjStages - 1>();  // this lane's copies of step `it` landed
-                const int j4 = lane + it * 32;
-                float q[4 * R];  // rows 4 j4 .. 4 j4 + 3 of Q, R values each
-                const float4* q4 = reinterpret_cast<const float4*>(qm + (long long)j4 * 4 * R);
+            const float vA = __fadd_rn(g0[j], eA);
+            const float vB = two ? __fadd_rn(g0[m + j], eB) : 0.f;
+            m0[j] = vA;
+            if (two) m0[m + j] = vB;
 #pragma unroll
-                for (int k = 0; k < R; ++k) {
-                    const float4 v = __ldg(q4 + k);
-                    q[4 * k] = v.x;
-                    q[4 * k + 1] = v.y;
-                    q[4 * k + 2] = v.z;
-                    q[4 * k + 3] = v.w;
-                }
-                const float4* d = ring + (it % kProjStages) * 128 + lane;
-                const float4 ga = d[0], ma = d[32];
-                float4 gb = make_float4(0.f, 0.f, 0.f, 0.f), mb = gb;
-                if (two) {
-                    gb = d[64];
-                    mb = d[96];
-                }
-                const float gA[4] = {ga.x, ga.y, ga.z, ga.w}, mA[4] = {ma.x, ma.y, ma.z, ma.w};
-                const float gB[4] = {gb.x, gb.y, gb.z, gb.w}, mB[4] = {mb.x, mb.y, mb.z, mb.w};
-                float outA[4], outB[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float* qc = q + c * R;
-                    float eA = mA[c], eB = mB[c];
-                    if (HAVE_PREV) {
-                        eA = __fsub_rn(eA, lowrank_value<R>(p0, qc));
-                        eB = __fsub_rn(eB, lowrank_value<R>(p1, qc));
-                    }
-                    outA[c] = __fadd_rn(gA[c], eA);
-                    outB[c] = __fadd_rn(gB[c], eB);
-#pragma unroll
-                    for (int k = 0; k < R; ++k) {
-                        acc0[k] = __fmaf_rn(outA[c], qc[k], acc0[k]);
-                        acc1[k] = __fmaf_rn(outB[c], qc[k], acc1[k]);
-                    }
-                }
-                __stcs(reinterpret_cast<float4*>(m0) + j4,
-                       make_float4(outA[0], outA[1], outA[2], outA[3]));
-                if (two)
-                    __stcs(reinterpret_cast<float4*>(m0 + m) + j4,
-                           make_float4(outB[0], outB[1], outB[2], outB[3]));
-            }
-            cp_async_wait<0>();
-        } else {
-            for (int j = lane; j < m; j += 32) {
-                float q[R];
-#pragma unroll
-                for (int k = 0; k < R; ++k) q[k] = __ldg(qm + (long long)j * R + k);
-                float eA = m0[j], eB = two ? m0[m + j] : 0.f;
-                if (HAVE_PREV) {
-                    eA = __fsub_rn(eA, lowrank_value<R>(p0, q));
-                    eB = __fsub_rn(eB, lowrank_value<R>(p1, q));
-                }
-                const float vA = __fadd_rn(g0[j], eA);
-                const float vB = two ? __fadd_rn(g0[m + j], eB) : 0.f;
-                m0[j] = vA;
-                if (two) m0[m + j] = vB;
-#pragma unroll
-                for (int k = 0; k < R; ++k) {
-                    acc0[k] = __fmaf_rn(vA, q[k], acc0[k]);
-                    acc1[k] = __fmaf_rn(vB, q[k], acc1[k]);
-                }
+            for (int k = 0; k < R; ++k) {
+                acc0[k] = __fmaf_rn(vA, q[k], acc0[k]);
+                acc1[k] = __fmaf_rn(vB, q[k], acc1[k]);
             }
         }
 #pragma unroll
@@ -226,9 +147,10 @@ __global__ void __launch_bounds__(kPsgdThreads, ProjCfg<R>::min_blocks)
 }
 
 // ---------------------------------------------------------------------------
-// project, ranks 5..8 (every m a multiple of 4): the same arithmetic and
-// summation order as psgd_project_kernel, but the Q slice of each column step
-// is staged once per block.  All 8 warps of a block walk the same column
+// project, every m a multiple of 4 (any rank): the same arithmetic and
+// summation order as psgd_project_kernel, with columns taken as float4 groups
+// (lane-sequential partials over j4 = lane + 32 it, four columns each) and the
+// Q slice of each column step staged once per block.  All 8 warps of a block walk the same column
 // groups (j4 = lane + 32 it) of their own two rows, so one copy of Q's rows
 // 4 j4 .. 4 j4 + 3 serves the block instead of being re-read by every row
 // pair through L1.  Ring of kQStages slots: per warp the lane-private G / M
@@ -666,17 +588,10 @@ static int resident_grid(const void* fn, size_t smem, long long tiles, int sms) 
 
 #define GQ_PSGD_RANKS(X) X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8)
 
-template <int R, bool HP, bool VEC>
+template <int R, bool HP>
 static cudaError_t project_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
-    auto kern = psgd_project_kernel<R, HP, VEC>;
-    const size_t smem = VEC ? (size_t)ProjCfg<R>::stages * 4 * kPsgdThreads * sizeof(float4) : 0;
-    if (VEC) {
-        static int limits[64] = {};
-        const cudaError_t e = ensure_dynamic_smem((const void*)kern, smem, limits);
-        if (e != cudaSuccess) return e;
-    }
-    kern<<<resident_grid((const void*)kern, smem, a.tile0[a.count], sms), kPsgdThreads, smem,
-           st>>>(a);
+    auto kern = psgd_project_kernel<R, HP>;
+    kern<<<resident_grid((const void*)kern, 0, a.tile0[a.count], sms), kPsgdThreads, 0, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -692,16 +607,10 @@ static cudaError_t project_q_inst(const PsgdArgs& a, int sms, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-#ifndef GQ_PSGD_SHARED_Q
-#define GQ_PSGD_SHARED_Q 1
-#endif
-#ifndef GQ_PSGD_SHARED_Q_MIN_RANK
-#define GQ_PSGD_SHARED_Q_MIN_RANK 1
-#endif
 
 cudaError_t launch_psgd_project(const PsgdArgs& a, bool vec, int sms, cudaStream_t st) {
     const bool hp = a.have_prev != 0;
-    if (GQ_PSGD_SHARED_Q && vec && a.rank >= GQ_PSGD_SHARED_Q_MIN_RANK) {
+    if (vec) {
         switch (a.rank) {
             case 1: return hp ? project_q_inst<1, true>(a, sms, st) : project_q_inst<1, false>(a, sms, st);
             case 2: return hp ? project_q_inst<2, true>(a, sms, st) : project_q_inst<2, false>(a, sms, st);
@@ -713,12 +622,8 @@ cudaError_t launch_psgd_project(const PsgdArgs& a, bool vec, int sms, cudaStream
             default: return hp ? project_q_inst<8, true>(a, sms, st) : project_q_inst<8, false>(a, sms, st);
         }
     }
-#define GQ_PROJ(RR)                                                           \
-    case RR:                                                                  \
-        if (hp) return vec ? project_inst<RR, true, true>(a, sms, st)         \
-                           : project_inst<RR, true, false>(a, sms, st);       \
-        return vec ? project_inst<RR, false, true>(a, sms, st)                \
-                   : project_inst<RR, false, false>(a, sms, st);
+#define GQ_PROJ(RR) \
+    case RR: return hp ? project_inst<RR, true>(a, sms, st) : project_inst<RR, false>(a, sms, st);
     switch (a.rank) {
         GQ_PSGD_RANKS(GQ_PROJ)
         default: return cudaErrorInvalidValue;
