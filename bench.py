@@ -193,20 +193,21 @@ def run_ours(args, rank, world, local_rank):
     buf = gq.StepBuffers(cfg, W, d, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(i, ev=None):
+    def step(i, ev=None, codes=True):
         cfg.step = i
         if ev is not None:
             ev[0].record(stream)
         gq.gq_global_norm(g, buf.e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws, stream)
         if ev is not None:
             ev[1].record(stream)
-        gq.gq_quantize_aggregate(g, buf.e, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws,
-                                 stream)
+        gq.gq_quantize_aggregate(g, buf.e, cfg, buf.scale, buf.codes if codes else None, buf.sum,
+                                 buf.out, buf.ws, stream)
         if ev is not None:
             ev[2].record(stream)
 
     for i in range(args.warmup):
         step(i)
+        step(i, codes=False)  # the instantiation without codes, timed below too
     if gq.gq_get_device_status(buf.ws, stream) != gq.GQ_OK:
         raise RuntimeError("non-finite scale in warm-up")
     K = args.steps
@@ -234,9 +235,19 @@ def run_ours(args, rank, world, local_rank):
     for i in range(K):
         step(args.warmup + K + i, evs[i])
     torch.cuda.synchronize()
+    # The fused pass without materialised codes (the sum-based exchange needs
+    # none): K more steps, events around the run only.
+    n0 = torch.cuda.Event(enable_timing=True)
+    n1 = torch.cuda.Event(enable_timing=True)
+    n0.record(stream)
+    for i in range(K):
+        step(args.warmup + 2 * K + i, codes=False)
+    n1.record(stream)
+    torch.cuda.synchronize()
     sampler.stop()
     if world > 1:
         torch.distributed.barrier()
+    nc_ms = job_time_ms(n0.elapsed_time(n1), world, dev)
     norm_ms = [e[0].elapsed_time(e[1]) for e in evs]
     quant_ms = [e[1].elapsed_time(e[2]) for e in evs]
     ms_per_step = elapsed_ms / K
@@ -263,6 +274,11 @@ def run_ours(args, rank, world, local_rank):
                          "frac": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
                          "frac_of_8000": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / 8000, 4)}}
 
+    p2_nc = p2 - W * gq.gq_packed_row_bytes(cfg, d)
+    without_codes = {"value": round(job_gbs(grad_bytes, K, nc_ms, world), 2), "unit": "GB/s",
+                     "ms_per_step": round(nc_ms / K, 5), "algorithmic_bytes": p1 + p2_nc,
+                     "step_frac": round((p1 + p2_nc) / (nc_ms / K * 1e-3) / 1e9 / peak, 4)}
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(gq, args, cfg, g, buf, stream, world, dev)
@@ -280,7 +296,8 @@ def run_ours(args, rank, world, local_rank):
                       f"vs {L2_BYTES / 1e6:.0f} MB L2"},
         roofline=roofline, gpu_launches=2 * K, clocks=sampler.summary(), e2e=e2e,
         timing="value, ms_per_step: K steps, CUDA events around the whole run only; "
-               "roofline avg_launch_ms: K further steps with CUDA events around each kernel")
+               "roofline avg_launch_ms: K further steps with CUDA events around each kernel",
+        fused_without_codes=without_codes)
     del g, buf
     torch.cuda.empty_cache()
     return result
