@@ -31,6 +31,15 @@ overlaps the all-reduce of chunk k: each chunk is quantized with
 uniforms it would draw in the whole vector, and the result is bit-identical
 to the unchunked exchange.
 
+``capture(g, e)`` records one whole exchange -- kernels, both NCCL
+all-reduces and, when chunked, the overlap between them -- into a CUDA graph,
+and ``replay()`` runs it with one host call per step.  The step then comes from
+a device word (``gq_config.step_dev``) that the graph itself advances, so
+replay k draws exactly the uniforms of step ``first + k``.  The graph is bound
+to the addresses of ``g`` and ``e``: write each step's gradients into ``g`` in
+place.  ``close()`` releases the graph; call it before the process group is
+destroyed.
+
 The library calls are reached through an ``ops`` object (``GpuOps`` by
 default) so that the host-side orchestration can be exercised with other
 backends in tests; the product path always uses ``GpuOps``.
@@ -40,9 +49,9 @@ from dataclasses import replace
 import torch
 import torch.distributed as dist
 
-from . import (GQ_OK, GQConfig, GQError, gq_dequantize_ef, gq_get_device_status,
-               gq_global_norm, gq_quantize_aggregate, gq_validate, gq_workspace_bytes,
-               gq_workspace_init)
+from . import (GQ_OK, GQConfig, GQError, gq_advance_step, gq_dequantize_ef,
+               gq_get_device_status, gq_global_norm, gq_quantize_aggregate, gq_validate,
+               gq_workspace_bytes, gq_workspace_init)
 
 
 class GpuOps:
@@ -100,38 +109,85 @@ class DataParallelStep:
                               device=dev)
         if dev.type == "cuda":
             gq_workspace_init(self.ws)
+        self.graph = None
+        self.step_dev = None
 
-    def __call__(self, g, e=None, step=None, check=False):
-        """g: [w_local][d] fp32 on this rank; e: the rank's error rows (updated in
-        place when cfg.ef).  Returns the mean over all W workers, [d] fp32."""
-        if step is not None:
-            self.cfg.step = int(step)
-        ef = e if self.cfg.ef else None
-        self.ops.global_norm(g, ef, self.cfg, self.scale, self.ws)
+    def _exchange(self, g, e, cfg):
+        ef = e if cfg.ef else None
+        self.ops.global_norm(g, ef, cfg, self.scale, self.ws)
         dist.all_reduce(self.scale, op=dist.ReduceOp.MAX, group=self.group)
         if self.chunks == 1:
-            self.ops.quantize_sum(g, e, self.cfg, self.scale, self.sum, self.ws)
+            self.ops.quantize_sum(g, e, cfg, self.scale, self.sum, self.ws)
             dist.all_reduce(self.sum, op=dist.ReduceOp.SUM, group=self.group)
-            self.ops.decode(self.sum, self.W, self.cfg, self.scale, self.out, self.ws)
+            self.ops.decode(self.sum, self.W, cfg, self.scale, self.out, self.ws)
         else:
             # quantize chunk k + 1 while the all-reduce of chunk k runs on the
             # collective's own stream; decode each chunk once its sum is in
             works = []
             for c0, c1 in self.bounds:
-                cfg_k = replace(self.cfg, coord0=c0)
+                cfg_k = replace(cfg, coord0=c0)
                 self.ops.quantize_sum(g[:, c0:c1], None if e is None else e[:, c0:c1], cfg_k,
                                       self.scale, self.sum[c0:c1], self.ws)
                 works.append(dist.all_reduce(self.sum[c0:c1], op=dist.ReduceOp.SUM,
                                              group=self.group, async_op=True))
             for (c0, c1), work in zip(self.bounds, works):
                 work.wait()
-                self.ops.decode(self.sum[c0:c1], self.W, self.cfg, self.scale,
+                self.ops.decode(self.sum[c0:c1], self.W, cfg, self.scale,
                                 self.out[c0:c1], self.ws)
+
+    def _check(self):
+        rc = self.ops.status(self.ws)
+        if rc != GQ_OK:
+            raise GQError(rc, "DataParallelStep")
+
+    def __call__(self, g, e=None, step=None, check=False):
+        """g: [w_local][d] fp32 on this rank; e: the rank's error rows (updated in
+        place when cfg.ef).  Returns the mean over all W workers, [d] fp32."""
+        if step is not None:
+            self.cfg.step = int(step)
+        self._exchange(g, e, self.cfg)
         if check:
-            rc = self.ops.status(self.ws)
-            if rc != GQ_OK:
-                raise GQError(rc, "DataParallelStep")
+            self._check()
         return self.out
+
+    def capture(self, g, e=None, first_step=0):
+        """Record one exchange on g (and e) into a CUDA graph; replay() runs it.
+        Every rank must capture at the same point, since the graph holds
+        collectives.  An eager warm-up on a copy of e first sets each kernel's
+        launch attributes and opens the NCCL communicator, leaving e as it was."""
+        import torch
+        self.close()
+        self.step_dev = torch.full((1,), int(first_step), dtype=torch.int32,
+                                   device=self.out.device)
+        cfg = replace(self.cfg, step_dev=self.step_dev)
+        e_warm = None if e is None else e.clone()
+        self._exchange(g, e_warm, cfg)
+        torch.cuda.synchronize()
+        self.step_dev.fill_(int(first_step))
+        del e_warm
+        graph = torch.cuda.CUDAGraph()
+        # thread-local: a CUDA call from the collective library's own threads
+        # during the capture does not invalidate it
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            self._exchange(g, e, cfg)
+            gq_advance_step(self.step_dev)
+        self.graph = graph
+
+    def replay(self, step=None, check=False):
+        """Run the captured exchange once (the step advances by one per replay;
+        `step` sets it first).  Returns the mean over all W workers."""
+        if self.graph is None:
+            raise RuntimeError("DataParallelStep.replay: nothing captured")
+        if step is not None:
+            self.step_dev.fill_(int(step))
+        self.graph.replay()
+        if check:
+            self._check()
+        return self.out
+
+    def close(self):
+        """Release the captured graph (before destroying the process group)."""
+        self.graph = None
 
 
 def gather_rows(local, out, group=None):

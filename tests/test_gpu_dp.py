@@ -133,3 +133,46 @@ def test_nccl_chunked_exchange_equals_unchunked(gq, chunks, kw):
                 assert torch.equal(e1, e2), t
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("chunks,w_local,kw", [(1, 4, dict(s=15, bits=5, wire="int8", ef=True)),
+                                               (3, 1, dict(s=15, bits=5, wire="int8", ef=True)),
+                                               (4, 1, dict(levels="exp", L=8, bits=5,
+                                                           wire="f16"))])
+def test_nccl_graph_replay_equals_eager_exchange(gq, chunks, w_local, kw):
+    """The exchange captured once in a CUDA graph (kernels, NCCL all-reduces and,
+    chunked, their overlap) and replayed with new gradients written in place
+    equals the eager exchange step for step, error buffers included; the graph
+    advances the device step word itself."""
+    from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    graphed = None
+    try:
+        d = 100_003
+        cfg = gq.GQConfig(seed=5, **kw)
+        eager = DataParallelStep(cfg, d, w_local=w_local, chunks=chunks)
+        graphed = DataParallelStep(cfg, d, w_local=w_local, chunks=chunks)
+        e1 = torch.zeros((w_local, d), dtype=torch.float32, device="cuda")
+        e2 = torch.zeros_like(e1)
+        g_in = torch.zeros_like(e1)
+        graphed.capture(g_in, e2 if cfg.ef else None, first_step=2)
+        assert torch.count_nonzero(e2) == 0  # the warm-up left the error rows alone
+        for t in range(2, 6):
+            g = synthetic.make_gradients(w_local, d, "student_t3", seed=100 + t, device="cuda",
+                                         seg=1000, lo=-4, hi=0)
+            g_in.copy_(g)
+            got = graphed.replay(check=True).clone()
+            want = eager(g, e1, step=t, check=True).clone()
+            torch.cuda.synchronize()
+            assert torch.equal(got.view(torch.int32), want.view(torch.int32)), t
+            if cfg.ef:
+                assert torch.equal(e1, e2), t
+        assert int(graphed.step_dev.item()) == 6
+    finally:
+        if graphed is not None:
+            graphed.close()
+        dist.destroy_process_group()
+
