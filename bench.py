@@ -375,6 +375,65 @@ def cpu_baseline(args, sample_coords=None):
                       f"({'the full workload' if n == d else 'a prefix'}), {dt:.1f} s"}
 
 
+def oracle_step_threaded(g, threads, *, levels, s, L, scale_kind, bits, seed, step=0):
+    """The oracle's step on `threads` host threads, for the threaded CPU figure.
+    The oracle's scale is per worker (an fp64 sum in ascending coordinate order
+    within a row, or the row's max |v|), so the rows run in parallel and S is
+    the max of their scales.  With S fixed, every code depends only on its own
+    coordinate (the uniforms are counter-based), so coordinate chunks of whole
+    128-coordinate packing blocks are quantized at their own indices, packed,
+    summed and decoded independently.  The oracle's C routines release the GIL
+    while they run.  Returns S, the packed rows, the integer sums and the mean."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    W, d = g.shape
+    per = -(-d // (threads * 4))
+    step_c = max(128, -(-per // 128) * 128)
+    bounds = [(c0, min(d, c0 + step_c)) for c0 in range(0, d, step_c)]
+
+    def row_scale(w):
+        return oracle.global_scale(g[w:w + 1], None, scale_kind)[0]
+
+    with ThreadPoolExecutor(max_workers=threads) as pool:
+        S = np.float32(max(pool.map(row_scale, range(W))))
+
+        def chunk(b):
+            c0, c1 = b
+            codes = oracle.quantize(g[:, c0:c1], None, levels=levels, s=s, L=L, seed=seed,
+                                    step=step, S=S, js=np.arange(c0, c1, dtype=np.int64))
+            packed = oracle.pack(codes, bits) if bits else None
+            total = oracle.aggregate(codes, levels=levels, L=L)
+            return packed, total, oracle.decode_mean(total, W, levels=levels, s=s, L=L, S=S)
+
+        parts = list(pool.map(chunk, bounds))
+    packed = np.concatenate([x[0] for x in parts], axis=1) if bits else None
+    return dict(S=S, packed=packed, sum=np.concatenate([x[1] for x in parts]),
+                out=np.concatenate([x[2] for x in parts]))
+
+
+def cpu_baseline_threads(args):
+    """The same oracle step run coordinate-parallel over every host core the
+    process may use (oracle_step_threaded): a second, fairer CPU figure."""
+    import oracle
+    wl = synthetic.WORKLOADS[args.workload]
+    W, d = wl["W"], wl["d"]
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else \
+        (os.cpu_count() or 1)
+    g = synthetic.workload_gradients(args.workload, device="cpu").numpy()
+    oracle.lib()
+    t = time.perf_counter()
+    oracle_step_threaded(g, threads, levels=0 if wl["levels"] == "uniform" else 1,
+                         s=wl.get("s", 15), L=wl.get("L", 8),
+                         scale_kind=0 if wl["scale"] == "l2" else 1, bits=wl["bits"],
+                         seed=0x5EED)
+    dt = time.perf_counter() - t
+    return {"value": round(4 * W * d / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": f"oracle x{threads} threads",
+            "sample": f"one oracle step on W={W} x {d} coordinates of the {args.workload} "
+                      f"recipe (the full workload), rows then coordinate chunks over "
+                      f"{threads} threads, {dt:.1f} s"}
+
+
 def run_reference(args):
     """Reference arm: the CPU oracle, each step a bounded sample."""
     import oracle
@@ -848,6 +907,8 @@ def main():
         if rank == 0:
             result["cpu_baseline"] = None if (args.no_cpu_baseline or world > 1) \
                 else cpu_baseline(args)
+            result["cpu_baseline_threads"] = None if (args.no_cpu_baseline or world > 1) \
+                else cpu_baseline_threads(args)
             print(json.dumps(result), flush=True)
     finally:
         if world > 1:
