@@ -60,6 +60,11 @@ def lib():
         L.gqo_logq_decode_one.restype = f32
         L.gqo_lowrank_fma.argtypes = [P, P, i64, i64, i32, P]
         L.gqo_lowrank_fma.restype = None
+        L.gqo_nat_quantize_workers.argtypes = [P, i32, i64, u32, u64, u32, P]
+        L.gqo_nat_value.argtypes = [ctypes.c_uint16]
+        L.gqo_nat_value.restype = f32
+        L.gqo_nat_decode.argtypes = [P, i64, P]
+        L.gqo_nat_decode_sum.argtypes = [P, i32, i64, P]
         _lib = L
     return _lib
 
@@ -282,3 +287,37 @@ def logq_map(xn, alpha=10.0):
 
 def logq_decode_one(k, m, alpha=10.0):
     return lib().gqo_logq_decode_one(k, m, alpha)
+
+
+# --------------------------------------------------------- natural compression
+NAT_TAG = 0x4E410000
+
+
+def nat_quantize(x, *, seed=0, step=0, worker0=0):
+    """[NC] natural compression of [W][n] float32: uint16 codes (sign bit << 8 |
+    biased exponent of the signed power of two, or of the signed zero); row w
+    draws its uniforms as worker worker0 + w from the stream tagged NAT_TAG."""
+    x = _f32(x)
+    W, n = x.shape
+    out = np.zeros((W, n), np.uint16)
+    _check(lib().gqo_nat_quantize_workers(_p(x), W, n, int(worker0), seed, step, _p(out)),
+           "nat_quantize")
+    return out
+
+
+def nat_decode(codes):
+    """The float value of every code (same shape)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint16)
+    out = np.zeros(c.shape, np.float32)
+    _check(lib().gqo_nat_decode(_p(c), c.size, _p(out)), "nat_decode")
+    return out
+
+
+def nat_decode_sum(codes):
+    """fp32 sum over workers (rows) in ascending order, from row 0's value."""
+    c = np.ascontiguousarray(codes, dtype=np.uint16)
+    W, n = c.shape
+    out = np.zeros(n, np.float32)
+    _check(lib().gqo_nat_decode_sum(_p(c), W, n, _p(out)), "nat_decode_sum")
+    return out
+

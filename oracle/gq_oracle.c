@@ -535,3 +535,82 @@ void gqo_lowrank_fma(const float* P, const float* Q, int64_t n, int64_t m, int r
             out[i * m + j] = acc;
         }
 }
+
+/* ------------------------------------------------------------------------
+ * [NC] Natural compression (Horvath, Ho, Horvath, Sahu, Canini, Richtarik,
+ * "Natural Compression for Distributed Deep Learning", MSML 2022, cited in
+ * the Global-QSGD record): stochastic rounding of |x| to one of the two
+ * powers of two around it, p = (|x| - 2^e) / 2^e of going up, so the result
+ * is unbiased and its variance (2^(e+1) - |x|)(|x| - 2^e) is at most x^2/8.
+ * Values below the smallest normal float have no exponent of their own: they
+ * round between 0 and 2^-126, with p = |x| / 2^-126.  The result keeps the
+ * sign of x, a zero result included.
+ * ---------------------------------------------------------------------- */
+static float nat_round(float x, uint32_t f)
+{
+    float ax = fabsf(x);
+    float lower, upper, p;
+    if (ax < 0x1p-126f) {
+        lower = 0.0f;
+        upper = 0x1p-126f;
+        p = ldexpf(ax, 126); /* exact: a subnormal has at most 23 significant bits */
+    } else {
+        int e2;
+        (void)frexpf(ax, &e2); /* ax = m * 2^e2 with m in [0.5, 1) */
+        lower = ldexpf(1.0f, e2 - 1);
+        upper = ldexpf(1.0f, e2); /* 2^128 overflows to infinity */
+        p = ax / lower - 1.0f;    /* exact: in [0, 1) with at most 23 fraction bits */
+    }
+    float mag = round_up(p, f) ? upper : lower;
+    return sign_negative(x) ? -mag : mag;
+}
+
+/* Sign and biased exponent of a signed power of two, zero or infinity: by
+ * definition the top nine bits of its IEEE-754 binary32 pattern. */
+static uint16_t nat_code_of(float v)
+{
+    uint32_t bits;
+    memcpy(&bits, &v, sizeof bits);
+    return (uint16_t)(bits >> 23);
+}
+
+int gqo_nat_quantize_workers(const float* x, int W, int64_t n, uint32_t worker0,
+                             uint64_t seed, uint32_t step, uint16_t* codes_out)
+{
+    if (!x || !codes_out || W < 1 || n < 0) return -1;
+    for (int w = 0; w < W; ++w) {
+        for (int64_t i = 0; i < n; ++i) {
+            int64_t at = (int64_t)w * n + i;
+            uint32_t f = gqo_uniform_bits(seed, GQO_NAT_TAG, step, worker0 + (uint32_t)w,
+                                          (uint64_t)i);
+            codes_out[at] = nat_code_of(nat_round(x[at], f));
+        }
+    }
+    return 0;
+}
+
+float gqo_nat_value(uint16_t code)
+{
+    int E = code & 0xFF;
+    float mag = E == 0 ? 0.0f : (E == 255 ? INFINITY : ldexpf(1.0f, E - 127));
+    return (code & 0x100) ? -mag : mag;
+}
+
+int gqo_nat_decode(const uint16_t* codes, int64_t n, float* out)
+{
+    if (!codes || !out || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) out[i] = gqo_nat_value(codes[i]);
+    return 0;
+}
+
+int gqo_nat_decode_sum(const uint16_t* codes, int W, int64_t n, float* out)
+{
+    if (!codes || !out || W < 1 || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        float acc = gqo_nat_value(codes[i]);
+        for (int w = 1; w < W; ++w) acc = acc + gqo_nat_value(codes[(int64_t)w * n + i]);
+        out[i] = acc;
+    }
+    return 0;
+}
+

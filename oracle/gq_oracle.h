@@ -25,6 +25,11 @@
  *        E_t = G'_t - Ghat_t), and referee major comment 1 on Section IV-A,
  *        Eqs. (5)-(6) (normalise by the maximum magnitude; Eq. (6) inverts
  *        the map).
+ *  [NC]  "Global-QSGD: Allreduce-Compatible Quantization for Distributed
+ *        Learning with Theoretical Guarantees" (crossref record) -- its
+ *        reference list cites Horvath et al., "Natural Compression for
+ *        Distributed Deep Learning" (MSML 2022); the compressor is restated
+ *        from that published method (power-of-two stochastic rounding).
  *
  * Where the pages leave a step open, the reading taken is stated at the
  * function.  Floating-point steps are fp32 in a fixed order with no FMA
@@ -153,6 +158,24 @@ int gqo_logq_decode_sum(const int8_t* codes, const float* maxabs, int W,
 /* Single-entry forms of the log map, for the property tests. */
 float gqo_logq_map(float xn, float alpha);           /* log1p(a*xn)/log1p(a) */
 float gqo_logq_decode_one(int32_t k, float m, float alpha);
+
+/* [NC] natural compression: a nonzero x with 2^e <= |x| < 2^(e+1) becomes
+ * sign(x) 2^e or sign(x) 2^(e+1), the upper one with probability
+ * |x|/2^e - 1 (unbiased); zero stays a signed zero; below 2^-126 the bracket
+ * is [0, 2^-126].  The uniforms come from the stream tagged GQO_NAT_TAG with
+ * row w drawing as worker worker0 + w.  codes_out[w][i] = sign bit << 8 |
+ * biased fp32 exponent of the result (0 for a zero).  Returns 0 or -1. */
+#define GQO_NAT_TAG 0x4E410000u
+int gqo_nat_quantize_workers(const float* x, int W, int64_t n, uint32_t worker0,
+                             uint64_t seed, uint32_t step, uint16_t* codes_out);
+
+/* The value of one code, and of n codes. */
+float gqo_nat_value(uint16_t code);
+int gqo_nat_decode(const uint16_t* codes, int64_t n, float* out);
+
+/* fp32 sum over workers in ascending order, starting from worker 0's value:
+ * out[i] = fl(...fl(value(c[0][i]) + value(c[1][i])) ... + value(c[W-1][i])). */
+int gqo_nat_decode_sum(const uint16_t* codes, int W, int64_t n, float* out);
 
 /* The low-rank value P Q^T of one n x m matrix in float32 as the library
  * states it: out[i*m + j] = acc_r with acc_0 = 0 and
