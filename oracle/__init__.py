@@ -60,7 +60,7 @@ def lib():
         L.gqo_logq_decode_one.restype = f32
         L.gqo_lowrank_fma.argtypes = [P, P, i64, i64, i32, P]
         L.gqo_lowrank_fma.restype = None
-        L.gqo_nat_quantize_workers.argtypes = [P, i32, i64, u32, u64, u32, P]
+        L.gqo_nat_quantize_workers.argtypes = [P, i32, i64, P, u32, u64, u32, P]
         L.gqo_nat_value.argtypes = [ctypes.c_uint16]
         L.gqo_nat_value.restype = f32
         L.gqo_nat_decode.argtypes = [P, i64, P]
@@ -293,15 +293,17 @@ def logq_decode_one(k, m, alpha=10.0):
 NAT_TAG = 0x4E410000
 
 
-def nat_quantize(x, *, seed=0, step=0, worker0=0):
+def nat_quantize(x, *, seed=0, step=0, worker0=0, js=None):
     """[NC] natural compression of [W][n] float32: uint16 codes (sign bit << 8 |
     biased exponent of the signed power of two, or of the signed zero); row w
-    draws its uniforms as worker worker0 + w from the stream tagged NAT_TAG."""
+    draws its uniforms as worker worker0 + w from the stream tagged NAT_TAG, and
+    column i as coordinate js[i] (default i)."""
     x = _f32(x)
     W, n = x.shape
+    jsa = None if js is None else np.ascontiguousarray(js, dtype=np.int64)
     out = np.zeros((W, n), np.uint16)
-    _check(lib().gqo_nat_quantize_workers(_p(x), W, n, int(worker0), seed, step, _p(out)),
-           "nat_quantize")
+    _check(lib().gqo_nat_quantize_workers(_p(x), W, n, _p(jsa), int(worker0), seed, step,
+                                          _p(out)), "nat_quantize")
     return out
 
 

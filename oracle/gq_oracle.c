@@ -574,15 +574,16 @@ static uint16_t nat_code_of(float v)
     return (uint16_t)(bits >> 23);
 }
 
-int gqo_nat_quantize_workers(const float* x, int W, int64_t n, uint32_t worker0,
-                             uint64_t seed, uint32_t step, uint16_t* codes_out)
+int gqo_nat_quantize_workers(const float* x, int W, int64_t n, const int64_t* js,
+                             uint32_t worker0, uint64_t seed, uint32_t step,
+                             uint16_t* codes_out)
 {
     if (!x || !codes_out || W < 1 || n < 0) return -1;
     for (int w = 0; w < W; ++w) {
         for (int64_t i = 0; i < n; ++i) {
             int64_t at = (int64_t)w * n + i;
-            uint32_t f = gqo_uniform_bits(seed, GQO_NAT_TAG, step, worker0 + (uint32_t)w,
-                                          (uint64_t)i);
+            uint64_t j = js ? (uint64_t)js[i] : (uint64_t)i;
+            uint32_t f = gqo_uniform_bits(seed, GQO_NAT_TAG, step, worker0 + (uint32_t)w, j);
             codes_out[at] = nat_code_of(nat_round(x[at], f));
         }
     }

@@ -163,11 +163,13 @@ float gqo_logq_decode_one(int32_t k, float m, float alpha);
  * sign(x) 2^e or sign(x) 2^(e+1), the upper one with probability
  * |x|/2^e - 1 (unbiased); zero stays a signed zero; below 2^-126 the bracket
  * is [0, 2^-126].  The uniforms come from the stream tagged GQO_NAT_TAG with
- * row w drawing as worker worker0 + w.  codes_out[w][i] = sign bit << 8 |
- * biased fp32 exponent of the result (0 for a zero).  Returns 0 or -1. */
+ * row w drawing as worker worker0 + w, column i as coordinate js[i] (js may be
+ * NULL: coordinate i).  codes_out[w][i] = sign bit << 8 | biased fp32 exponent
+ * of the result (0 for a zero).  Returns 0 or -1. */
 #define GQO_NAT_TAG 0x4E410000u
-int gqo_nat_quantize_workers(const float* x, int W, int64_t n, uint32_t worker0,
-                             uint64_t seed, uint32_t step, uint16_t* codes_out);
+int gqo_nat_quantize_workers(const float* x, int W, int64_t n, const int64_t* js,
+                             uint32_t worker0, uint64_t seed, uint32_t step,
+                             uint16_t* codes_out);
 
 /* The value of one code, and of n codes. */
 float gqo_nat_value(uint16_t code);

@@ -129,3 +129,12 @@ def test_worker_offset_selects_the_rows_stream(oracle):
     full = oracle.nat_quantize(x, seed=3, step=4)
     part = oracle.nat_quantize(x[2:4], seed=3, step=4, worker0=2)
     assert np.array_equal(full[2:4], part)
+
+
+def test_coordinate_list_selects_the_columns_stream(oracle):
+    x = np.random.default_rng(2).standard_normal((3, 400)).astype(np.float32)
+    full = oracle.nat_quantize(x, seed=6, step=1)
+    js = np.array([0, 5, 7, 128, 399], np.int64)
+    part = oracle.nat_quantize(x[:, js], seed=6, step=1, js=js)
+    assert np.array_equal(full[:, js], part)
+
