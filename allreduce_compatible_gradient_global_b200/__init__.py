@@ -27,11 +27,11 @@ GQ_ERR_NONFINITE = -5
 GQ_ERR_SIZE = -6
 GQ_ERR_TIMEOUT = -7
 
-UNIFORM, EXP, LOG = 0, 1, 2
+UNIFORM, EXP, LOG, NAT = 0, 1, 2, 3
 SCALE_L2, SCALE_MAXABS = 0, 1
 WIRE_INT8, WIRE_INT16, WIRE_F16 = 1, 2, 3
 
-_LEVELS = {"uniform": UNIFORM, "exp": EXP, "log": LOG}
+_LEVELS = {"uniform": UNIFORM, "exp": EXP, "log": LOG, "nat": NAT}
 _SCALES = {"l2": SCALE_L2, "maxabs": SCALE_MAXABS}
 _WIRES = {"int8": WIRE_INT8, "int16": WIRE_INT16, "f16": WIRE_F16}
 
@@ -125,6 +125,8 @@ def _load():
         "gq_lqsgd_step": ([P, P, I, I, P, P, I, I, CP, P, P, P, P, P], I),
         "gq_logq_quantize": ([P, I, I, P, P, CP, P, P, P, P], I),
         "gq_logq_decode_sum": ([P, P, I, I, P, P, CP, P, P], I),
+        "gq_nat_quantize": ([P, I, LL, CP, P, P, P], I),
+        "gq_nat_decode_sum": ([P, I, LL, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -369,6 +371,28 @@ def gq_logq_decode_sum(codes, maxabs, rows, cols, cfg: GQConfig, out, stream=Non
     _check(lib().gq_logq_decode_sum(_ptr(codes), _ptr(maxabs), W, len(rows), r, cc,
                                    ctypes.byref(c), _ptr(out), _stream(stream)),
            "gq_logq_decode_sum")
+
+
+# ------------------------------------------------------------------ natural compression
+def gq_nat_quantize(x, cfg: GQConfig, codes, ws, stream=None):
+    """x [W][n] fp32 -> codes [W][n] int16 (sign << 8 | exponent of the signed power
+    of two); cfg.levels == "nat" (seed, step / step_dev and worker0 are used)."""
+    W, n = _wd(x)
+    _need(x, torch.float32, (W, n), "x")
+    _need(codes, torch.int16, (W, n), "codes")
+    c = cfg.c()
+    _check(lib().gq_nat_quantize(_ptr(x), W, n, ctypes.byref(c), _ptr(codes), _ptr(ws),
+                                 _stream(stream)), "gq_nat_quantize")
+
+
+def gq_nat_decode_sum(codes, out, stream=None):
+    """codes [W][n] int16 -> out [n] fp32, the values summed over workers in
+    ascending order."""
+    W, n = _wd(codes)
+    _need(codes, torch.int16, (W, n), "codes")
+    _need(out, torch.float32, (n,), "out")
+    _check(lib().gq_nat_decode_sum(_ptr(codes), W, n, _ptr(out), _stream(stream)),
+           "gq_nat_decode_sum")
 
 
 # ------------------------------------------------------------------ per-bucket scales

@@ -13,6 +13,7 @@
 #include "gq_api.h"
 #include "gq_internal.h"
 #include "gq_psgd.h"
+#include "gq_nat.h"
 
 using namespace gq;
 
@@ -498,6 +499,48 @@ static void logq_group(LogqArgs& a, int m0, int count, const int* rows, const in
     for (int m = 0; m < m0; ++m) off += (long long)rows[m] * cols[m];
     a.off[0] = off;
     for (int i = 0; i < count; ++i) a.off[i + 1] = a.off[i] + (long long)rows[m0 + i] * cols[m0 + i];
+}
+
+GQ_API int gq_nat_quantize(const float* x_dev, int W, long long n, const gq_config* cfg,
+                           unsigned short* codes_dev, void* ws_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_nat_quantize");
+    if (!cfg || cfg->levels != GQ_NAT || !ws_dev || W > 65535) return GQ_ERR_ARG;
+    int rc = check_sizes(W, n);
+    if (rc) return rc;
+    if (n > 0 && (!x_dev || !codes_dev)) return GQ_ERR_ARG;
+    if (!aligned16(x_dev) || !aligned16(codes_dev) || !aligned16(ws_dev) ||
+        (cfg->step_dev && !aligned4(cfg->step_dev)))
+        return GQ_ERR_ALIGN;
+    if (n == 0) return GQ_OK;
+    NatArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.x = x_dev;
+    a.codes = codes_dev;
+    a.n = n;
+    a.W = W;
+    a.worker0 = cfg->worker0;
+    a.step = cfg->step;
+    a.step_dev = cfg->step_dev;
+    round_keys(cfg->seed, kNatTag, a.rk);
+    a.hdr = header_of(ws_dev);
+    return cuda_status(launch_nat_quantize(a, (n % 4) == 0, sm_count(), stream));
+}
+
+GQ_API int gq_nat_decode_sum(const unsigned short* codes_dev, int W, long long n,
+                             float* out_dev, cudaStream_t stream) {
+    const NvtxRange nvtx_range("gq_nat_decode_sum");
+    int rc = check_sizes(W, n);
+    if (rc) return rc;
+    if (n > 0 && (!codes_dev || !out_dev)) return GQ_ERR_ARG;
+    if (!aligned16(codes_dev) || !aligned16(out_dev)) return GQ_ERR_ALIGN;
+    if (n == 0) return GQ_OK;
+    NatArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.ccodes = codes_dev;
+    a.out = out_dev;
+    a.n = n;
+    a.W = W;
+    return cuda_status(launch_nat_decode_sum(a, (n % 4) == 0, sm_count(), stream));
 }
 
 GQ_API int gq_logq_quantize(const float* x_dev, int W, int nmats, const int* rows_host,

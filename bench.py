@@ -780,6 +780,75 @@ def run_dp(args, rank, world, local_rank):
             "bytes_on_wire_per_rank": {"compressed": d + 4, "fp32": 4 * d}}
 
 
+def run_nat(args):
+    """Natural compression on the bench workload (W = 8 x 25,557,032): per step
+    gq_nat_quantize of every worker's row and gq_nat_decode_sum of the codes
+    over workers (the gather-style exchange done on one GPU).  value and
+    ms_per_step from K steps with events around the run only; per-kernel
+    launch times from K further steps with events around each kernel."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    wl = synthetic.WORKLOADS[args.workload]
+    W, d = wl["W"], (args.coords or wl["d"])
+    x = synthetic.workload_gradients(args.workload, device="cuda", d=d)
+    codes = torch.empty((W, d), dtype=torch.int16, device="cuda")
+    out = torch.empty(d, dtype=torch.float32, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    gq.gq_workspace_init(ws)
+    cfg = gq.GQConfig(levels="nat", seed=0x5EED)
+    K = args.steps
+
+    def step(i, ev=None):
+        cfg.step = i
+        if ev is not None:
+            ev[0].record(stream)
+        gq.gq_nat_quantize(x, cfg, codes, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        gq.gq_nat_decode_sum(codes, out, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(args.warmup + i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(K):
+        step(args.warmup + K + i, evs[i])
+    torch.cuda.synchronize()
+    sampler.stop()
+    if gq.gq_get_device_status(ws, stream) != gq.GQ_OK:
+        raise RuntimeError("non-finite input in the natural-compression run")
+    ms = t0.elapsed_time(t1) / K
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    s_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    peak, peak_kind = measured_hbm_peak()
+    qb = 4 * W * d + 2 * W * d      # read x, write int16 codes
+    sb = 2 * W * d + 4 * d          # read the codes, write the fp32 sum
+    return {"metric": "natural compression: quantize + decode-sum, fp32 gradient GB/s",
+            "mode": "nat", "unit": "GB/s", "workload": args.workload, "W": W, "d": d,
+            "value": round(4 * W * d * 1e-9 / (ms * 1e-3), 2), "ms_per_step": round(ms, 5),
+            "steps": K, "warmup": args.warmup,
+            "quantize": {"avg_launch_ms": round(q_ms, 5), "algorithmic_bytes": qb,
+                         "achieved_gbs": round(qb / (q_ms * 1e-3) / 1e9, 1),
+                         "frac": round(qb / (q_ms * 1e-3) / 1e9 / peak, 4)},
+            "decode_sum": {"avg_launch_ms": round(s_ms, 5), "algorithmic_bytes": sb,
+                           "achieved_gbs": round(sb / (s_ms * 1e-3) / 1e9, 1),
+                           "frac": round(sb / (s_ms * 1e-3) / 1e9 / peak, 4)},
+            "peak": peak, "peak_source": f"{peak_kind} (hbm_gbs)",
+            "wire_bytes_per_worker_coordinate": 2, "clocks": sampler.summary()}
+
+
 def run_lq(args):
     """The LQ-SGD log quantizer: quantize + decode-sum of 24 factor pairs of
     4096 x r per worker, W = 8, r in {1, 4, 7}."""
@@ -846,6 +915,8 @@ def main():
                          "of the same recipe, for profiling; not a bench line)")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line with the d = 2^16..2^30 sweep instead of the bench line")
+    ap.add_argument("--nat", action="store_true",
+                    help="one JSON line timing natural compression (quantize + decode-sum)")
     ap.add_argument("--lq", action="store_true",
                     help="one JSON line with the LQ-SGD log-quantizer timings")
     ap.add_argument("--buckets", action="store_true",
@@ -874,10 +945,10 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
-    if args.sweep or args.lq or args.buckets or args.lqsgd:
+    if args.sweep or args.lq or args.buckets or args.lqsgd or args.nat:
         if rank == 0:
             fn = (run_sweep if args.sweep else run_lq if args.lq else
-                  run_buckets if args.buckets else run_lqsgd)
+                  run_buckets if args.buckets else run_nat if args.nat else run_lqsgd)
             print(json.dumps(fn(args)), flush=True)
         return
 

@@ -78,6 +78,7 @@ extern "C" {
 #define GQ_UNIFORM 0 /* {0, 1/s, ..., 1}: QSGD levels */
 #define GQ_EXP 1     /* {0, 2^-(L-1), ..., 1/2, 1}: NUQSGD-style levels */
 #define GQ_LOG 2     /* LQ-SGD log map, 8-bit codes (gq_logq_* only) */
+#define GQ_NAT 3     /* natural compression, sign + exponent codes (gq_nat_* only) */
 
 /* Scale kinds. */
 #define GQ_SCALE_L2 0     /* S = max_w ||v_w||_2 */
@@ -401,6 +402,41 @@ GQ_API int gq_lqsgd_step(const float* g_dev, float* m_dev, int W, int nmats,
                          const int* rows_host, const int* cols_host, int rank, int have_prev,
                          const gq_config* cfg, float* p_dev, float* q_dev, float* ghat_dev,
                          void* ws_dev, cudaStream_t stream);
+
+/* Natural compression: Horvath et al., "Natural Compression for Distributed
+ * Deep Learning" (MSML 2022), cited in the reference list of "Global-QSGD:
+ * Allreduce-Compatible Quantization for Distributed Learning with Theoretical
+ * Guarantees" (crossref record).  A gather-style compressor, not an
+ * allreduce-compatible one: its values span the whole fp32 exponent range, so
+ * they cannot be summed as fixed-width integers (the bounded form of the same
+ * rounding, with a zero level, is GQ_EXP).
+ *
+ * Each x_dev[w][i] (finite, |x| < 2^127) with 2^e <= |x| < 2^(e+1) becomes
+ * sign(x) 2^e or sign(x) 2^(e+1), the upper one exactly when m + f >= 2^23,
+ * where m is the 23-bit mantissa field of x and f the top 23 bits of a Philox
+ * word: probability |x|/2^e - 1, so the result is unbiased.  Zero stays a
+ * zero; a subnormal rounds between 0 and 2^-126 the same way.  The result
+ * keeps the sign of x (a zero result too).  codes_dev[w][i] is the top nine
+ * bits of the result's binary32 pattern: sign << 8 | biased exponent.
+ * Uniforms: Philox-4x32-10 keyed (lo32 seed, hi32 seed ^ 0x4E410000), counter
+ * (lo32(i>>2), step, worker0 + w, hi32(i>>2)), word i & 3 (step from
+ * cfg->step_dev when that is not NULL).  cfg->levels must be GQ_NAT; the
+ * other fields but seed, step, step_dev and worker0 are ignored.
+ * x_dev [W][n] fp32 and codes_dev [W][n] uint16, 16-byte aligned; n >= 0,
+ * 1 <= W <= 65535 (one grid row per worker).
+ * An infinite or NaN input, or a rounding that overflows to infinity, sets the
+ * NONFINITE flag of the workspace (gq_get_device_status); its code is then
+ * exponent 255.  ws_dev: any workspace of at least 256 bytes zero-filled
+ * once with gq_workspace_init (only its status word is used). */
+GQ_API int gq_nat_quantize(const float* x_dev, int W, long long n, const gq_config* cfg,
+                           unsigned short* codes_dev, void* ws_dev, cudaStream_t stream);
+
+/* Decode and sum over workers: out_dev[i] = fl(...fl(v_0 + v_1) ... + v_{W-1})
+ * with v_w the float whose top nine bits are codes_dev[w][i] (the rest zero),
+ * summed in ascending worker order in fp32.  codes_dev [W][n] uint16 and
+ * out_dev [n] fp32, 16-byte aligned. */
+GQ_API int gq_nat_decode_sum(const unsigned short* codes_dev, int W, long long n,
+                             float* out_dev, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

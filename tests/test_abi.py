@@ -225,3 +225,34 @@ def test_workspace_and_config_layout(gq):
     assert gq._Config.coord0.offset == 48
     assert gq.gq_validate(cfg(gq, coord0=4096), 1, 10) == gq.GQ_OK
     assert gq.gq_validate(cfg(gq, coord0=6), 1, 10) == gq.GQ_ERR_ARG
+
+
+def test_natural_compression_argument_checks(gq):
+    """Checked on the host before any launch (nothing here reaches a GPU)."""
+    lib = gq.lib()
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    cnat = cfg(gq, levels="nat", seed=3).c()
+    cuni = cfg(gq).c()
+    assert lib.gq_nat_quantize(good, 4, 100, ctypes.byref(cuni), good, good, None) == \
+        gq.GQ_ERR_ARG                                   # levels must be GQ_NAT
+    assert lib.gq_nat_quantize(good, 0, 100, ctypes.byref(cnat), good, good, None) == \
+        gq.GQ_ERR_ARG                                   # no workers
+    assert lib.gq_nat_quantize(good, 4, -1, ctypes.byref(cnat), good, good, None) == \
+        gq.GQ_ERR_ARG
+    assert lib.gq_nat_quantize(good, 65536, 4, ctypes.byref(cnat), good, good, None) == \
+        gq.GQ_ERR_ARG                                   # one grid row per worker
+    assert lib.gq_nat_quantize(good, 4, 100, ctypes.byref(cnat), good, None, None) == \
+        gq.GQ_ERR_ARG                                   # no workspace
+    assert lib.gq_nat_quantize(odd, 4, 100, ctypes.byref(cnat), good, good, None) == \
+        gq.GQ_ERR_ALIGN
+    assert lib.gq_nat_quantize(good, 4, 100, ctypes.byref(cnat), odd, good, None) == \
+        gq.GQ_ERR_ALIGN
+    assert lib.gq_nat_quantize(None, 4, 0, ctypes.byref(cnat), None, good, None) == gq.GQ_OK
+    assert lib.gq_nat_decode_sum(good, 0, 100, good, None) == gq.GQ_ERR_ARG
+    assert lib.gq_nat_decode_sum(None, 4, 100, good, None) == gq.GQ_ERR_ARG
+    assert lib.gq_nat_decode_sum(good, 4, 100, odd, None) == gq.GQ_ERR_ALIGN
+    assert lib.gq_nat_decode_sum(None, 4, 0, None, None) == gq.GQ_OK
+    # the main path does not take the natural-compression level
+    assert gq.gq_validate(gq.GQConfig(levels="nat"), 4, 100) == gq.GQ_ERR_ARG
+
