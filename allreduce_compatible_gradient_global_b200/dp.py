@@ -274,3 +274,49 @@ class DataParallelLqsgdStep:
             if rc != GQ_OK:
                 raise GQError(rc, "DataParallelLqsgdStep")
         return ghat
+
+
+class DataParallelNatStep:
+    """Natural compression (Horvath et al., "Natural Compression for Distributed
+    Deep Learning", cited in the Global-QSGD record) across ranks: each rank
+    rounds its own W_local rows to signed powers of two (gq_nat_quantize, workers
+    rank * W_local + w), the 16-bit codes are all-gathered (as bytes, rank-major),
+    and every rank decodes and sums all W workers in ascending order
+    (gq_nat_decode_sum), so the sum is the same on every rank and equals the
+    single-GPU one.  Powers of two over the whole exponent range cannot be summed
+    as fixed-width integers, so this exchange gathers instead of all-reducing:
+    (N - 1) * 2n bytes in per rank, against 2 (N - 1)/N * 4n for a ring fp32
+    all-reduce."""
+
+    def __init__(self, n, w_local=1, seed=0, group=None, device=None):
+        from . import gq_workspace_init as _init
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.n = int(n)
+        self.w_local = int(w_local)
+        self.W = self.world * self.w_local
+        self.seed = int(seed)
+        dev = torch.device(device) if device is not None else torch.device("cuda")
+        self.codes_l = torch.empty((self.w_local, self.n), dtype=torch.int16, device=dev)
+        self.codes = torch.empty((self.W, self.n), dtype=torch.int16, device=dev)
+        self.out = torch.empty(self.n, dtype=torch.float32, device=dev)
+        self.ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+        if dev.type == "cuda":
+            _init(self.ws)
+
+    def __call__(self, x, step, check=False):
+        """x: this rank's [w_local][n] fp32 rows.  Returns the sum over all W
+        workers' compressed rows, [n] fp32 (divide by W for the mean)."""
+        from . import gq_nat_decode_sum, gq_nat_quantize
+        cfg = GQConfig(levels="nat", seed=self.seed, step=int(step),
+                       worker0=self.rank * self.w_local)
+        gq_nat_quantize(x, cfg, self.codes_l, self.ws)
+        gather_rows(self.codes_l.view(torch.uint8), self.codes.view(torch.uint8), self.group)
+        gq_nat_decode_sum(self.codes, self.out)
+        if check:
+            rc = gq_get_device_status(self.ws)
+            if rc != GQ_OK:
+                raise GQError(rc, "DataParallelNatStep")
+        return self.out
+

@@ -206,3 +206,39 @@ def test_gathered_log_codes_decode_like_one_process(oracle, tmp_path):
     for r in range(world):
         got = np.load(tmp_path / f"lq{r}.npy")
         assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), r
+
+
+def _nat_main(rank, world, port, outdir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from allreduce_compatible_gradient_global_b200.dp import gather_rows
+        w_local, n = 2, 301
+        W = world * w_local
+        x = synthetic.make_gradients(W, n, "student_t3", seed=6, seg=50, lo=-20, hi=3).numpy()
+        rows = slice(rank * w_local, (rank + 1) * w_local)
+        mine = oracle.nat_quantize(x[rows], seed=4, step=9, worker0=rank * w_local)
+        codes = torch.empty((W, n), dtype=torch.int16)
+        # the 16-bit codes travel as bytes (gloo reduces no 16-bit integers)
+        gather_rows(torch.from_numpy(mine.view(np.int16)).view(torch.uint8),
+                    codes.view(torch.uint8))
+        total = oracle.nat_decode_sum(codes.numpy().view(np.uint16))
+        np.save(os.path.join(outdir, f"nat{rank}.npy"), total)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gathered_natural_codes_sum_like_one_process(oracle, tmp_path):
+    """Each rank compresses its own workers (worker offset rank * W_local), the
+    codes are all-gathered as bytes, rank-major, and every rank's decoded sum
+    equals the single-process sum of all workers, bit for bit."""
+    world = 2
+    mp.start_processes(_nat_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    x = synthetic.make_gradients(4, 301, "student_t3", seed=6, seg=50, lo=-20, hi=3).numpy()
+    ref = oracle.nat_decode_sum(oracle.nat_quantize(x, seed=4, step=9))
+    for r in range(world):
+        got = np.load(tmp_path / f"nat{r}.npy")
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), r
+
