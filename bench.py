@@ -465,27 +465,39 @@ def run_reference(args):
 
 
 def time_step_pair(gq, g, e, cfg, buf, K, warmup, stream):
-    """Median per-kernel and mean step times (ms) of norm + fused pass."""
-    for i in range(warmup):
+    """Median per-kernel times and the mean step time (ms) of norm + fused pass.
+    The step time comes from K steps with events around the run only; the
+    per-kernel medians from K further steps with an event around each kernel."""
+    def step(i, ev=None):
         cfg.step = i
+        if ev is not None:
+            ev[0].record(stream)
         gq.gq_global_norm(g, e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
         gq.gq_quantize_aggregate(g, e, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(warmup + i)
+    t1.record(stream)
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     for i in range(K):
-        cfg.step = warmup + i
-        evs[i][0].record(stream)
-        gq.gq_global_norm(g, e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws, stream)
-        evs[i][1].record(stream)
-        gq.gq_quantize_aggregate(g, e, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws, stream)
-        evs[i][2].record(stream)
+        step(warmup + K + i, evs[i])
     torch.cuda.synchronize()
     if gq.gq_get_device_status(buf.ws, stream) != gq.GQ_OK:
         raise RuntimeError("device flag raised during the sweep")
     n = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
     q = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
-    step = sum(e[0].elapsed_time(e[2]) for e in evs) / K
-    return n, q, step
+    return n, q, t0.elapsed_time(t1) / K
 
 
 def time_step_graph(gq, g, cfg, W, d, K):
