@@ -15,7 +15,8 @@
 // between 0 and 2^-126 by the same carry.
 //
 // nat_quantize_kernel: one grid row per worker, one thread per group of four
-// coordinates (kNatUnroll groups in flight per thread on vector rows); the
+// coordinates (on vector rows, kNatStages - 1 groups in flight per thread
+// through a cp.async ring in shared memory); the
 // group's Philox block serves its four coordinates (word k for coordinate
 // 4q + k).  nat_decode_sum_kernel: one thread per group of four coordinates,
 // fp32 sum over workers in ascending order.  Both stream HBM: 4 B read + 2 B
@@ -39,8 +40,26 @@ __device__ __forceinline__ uint32_t nat_code(float x, uint32_t word, bool& bad) 
 
 __device__ __forceinline__ float nat_value(uint32_t code) { return __uint_as_float(code << 23); }
 
-// Groups of four coordinates a thread has in flight at once (vector rows).
-constexpr int kNatUnroll = 4;
+// Vector rows: every thread streams its groups through a private ring of
+// kNatStages 16-byte slots in shared memory, filled by cp.async, so that
+// kNatStages - 1 loads stay in flight while Philox runs on the current group,
+// without holding registers for them.  A thread reads back only its own slots
+// after its own cp.async.wait_group, so no block barrier is needed.
+constexpr int kNatStages = 8;
+
+__device__ __forceinline__ void nat_cp_async16(void* smem_dst, const void* gmem_src) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+
+__device__ __forceinline__ void nat_cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void nat_cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) nat_quantize_kernel(const __grid_constant__ NatArgs a) {
@@ -53,29 +72,29 @@ __global__ void __launch_bounds__(kThreads) nat_quantize_kernel(const __grid_con
     unsigned short* cr = a.codes + (long long)w * a.n;
     bool bad = false;
     if (VEC) {  // n % 4 == 0: every group is whole and 16-byte aligned
-        for (long long q0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; q0 < nq;
-             q0 += kNatUnroll * stride) {
-            float4 v[kNatUnroll];
+        __shared__ float4 ring[kNatStages][kThreads];
+        const long long q0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+        const long long nit = q0 < nq ? (nq - q0 + stride - 1) / stride : 0;
+        const float4* x4 = reinterpret_cast<const float4*>(xr);
 #pragma unroll
-            for (int k = 0; k < kNatUnroll; ++k) {  // all loads first, then the arithmetic
-                const long long q = q0 + k * stride;
-                if (q < nq) v[k] = __ldcs(reinterpret_cast<const float4*>(xr) + q);
-            }
-#pragma unroll
-            for (int k = 0; k < kNatUnroll; ++k) {
-                const long long q = q0 + k * stride;
-                if (q < nq) {
-                    const uint4 rnd = philox10(philox_counter((unsigned long long)q, step, wid),
-                                               a.rk);
-                    const uint32_t c0 = nat_code(v[k].x, rnd.x, bad);
-                    const uint32_t c1 = nat_code(v[k].y, rnd.y, bad);
-                    const uint32_t c2 = nat_code(v[k].z, rnd.z, bad);
-                    const uint32_t c3 = nat_code(v[k].w, rnd.w, bad);
-                    __stcs(reinterpret_cast<uint2*>(cr) + q,
-                           make_uint2(c0 | (c1 << 16), c2 | (c3 << 16)));
-                }
-            }
+        for (int k = 0; k < kNatStages - 1; ++k) {
+            if (k < nit) nat_cp_async16(&ring[k][threadIdx.x], x4 + q0 + k * stride);
+            nat_cp_async_commit();
         }
+        for (long long it = 0; it < nit; ++it) {
+            const long long ahead = it + kNatStages - 1;
+            if (ahead < nit)
+                nat_cp_async16(&ring[ahead % kNatStages][threadIdx.x], x4 + q0 + ahead * stride);
+            nat_cp_async_commit();
+            nat_cp_async_wait<kNatStages - 1>();  // this thread's copy of group `it` landed
+            const float4 v = ring[it % kNatStages][threadIdx.x];
+            const long long q = q0 + it * stride;
+            const uint4 rnd = philox10(philox_counter((unsigned long long)q, step, wid), a.rk);
+            const uint32_t c0 = nat_code(v.x, rnd.x, bad), c1 = nat_code(v.y, rnd.y, bad);
+            const uint32_t c2 = nat_code(v.z, rnd.z, bad), c3 = nat_code(v.w, rnd.w, bad);
+            __stcs(reinterpret_cast<uint2*>(cr) + q, make_uint2(c0 | (c1 << 16), c2 | (c3 << 16)));
+        }
+        nat_cp_async_wait<0>();
     } else {
         for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < nq;
              q += stride) {
@@ -161,8 +180,7 @@ cudaError_t launch_nat_quantize(const NatArgs& a, bool vec, int sms, cudaStream_
     const void* fn = vec ? (const void*)nat_quantize_kernel<true>
                          : (const void*)nat_quantize_kernel<false>;
     const long long per_row = (long long)sms * resident_blocks(fn) / a.W;
-    const long long need = (nq + (long long)kThreads * (vec ? kNatUnroll : 1) - 1) /
-                           ((long long)kThreads * (vec ? kNatUnroll : 1));
+    const long long need = (nq + kThreads - 1) / kThreads;
     long long gx = need < per_row ? need : per_row;
     if (gx < 1) gx = 1;
     const dim3 grid((unsigned)gx, (unsigned)a.W);
