@@ -8,11 +8,20 @@ gradients already resident in HBM: gq_global_norm (read 1) then
 gq_quantize_aggregate (read 2: Philox uniforms, stochastic rounding, packed
 codes at wire width, integer sum over workers, decoded mean).  These two calls
 are exactly what gq_step_fused issues; the benchmark makes them separately so
-that CUDA events bracket the dominant kernel on its own stream.
+that, in a second pass of K steps, CUDA events can bracket each kernel.  The
+job's own time comes from K steps with events around the run only.
 
 Metric: fp32 gradient GB/s = 4 * W * d bytes / step time (whole job: summed
 over ranks under torchrun, each rank an independent replica, timed as the max
-over ranks).  Prints one JSON line on rank 0.
+over ranks).  Prints one JSON line on rank 0.  The line also carries the step
+without materialised codes, the roofline of the dominant kernel, an end-to-end
+figure through host buffers, and the CPU oracle single- and multi-threaded.
+
+Other modes print their own JSON line: --sweep (d = 2^16..2^30, EF off/on,
+eager and graph-replayed), --buckets (per-bucket scales), --lq (the log
+quantizer), --lqsgd (the PowerSGD + LQ step), --nat (natural compression),
+--dp (the real exchange under torchrun, eager and graph-replayed, against an
+fp32 all-reduce).
 
 --impl reference times the CPU oracle (the plain restatement of the method
 used by the tests) on the host cores, on a bounded sample of the same
