@@ -276,19 +276,42 @@ class DataParallelLqsgdStep:
         return ghat
 
 
+class GpuNatOps:
+    """The library's natural-compression kernels."""
+
+    def quantize(self, x, cfg, codes, ws):
+        from . import gq_nat_quantize
+        gq_nat_quantize(x, cfg, codes, ws)
+
+    def decode_sum(self, codes, out):
+        from . import gq_nat_decode_sum
+        gq_nat_decode_sum(codes, out)
+
+    def status(self, ws):
+        return gq_get_device_status(ws)
+
+
 class DataParallelNatStep:
     """Natural compression (Horvath et al., "Natural Compression for Distributed
-    Deep Learning", cited in the Global-QSGD record) across ranks: each rank
+    Deep Learning", cited in the Global-QSGD record) across ranks.  Each rank
     rounds its own W_local rows to signed powers of two (gq_nat_quantize, workers
-    rank * W_local + w), the 16-bit codes are all-gathered (as bytes, rank-major),
-    and every rank decodes and sums all W workers in ascending order
-    (gq_nat_decode_sum), so the sum is the same on every rank and equals the
-    single-GPU one.  Powers of two over the whole exponent range cannot be summed
-    as fixed-width integers, so this exchange gathers instead of all-reducing:
-    (N - 1) * 2n bytes in per rank, against 2 (N - 1)/N * 4n for a ring fp32
-    all-reduce."""
+    rank * W_local + w); every coordinate's result is the fp32 sum of all W
+    workers' decoded values in ascending worker order, the same on every rank
+    and equal to the single-GPU sum.  Powers of two over the whole exponent range
+    cannot be summed as fixed-width integers, so the codes travel instead:
 
-    def __init__(self, n, w_local=1, seed=0, group=None, device=None):
+    - gather (default): the 16-bit codes are all-gathered (as bytes, rank-major)
+      and every rank decodes the whole sum: (N - 1) * 2n bytes in per rank;
+    - sharded (one worker per rank): an all-to-all sends each rank the codes of
+      its column shard, it decodes and sums that shard, and the fp32 shard sums
+      are all-gathered: (N - 1)/N * 6n bytes, against (N - 1)/N * 8n for a ring
+      fp32 all-reduce.  Shards are rounded up to 8 coordinates (padding columns
+      carry code 0, value 0).
+
+    The kernels are reached through ``ops`` (``GpuNatOps`` by default) so that
+    the host orchestration can be tested with other backends."""
+
+    def __init__(self, n, w_local=1, seed=0, group=None, device=None, sharded=False, ops=None):
         from . import gq_workspace_init as _init
         self.group = group
         self.world = dist.get_world_size(group)
@@ -297,10 +320,26 @@ class DataParallelNatStep:
         self.w_local = int(w_local)
         self.W = self.world * self.w_local
         self.seed = int(seed)
+        self.sharded = bool(sharded)
+        self.ops = ops if ops is not None else GpuNatOps()
         dev = torch.device(device) if device is not None else torch.device("cuda")
-        self.codes_l = torch.empty((self.w_local, self.n), dtype=torch.int16, device=dev)
-        self.codes = torch.empty((self.W, self.n), dtype=torch.int16, device=dev)
-        self.out = torch.empty(self.n, dtype=torch.float32, device=dev)
+        if self.sharded:
+            if self.w_local != 1:
+                raise ValueError("sharded exchange: one worker per rank")
+            shard = -(-self.n // self.world)
+            self.shard = -(-shard // 8) * 8
+            # padded row [N][shard] rank-major; the padding stays code 0
+            self.codes_row = torch.zeros((1, self.world * self.shard), dtype=torch.int16,
+                                         device=dev)
+            self.codes_l = self.codes_row[:, :self.n]
+            self.recv = torch.empty((self.world, self.shard), dtype=torch.int16, device=dev)
+            self.part = torch.empty(self.shard, dtype=torch.float32, device=dev)
+            self.full = torch.empty(self.world * self.shard, dtype=torch.float32, device=dev)
+            self.out = self.full[:self.n]
+        else:
+            self.codes_l = torch.empty((self.w_local, self.n), dtype=torch.int16, device=dev)
+            self.codes = torch.empty((self.W, self.n), dtype=torch.int16, device=dev)
+            self.out = torch.empty(self.n, dtype=torch.float32, device=dev)
         self.ws = torch.zeros(256, dtype=torch.uint8, device=dev)
         if dev.type == "cuda":
             _init(self.ws)
@@ -308,15 +347,20 @@ class DataParallelNatStep:
     def __call__(self, x, step, check=False):
         """x: this rank's [w_local][n] fp32 rows.  Returns the sum over all W
         workers' compressed rows, [n] fp32 (divide by W for the mean)."""
-        from . import gq_nat_decode_sum, gq_nat_quantize
         cfg = GQConfig(levels="nat", seed=self.seed, step=int(step),
                        worker0=self.rank * self.w_local)
-        gq_nat_quantize(x, cfg, self.codes_l, self.ws)
-        gather_rows(self.codes_l.view(torch.uint8), self.codes.view(torch.uint8), self.group)
-        gq_nat_decode_sum(self.codes, self.out)
+        self.ops.quantize(x, cfg, self.codes_l, self.ws)
+        if self.sharded:
+            dist.all_to_all_single(self.recv.view(torch.uint8).view(-1),
+                                   self.codes_row.view(torch.uint8).view(-1), group=self.group)
+            self.ops.decode_sum(self.recv, self.part)
+            gather_rows(self.part.view(1, -1), self.full.view(self.world, -1), self.group)
+        else:
+            gather_rows(self.codes_l.view(torch.uint8), self.codes.view(torch.uint8),
+                        self.group)
+            self.ops.decode_sum(self.codes, self.out)
         if check:
-            rc = gq_get_device_status(self.ws)
+            rc = self.ops.status(self.ws)
             if rc != GQ_OK:
                 raise GQError(rc, "DataParallelNatStep")
         return self.out
-

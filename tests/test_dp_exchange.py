@@ -208,37 +208,55 @@ def test_gathered_log_codes_decode_like_one_process(oracle, tmp_path):
         assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), r
 
 
-def _nat_main(rank, world, port, outdir):
+class OracleNatOps:
+    """The oracle in place of the natural-compression kernels (host tests only)."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    def quantize(self, x, cfg, codes, ws):
+        c = self.o.nat_quantize(x.numpy(), seed=cfg.seed, step=cfg.step, worker0=cfg.worker0)
+        codes.copy_(torch.from_numpy(c.view(np.int16)))
+
+    def decode_sum(self, codes, out):
+        out.copy_(torch.from_numpy(self.o.nat_decode_sum(codes.numpy().view(np.uint16))))
+
+    def status(self, ws):
+        return 0
+
+
+def _nat_main(rank, world, port, outdir, w_local, n, sharded):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         import oracle
-        from allreduce_compatible_gradient_global_b200.dp import gather_rows
-        w_local, n = 2, 301
+        from allreduce_compatible_gradient_global_b200.dp import DataParallelNatStep
         W = world * w_local
-        x = synthetic.make_gradients(W, n, "student_t3", seed=6, seg=50, lo=-20, hi=3).numpy()
+        x = synthetic.make_gradients(W, n, "student_t3", seed=6, seg=50, lo=-20, hi=3)
         rows = slice(rank * w_local, (rank + 1) * w_local)
-        mine = oracle.nat_quantize(x[rows], seed=4, step=9, worker0=rank * w_local)
-        codes = torch.empty((W, n), dtype=torch.int16)
-        # the 16-bit codes travel as bytes (gloo reduces no 16-bit integers)
-        gather_rows(torch.from_numpy(mine.view(np.int16)).view(torch.uint8),
-                    codes.view(torch.uint8))
-        total = oracle.nat_decode_sum(codes.numpy().view(np.uint16))
-        np.save(os.path.join(outdir, f"nat{rank}.npy"), total)
+        step = DataParallelNatStep(n, w_local=w_local, seed=4, device="cpu", sharded=sharded,
+                                   ops=OracleNatOps(oracle))
+        outs = [step(x[rows].clone(), t).clone().numpy() for t in (9, 10)]
+        np.savez(os.path.join(outdir, f"nat{rank}.npz"), out0=outs[0], out1=outs[1])
     finally:
         dist.destroy_process_group()
 
 
-def test_gathered_natural_codes_sum_like_one_process(oracle, tmp_path):
-    """Each rank compresses its own workers (worker offset rank * W_local), the
-    codes are all-gathered as bytes, rank-major, and every rank's decoded sum
-    equals the single-process sum of all workers, bit for bit."""
-    world = 2
-    mp.start_processes(_nat_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
-                       join=True, start_method="spawn")
-    x = synthetic.make_gradients(4, 301, "student_t3", seed=6, seg=50, lo=-20, hi=3).numpy()
-    ref = oracle.nat_decode_sum(oracle.nat_quantize(x, seed=4, step=9))
-    for r in range(world):
-        got = np.load(tmp_path / f"nat{r}.npy")
-        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), r
+@pytest.mark.parametrize("world,w_local,n,sharded", [(2, 2, 301, False), (2, 1, 301, True),
+                                                     (3, 1, 1000, True), (3, 1, 5, True)])
+def test_natural_exchange_sums_like_one_process(oracle, tmp_path, world, w_local, n, sharded):
+    """Gather: each rank compresses its own workers (worker offset rank * W_local)
+    and the codes are all-gathered as bytes.  Sharded: an all-to-all hands each
+    rank the codes of its column shard, which it decodes and sums, and the fp32
+    shard sums are all-gathered.  Either way every rank's sum equals the
+    single-process sum of all workers, bit for bit."""
+    mp.start_processes(_nat_main, args=(world, _free_port(), str(tmp_path), w_local, n, sharded),
+                       nprocs=world, join=True, start_method="spawn")
+    W = world * w_local
+    x = synthetic.make_gradients(W, n, "student_t3", seed=6, seg=50, lo=-20, hi=3).numpy()
+    for t in (9, 10):
+        ref = oracle.nat_decode_sum(oracle.nat_quantize(x, seed=4, step=t))
+        for r in range(world):
+            got = np.load(tmp_path / f"nat{r}.npz")[f"out{t - 9}"]
+            assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (t, r)
 

@@ -177,23 +177,25 @@ def test_nccl_graph_replay_equals_eager_exchange(gq, chunks, w_local, kw):
         dist.destroy_process_group()
 
 
-def test_nccl_single_rank_natural_exchange_matches_the_oracle(gq, oracle):
-    """DataParallelNatStep on one NCCL rank holding all W workers: the gathered
-    codes and the decoded sum equal the oracle's, bit for bit."""
+@pytest.mark.parametrize("W,sharded", [(4, False), (1, True)])
+def test_nccl_single_rank_natural_exchange_matches_the_oracle(gq, oracle, W, sharded):
+    """DataParallelNatStep on one NCCL rank (all W workers gathered, or one
+    worker through the all-to-all of the sharded form): the codes and the
+    decoded sum equal the oracle's, bit for bit."""
     from allreduce_compatible_gradient_global_b200.dp import DataParallelNatStep
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
     dist.init_process_group("nccl", rank=0, world_size=1,
                             timeout=datetime.timedelta(seconds=60),
                             device_id=torch.device("cuda", 0))
     try:
-        W, n = 4, 50_001
+        n = 50_001
         x = synthetic.make_gradients(W, n, "student_t3", seed=8, device="cuda", seg=100, lo=-25,
                                      hi=2)
-        step = DataParallelNatStep(n, w_local=W, seed=21)
+        step = DataParallelNatStep(n, w_local=W, seed=21, sharded=sharded)
         for t in range(2):
             out = step(x, t, check=True).clone()
             ref = oracle.nat_quantize(x.cpu().numpy(), seed=21, step=t)
-            assert np.array_equal(step.codes.cpu().numpy().view(np.uint16), ref)
+            assert np.array_equal(step.codes_l.cpu().numpy().view(np.uint16), ref)
             want = oracle.nat_decode_sum(ref)
             assert np.array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32)), t
     finally:
