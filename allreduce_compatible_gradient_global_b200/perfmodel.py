@@ -12,6 +12,10 @@ method across hardware; its content is not given.  This is a plain one:
   local quantize pass, a SUM all-reduce of the int8/int16 codes, and the local
   decode.  The uncompressed step is one fp32 SUM all-reduce.  A ring all-reduce
   of B bytes over N ranks costs alpha + 2 (N - 1) / N * B / link_bandwidth.
+* Natural compression (a gather-style compressor) exchanges codes instead of a
+  sum: an all-gather of every rank's 2n bytes ((N - 1) * 2n in per rank), or,
+  sharded, an all-to-all of code shards ((N - 1)/N * 2n) and an all-gather of
+  fp32 shard sums ((N - 1)/N * 4n).
 
 Everything here is host arithmetic on numbers the caller measures or chooses;
 nothing runs on the GPU.
@@ -110,3 +114,41 @@ def crossover_d(ranks, bits=8, sum_bytes=1, m=Machine(), lo=1, hi=1 << 40):
         else:
             lo = mid
     return hi
+
+
+def all_gather_seconds(nbytes_per_rank, ranks, link_bytes_per_s, alpha_s):
+    """Ring all-gather of nbytes from every rank: each rank receives the other
+    N - 1 contributions, alpha + (N - 1) * bytes / link bandwidth."""
+    if ranks <= 1:
+        return 0.0
+    return alpha_s + (ranks - 1) * nbytes_per_rank / link_bytes_per_s
+
+
+def all_to_all_seconds(nbytes_per_rank, ranks, link_bytes_per_s, alpha_s):
+    """All-to-all of an nbytes buffer split evenly over N ranks: each rank sends
+    and receives (N - 1)/N of it, alpha + (N - 1)/N * bytes / link bandwidth."""
+    if ranks <= 1:
+        return 0.0
+    return alpha_s + (ranks - 1) / ranks * nbytes_per_rank / link_bytes_per_s
+
+
+def nat_step_seconds(n, ranks, m=Machine(), sharded=False, quant_efficiency=0.77,
+                     decode_efficiency=0.91):
+    """One natural-compression exchange with one worker per GPU: the quantize
+    pass (read 4n, write 2n), then either an all-gather of the 2n-byte codes and
+    a decode-sum over all N workers (read 2Nn, write 4n), or, sharded, an
+    all-to-all of code shards, a decode-sum of this rank's shard (read 2N
+    shard, write 4 shard) and an all-gather of the fp32 shard sums.  The two
+    efficiencies are the measured fractions of hbm the two kernels reach."""
+    N = max(1, int(ranks))
+    quant = m.launch + 6.0 * n / (m.hbm * quant_efficiency)
+    if not sharded:
+        move = all_gather_seconds(2.0 * n, N, m.link, m.allreduce_alpha)
+        decode = m.launch + (2.0 * N * n + 4.0 * n) / (m.hbm * decode_efficiency)
+        return quant + move + decode
+    shard = -(-int(n) // N)
+    a2a = all_to_all_seconds(2.0 * N * shard, N, m.link, m.allreduce_alpha)
+    decode = m.launch + (2.0 * N * shard + 4.0 * shard) / (m.hbm * decode_efficiency)
+    gather = all_gather_seconds(4.0 * shard, N, m.link, m.allreduce_alpha)
+    return quant + a2a + decode + gather
+

@@ -91,3 +91,47 @@ def test_chunked_pipeline_model():
     assert four < one
     assert four > norm + scale + decode + max(quant, summ)
     assert pm.dp_step_seconds(d, N, m=m, chunks=1 << 16) > four
+
+
+def test_natural_exchange_link_bytes():
+    """Sharded: (N-1)/N * 2n (all-to-all of codes) + (N-1)/N * 4n (all-gather of
+    fp32 shard sums) = 3/4 of a ring fp32 all-reduce's 2 (N-1)/N * 4n; gather:
+    (N-1) * 2n.  Checked with free HBM and latencies so only link time is left."""
+    m = pm.Machine(hbm=float("inf"), allreduce_alpha=0.0, launch=0.0)
+    n = 8 * 1_000_000
+    for N in (2, 4, 8):
+        fp32 = pm.dp_step_seconds(n, N, m=m, compressed=False)
+        sharded = pm.nat_step_seconds(n, N, m=m, sharded=True)
+        gather = pm.nat_step_seconds(n, N, m=m)
+        assert sharded == pytest.approx(0.75 * fp32, rel=1e-12)
+        assert gather == pytest.approx((N - 1) * 2 * n / m.link, rel=1e-12)
+
+
+def test_natural_exchange_on_one_rank_is_the_two_kernels():
+    m = pm.Machine()
+    n = 1 << 24
+    want = (m.launch + 6.0 * n / (m.hbm * 0.77)) + (m.launch + 6.0 * n / (m.hbm * 0.91))
+    assert pm.nat_step_seconds(n, 1, m=m) == pytest.approx(want)
+    assert pm.nat_step_seconds(n, 1, m=m, sharded=True) == pytest.approx(want)
+
+
+def test_allreduce_compatible_exchange_beats_natural_compression():
+    """Bandwidth regime (d >= 2^25): the integer all-reduce of the shared-scale
+    codes beats both natural-compression exchanges at every rank count, and the
+    sharded form beats the gather from 4 ranks on.  Latency regime (d = 2^20,
+    2 and 4 ranks; at 8 ranks the three are within 0.2 us): the integer exchange
+    pays two collectives (the scale's MAX and the sum), the natural gather one,
+    and the gather is the fastest of the three."""
+    for N in (2, 4, 8):
+        for d in (1 << 25, 1 << 30):
+            int8 = pm.dp_step_seconds(d, N)
+            assert int8 < pm.nat_step_seconds(d, N, sharded=True)
+            assert int8 < pm.nat_step_seconds(d, N)
+            if N >= 4:
+                assert pm.nat_step_seconds(d, N, sharded=True) < pm.nat_step_seconds(d, N)
+    for N in (2, 4):
+        d = 1 << 20
+        gather = pm.nat_step_seconds(d, N)
+        assert gather < pm.dp_step_seconds(d, N)
+        assert gather < pm.nat_step_seconds(d, N, sharded=True)
+
