@@ -260,3 +260,18 @@ def test_natural_exchange_sums_like_one_process(oracle, tmp_path, world, w_local
             got = np.load(tmp_path / f"nat{r}.npz")[f"out{t - 9}"]
             assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (t, r)
 
+
+def test_sharded_natural_exchange_needs_one_worker_per_rank():
+    """The column shards are slices of one code row: more rows per rank are refused."""
+    from allreduce_compatible_gradient_global_b200.dp import DataParallelNatStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        with pytest.raises(ValueError):
+            DataParallelNatStep(100, w_local=2, device="cpu", sharded=True)
+        step = DataParallelNatStep(101, w_local=1, device="cpu", sharded=True)
+        assert step.shard % 8 == 0 and step.shard * step.world >= 101
+        assert step.codes_l.is_contiguous() and step.codes_l.shape == (1, 101)
+    finally:
+        dist.destroy_process_group()
+
