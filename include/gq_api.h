@@ -28,7 +28,11 @@
  * Side variant: the LQ-SGD log quantizer on low-rank factors (same review,
  * "Core claim": q(x) = sign(x) log(1 + a|x|)/log(1 + a), 2^b bins, b = 8;
  * referee major comment 1 on Section IV-A, Eqs. (5)-(6): normalise by the max
- * magnitude; Eq. (6) is the inverse map).
+ * magnitude; Eq. (6) is the inverse map), alone (gq_logq_*) or inside the
+ * PowerSGD step (gq_psgd_*, gq_lqsgd_step).  Further variants: per-bucket
+ * scales (gq_bucket_*, gq_*_bucketed) and natural compression (gq_nat_*,
+ * Horvath et al., cited in the Global-QSGD crossref record), a gather-style
+ * compressor outside the all-reduce path.
  *
  * Conventions for every entry point:
  *  - Pointers named *_dev are device pointers, owned by the caller; the library
