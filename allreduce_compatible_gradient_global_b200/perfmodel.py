@@ -152,3 +152,23 @@ def nat_step_seconds(n, ranks, m=Machine(), sharded=False, quant_efficiency=0.77
     gather = all_gather_seconds(4.0 * shard, N, m.link, m.allreduce_alpha)
     return quant + a2a + decode + gather
 
+
+def nat_crossover_d(ranks, m=Machine(), sharded=True, lo=1, hi=1 << 40):
+    """Smallest n (bisection over integers) from which the natural-compression
+    exchange is faster than the fp32 all-reduce; None if it never is in
+    [lo, hi]."""
+    def gain(n):
+        return (dp_step_seconds(n, ranks, m=m, compressed=False)
+                - nat_step_seconds(n, ranks, m=m, sharded=sharded))
+    if gain(hi) <= 0:
+        return None
+    if gain(lo) > 0:
+        return lo
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if gain(mid) > 0:
+            hi = mid
+        else:
+            lo = mid
+    return hi
+

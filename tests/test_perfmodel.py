@@ -135,3 +135,18 @@ def test_allreduce_compatible_exchange_beats_natural_compression():
         assert gather < pm.dp_step_seconds(d, N)
         assert gather < pm.nat_step_seconds(d, N, sharded=True)
 
+
+def test_natural_exchange_crossover_against_fp32():
+    """Sharded natural compression overtakes the fp32 all-reduce only at large n
+    (about 92 M coordinates on 4 ranks and 35 M on 8 with the default machine),
+    never on 2 ranks; the gather form never does from 4 ranks on."""
+    assert pm.nat_crossover_d(2) is None
+    c4, c8 = pm.nat_crossover_d(4), pm.nat_crossover_d(8)
+    assert 85e6 < c4 < 100e6 and 30e6 < c8 < 40e6
+    for N in (4, 8):
+        c = pm.nat_crossover_d(N)
+        assert pm.nat_step_seconds(c, N, sharded=True) < pm.dp_step_seconds(c, N, compressed=False)
+        assert pm.nat_step_seconds(c - 1, N, sharded=True) >= \
+            pm.dp_step_seconds(c - 1, N, compressed=False)
+        assert pm.nat_crossover_d(N, sharded=False) is None
+
