@@ -99,18 +99,6 @@ int check_sizes(int W, long long d) {
     return GQ_OK;
 }
 
-// Blocks per worker of the norm pass: one full wave of resident blocks over
-// all workers, so that no block starts late and leaves a tail.
-int norm_blocks_per_worker(int W, long long d, int kind, bool has_e) {
-    const long long resident = (long long)sm_count() * norm_resident_blocks(kind, has_e, d % 4 == 0);
-    const long long want = resident / W > 0 ? resident / W : 1;
-    const long long useful = (d + (long long)kThreads * 16 - 1) / ((long long)kThreads * 16);
-    long long nb = want < useful ? want : useful;
-    if (nb < 1) nb = 1;
-    if (nb > kMaxNormBlocks) nb = kMaxNormBlocks;
-    return (int)nb;
-}
-
 int stream_grid(long long d);
 
 // The bulk-copy pipeline of the fused pass: stages per block (compile-time
@@ -196,6 +184,7 @@ void fill_quant_args(QuantArgs& a, const gq_config* cfg, int W, long long d) {
     a.smax = (float)cfg->s;
     a.finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, -(cfg->L - 1)) : 1.0f;
     a.inv_finest = cfg->levels == GQ_EXP ? std::ldexp(1.0f, cfg->L - 1) : 1.0f;
+    a.exp_shift = cfg->levels == GQ_EXP ? std::ldexp(1.0f, cfg->L - 127) : 1.0f;
     a.w_pow2 = is_pow2(W) ? 1 : 0;
     a.inv_w = a.w_pow2 ? 1.0f / (float)W : 0.0f;
 }
@@ -216,6 +205,24 @@ size_t bucket_ws_bytes(int W, long long d, int b) {
 }
 
 }  // namespace
+
+namespace gq {
+
+// Blocks per worker of the norm pass: one full wave of resident blocks over
+// all workers, so that no block starts late and leaves a tail.  The fp32 runs
+// and the fp64 combine order follow from this count, so every caller of the
+// norm kernel that wants gq_global_norm's exact scale uses it.
+int norm_blocks_per_worker(int W, long long d, int kind, bool has_e) {
+    const long long resident = (long long)sm_count() * norm_resident_blocks(kind, has_e, d % 4 == 0);
+    const long long want = resident / W > 0 ? resident / W : 1;
+    const long long useful = (d + (long long)kThreads * 16 - 1) / ((long long)kThreads * 16);
+    long long nb = want < useful ? want : useful;
+    if (nb < 1) nb = 1;
+    if (nb > kMaxNormBlocks) nb = kMaxNormBlocks;
+    return (int)nb;
+}
+
+}  // namespace gq
 
 extern "C" {
 

@@ -140,32 +140,31 @@ __device__ __forceinline__ int quant_exp(float v, float a, int L, float finest, 
     return with_sign_of(idx, v);
 }
 
-// Exponential levels without branches, for a = 1/S rounded down (so |r| <= 1
-// for every |v| <= S).  The signed level value Q (0, +-2^-(L-1), ..., +-1) is
-// built in the bit pattern of r: for |r| >= 2^-(L-1), adding the 23 random
-// bits f to the pattern carries out of the mantissa exactly when
-// m + f >= 2^23 -- the round-up event -- and bumps the exponent to the upper
-// level; masking to sign and exponent leaves +-2^E or +-2^(E+1).  Below the
-// finest level, r' = r + sign * 2^-(L-1) rounded toward zero has mantissa
-// floor(p 2^23) with p = |r| 2^(L-1), the same carry decides p + u >= 1, and
-// subtracting the added level leaves 0 or +-2^-(L-1).
-__device__ __forceinline__ float quant_exp_level(float v, float a, float finest, uint32_t word) {
-    const float r = __fmul_rn(v, a);
-    const uint32_t f = top23(word);
-    const float fin_s = __uint_as_float(__float_as_uint(finest) | (__float_as_uint(r) & 0x80000000u));
-    const bool small = fabsf(r) < finest;
-    const float x = small ? __fadd_rz(r, fin_s) : r;
-    const float q = __uint_as_float((__float_as_uint(x) + f) & 0xFF800000u);
-    return small ? __fsub_rn(q, fin_s) : q;
+// Exponential levels by the exponent carry, with the finest level moved onto
+// 2^-126 so that no bracket needs a case of its own.  r = fl(v a) is scaled
+// by shift = 2^(L-127) rounding toward zero: exact for |r| >= 2^-(L-1), and
+// below that the subnormal result's mantissa is floor(p 2^23) with
+// p = |r| 2^(L-1), the bottom bracket's round-up probability.  The 23 random
+// bits f are added to the bit pattern in one multiply-add (the high half of
+// word * 2^23 is word >> 9): the carry out of the mantissa is the round-up
+// event m + f >= 2^23 in every bracket.  Masking the result to sign and
+// exponent gives the rounded level +-2^(idx-127) (idx = the level index,
+// exponent field 0 for the zero level); its top nine bits are sign and index.
+__device__ __forceinline__ uint32_t exp_round_bits(float v, float a, float shift, uint32_t word) {
+    const float rs = __fmul_rz(__fmul_rn(v, a), shift);
+    uint32_t y;
+    asm("mad.hi.u32 %0, %1, %2, %3;"
+        : "=r"(y)
+        : "r"(word), "r"(0x00800000u), "r"(__float_as_uint(rs)));
+    return y;
 }
 
-// The signed level index (the code) of a level value Q from its exponent:
-// Q = +-2^E has index L + E; Q = 0 has index 0.
-__device__ __forceinline__ int exp_code_of_level(float q, int L) {
-    const uint32_t qb = __float_as_uint(q);
-    const int idx = max((int)((qb >> 23) & 0xFFu) - (127 - L), 0);
-    const int sgn = (int)qb >> 31;
-    return (idx ^ sgn) - sgn;
+// A float holding a sum of rounded levels from exp_round_bits, as the integer
+// number of finest levels it holds: t = f 2^126 is that integer (exact), and
+// for |t| < 2^22 the bits of 1.5 * 2^23 + t are those of 1.5 * 2^23 plus t.
+__device__ __forceinline__ int float_units_to_int(float f) {
+    const float t = __fmul_rn(f, 0x1p126f);
+    return __float_as_int(__fadd_rn(t, 12582912.0f)) - 0x4B400000;
 }
 
 // Value a code adds to the sum: the code itself (uniform levels) or
@@ -316,9 +315,11 @@ struct Unpacker {
 // ---------------------------------------------------------------------------
 // Per-coordinate outputs shared by the fused kernels.
 // ---------------------------------------------------------------------------
-// The [d] mean output: its base is 16-byte aligned and j0 % 4 == 0.
+// The [d] mean output: its base is 16-byte aligned and j0 % 4 == 0.  FULL:
+// the caller knows that j0 + 3 < d.
+template <bool FULL = false>
 __device__ __forceinline__ void store_out4(float* out, long long j0, long long d, float4 v) {
-    if (j0 + 3 < d) {
+    if (FULL || j0 + 3 < d) {
         __stcs(reinterpret_cast<float4*>(out + j0), v);
         return;
     }
@@ -344,10 +345,11 @@ __device__ __forceinline__ int f16_bits_to_int(uint32_t h) {
 // The [d] outputs (sum, mean) are vectors of their own: j0 is a multiple of 4,
 // so a 4-wide store is aligned whenever all 4 coordinates are in range.
 // wire: 1 int8, 2 int16, 3 fp16 holding the integer.
+template <bool FULL = false>
 __device__ __forceinline__ void store_sum_16(void* sum, long long j0, long long d, uint32_t s0,
                                              uint32_t s1, uint32_t s2, uint32_t s3) {
     unsigned short* p = reinterpret_cast<unsigned short*>(sum) + j0;
-    if (j0 + 3 < d) {
+    if (FULL || j0 + 3 < d) {
         uint2 x;
         x.x = (s0 & 0xFFFFu) | (s1 << 16);
         x.y = (s2 & 0xFFFFu) | (s3 << 16);
@@ -359,16 +361,17 @@ __device__ __forceinline__ void store_sum_16(void* sum, long long j0, long long 
     }
 }
 
+template <bool FULL = false>
 __device__ __forceinline__ void store_sum(void* sum, int wire, long long j0, long long d, int s0,
                                           int s1, int s2, int s3) {
     if (wire == 3) {
-        store_sum_16(sum, j0, d, int_to_f16_bits(s0), int_to_f16_bits(s1), int_to_f16_bits(s2),
-                     int_to_f16_bits(s3));
+        store_sum_16<FULL>(sum, j0, d, int_to_f16_bits(s0), int_to_f16_bits(s1),
+                           int_to_f16_bits(s2), int_to_f16_bits(s3));
         return;
     }
     if (wire == 1) {
         signed char* p = reinterpret_cast<signed char*>(sum) + j0;
-        if (j0 + 3 < d) {
+        if (FULL || j0 + 3 < d) {
             const uint32_t x = (uint32_t)(s0 & 255) | ((uint32_t)(s1 & 255) << 8) |
                                ((uint32_t)(s2 & 255) << 16) | ((uint32_t)(s3 & 255) << 24);
             __stcs(reinterpret_cast<unsigned int*>(p), x);
@@ -378,7 +381,7 @@ __device__ __forceinline__ void store_sum(void* sum, int wire, long long j0, lon
             if (j0 + 2 < d) p[2] = (signed char)s2;
         }
     } else {
-        store_sum_16(sum, j0, d, (uint32_t)s0, (uint32_t)s1, (uint32_t)s2, (uint32_t)s3);
+        store_sum_16<FULL>(sum, j0, d, (uint32_t)s0, (uint32_t)s1, (uint32_t)s2, (uint32_t)s3);
     }
 }
 

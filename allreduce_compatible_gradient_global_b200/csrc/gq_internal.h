@@ -18,6 +18,8 @@ constexpr int kWorkspaceHeader = 256;  // flag word, ticket counter, padding
 struct WsHeader {
     unsigned int flags;    // bit 0: non-finite scale; bit 1: non-finite LQ max
     unsigned int counter;  // last-block ticket of the norm kernel (0 between calls)
+    unsigned int tile_next;  // fused pass: next unclaimed tile (0 between calls)
+    unsigned int tile_done;  // fused pass: producers finished (0 between calls)
 };
 
 constexpr unsigned kFlagNonfiniteScale = 1u;
@@ -58,6 +60,7 @@ struct QuantArgs {
     float smax;        // (float)s
     float finest;      // 2^-(L-1)
     float inv_finest;  // 2^(L-1)
+    float exp_shift;   // 2^(L-127): moves the finest level onto 2^-126
     float inv_w;       // 1/W when W is a power of two
     int w_pow2;
     WsHeader* hdr;  // flag word for pipeline timeouts
@@ -156,6 +159,8 @@ inline cudaError_t ensure_dynamic_smem(const void* kern, size_t smem, int* limit
 cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st);
 // Resident blocks per SM of the norm kernel instantiation for (kind, e?, vec).
 int norm_resident_blocks(int kind, bool has_e, bool vec);
+// Blocks per worker row of the norm kernel on the current device (its grid's x).
+int norm_blocks_per_worker(int W, long long d, int kind, bool has_e);
 cudaError_t launch_quant(const QuantArgs& a, int levels, int bits, bool ef, bool vec, int grid,
                          cudaStream_t st);
 cudaError_t launch_aggregate(const AggArgs& a, int levels, int bits, int grid, cudaStream_t st);

@@ -17,7 +17,27 @@
 // producer drains the copies it issued before the block exits.
 //
 // Arithmetic, packing and outputs are those of quant_kernel, bit for bit.
+//
+// Exponential levels take a shorter road to the same codes.  r = fl(v a) is
+// scaled by 2^(L-127) rounding toward zero, which puts the finest level
+// 2^-(L-1) on 2^-126: a level's index becomes the biased exponent field, and
+// the bottom bracket [0, 2^-(L-1)) becomes the subnormal range, whose mantissa
+// is floor(p 2^23) with p = |r| 2^(L-1).  Adding the 23 random bits to the bit
+// pattern carries out of the mantissa exactly on the round-up event in every
+// bracket, the bottom one included, so one integer add and one mask give the
+// rounded level as a float (+-2^(idx-127), or +-0), and the top nine bits
+// (sign, exponent) index a 512-entry table of signed codes in shared memory.
+//
+// Tile order: each block's producer claims the next tile from a counter in
+// the workspace header, so every block works inside the same narrow window of
+// the rows however unevenly the blocks progress (measured on W = 8 rows of
+// 2^26 to 2^30 coordinates: 3-4% faster than block b taking tiles b, b + grid,
+// b + 2 grid, ...).  The last producer to finish puts the counter back to zero,
+// so two launches must not share a workspace at the same time.  The
+// per-bucket instantiation keeps the static order: it prefetches the next
+// block's scale a tile ahead.
 #include <cfloat>
+#include <type_traits>
 
 #include "gq_internal.h"
 
@@ -37,6 +57,29 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 #ifndef GQ_TMA_SPECIALIZE_W8
 #define GQ_TMA_SPECIALIZE_W8 1
 #endif
+
+// 1: exponential-level codes in a byte table at a fixed shared address (the
+// top nine bits index it directly); 0: a 32-bit table after the ring.
+#ifndef GQ_EXP_BYTE_TABLE
+#define GQ_EXP_BYTE_TABLE 1
+#endif
+// 1: whole tiles take a copy of the block body without bounds checks.
+#ifndef GQ_TMA_FULL_TILES
+#define GQ_TMA_FULL_TILES 0
+#endif
+// 1: with the worker count fixed at compile time, uniform-level patterns of
+// two workers enter the sums in one three-input add.
+#ifndef GQ_PAIR_SUMS
+#define GQ_PAIR_SUMS 0
+#endif
+
+constexpr int kExpTableSize = 512;  // indexed by the top nine bits of a rounded level
+// Shared memory after the ring: 2 * stages mbarriers, a tile number per stage
+// (at most kMaxStages), then the exponential-level code table.
+constexpr int kMaxStages = 8;
+constexpr size_t kTmaTailBytes = 2 * kMaxStages * sizeof(unsigned long long) +
+                                 kMaxStages * sizeof(long long) +
+                                 (GQ_EXP_BYTE_TABLE ? 0 : kExpTableSize * sizeof(int));
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -119,17 +162,35 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         : "memory");
 }
 
+// Signed code of a rounded exponential level from its top nine bits h
+// (sign, biased exponent): the exponent field is the level index once the
+// finest level sits on 2^-126.  Fields past L (only reachable from a
+// non-finite input, which also raises the scale flag) give code 0.
+__device__ __forceinline__ int exp_table_entry(int h, int L) {
+    const int e = h & 255;
+    const int idx = e <= L ? e : 0;
+    return (h >> 8) ? -idx : idx;
+}
+
 // WT: the number of workers when known at compile time (the worker loop is
 // then fully unrolled and the Philox chains of all workers interleave), or 0.
 template <int LEVELS, int BITS, bool EF, int WT, bool BQ, bool WOFF>
 __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     quant_tma_kernel(const __grid_constant__ QuantArgs a, int stages) {
     extern __shared__ __align__(128) unsigned char smem[];
+    // per-bucket scales are prefetched one tile ahead in the static order
+    constexpr bool kDynamic = !BQ;
     const int W = WT > 0 ? WT : a.W;
     const int rows = EF ? 2 * W : W;  // g rows, then e rows
     float* buf = reinterpret_cast<float*>(smem);
     unsigned long long* bars = reinterpret_cast<unsigned long long*>(
         smem + (size_t)stages * rows * kTmaTile * sizeof(float));
+    long long* tile_of = reinterpret_cast<long long*>(bars + 2 * kMaxStages);
+#if GQ_EXP_BYTE_TABLE
+    __shared__ signed char code_table[kExpTableSize];
+#else
+    int* code_table = reinterpret_cast<int*>(tile_of + kMaxStages);
+#endif
     const uint32_t full0 = smem_addr(bars);
     const uint32_t empty0 = smem_addr(bars + stages);
 
@@ -144,22 +205,36 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (LEVELS != 0 && BITS != 0)
+        for (int h = threadIdx.x; h < kExpTableSize; h += kTmaThreads)
+            code_table[h] = exp_table_entry(h, a.L);  // |code| <= 15
     __syncthreads();
 
     if (warp == kTmaComputeWarps) {
         // ---------------- producer: one lane issues every copy ----------------
         if (lane == 0) {
-            // stage s of round `round` holds this CTA's tile number round * stages + s
+            // stage s of round `round` holds this CTA's k-th tile, k = round * stages + s
             int s = 0;
             uint32_t round = 0;
             long long issued = 0;
             bool ok = true;
-            for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++issued) {
+            long long t = kDynamic ? (long long)atomicAdd(&a.hdr->tile_next, 1u) : blockIdx.x;
+            for (;; ++issued) {
+                if (!kDynamic && t >= ntiles) break;
                 if (round > 0 && !mbar_wait_bounded(empty0 + 8 * s, (round - 1) & 1u, a.hdr)) {
                     ok = false;
                     break;
                 }
+                if (kDynamic && t >= ntiles) {  // no tile left: tell the compute warps
+                    tile_of[s] = -1;
+                    mbar_arrive(full0 + 8 * s);
+                    break;
+                }
                 const long long j0 = t * kTmaTile;
+                // claim the next tile now, so the atomic's round trip overlaps this one
+                const long long t_next =
+                    kDynamic ? (long long)atomicAdd(&a.hdr->tile_next, 1u) : t + gridDim.x;
+                tile_of[s] = t;
                 const long long n = a.d - j0 < kTmaTile ? a.d - j0 : kTmaTile;
                 const uint32_t bytes = (uint32_t)(n * sizeof(float));
                 mbar_arrive_expect_tx(full0 + 8 * s, bytes * (uint32_t)rows);
@@ -169,6 +244,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                     bulk_g2s(smem_addr(buf + ((size_t)s * rows + r) * kTmaTile), src, bytes,
                              full0 + 8 * s);
                 }
+                t = t_next;
                 if (++s == stages) {
                     s = 0;
                     ++round;
@@ -182,6 +258,15 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 for (long long k = first; k < issued; ++k)
                     mbar_wait_bounded(full0 + 8 * (int)(k % stages), (uint32_t)((k / stages) & 1),
                                       a.hdr);
+            }
+            if (kDynamic) {
+                // The last producer to finish claiming resets the counters for the
+                // next launch on this workspace (stream order publishes them).
+                __threadfence();
+                if (atomicAdd(&a.hdr->tile_done, 1u) == gridDim.x - 1) {
+                    atomicExch(&a.hdr->tile_next, 0u);
+                    atomicExch(&a.hdr->tile_done, 0u);
+                }
             }
         }
         return;
@@ -217,10 +302,15 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
             c_next = __ldg(a.bq_unit + (b0 >> a.bucket_shift));
         }
     }
-    for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    for (long long tt = blockIdx.x;; tt += gridDim.x) {
+        if (!kDynamic && tt >= ntiles) break;
         if (!mbar_wait_bounded(full0 + 8 * s, phase, a.hdr)) break;
+        const long long t = kDynamic ? tile_of[s] : tt;
+        if (t < 0) break;  // the producer found no tile left
         const long long blk = t * kTmaComputeWarps + warp;
-        if (blk < nblk) {
+        // FULL: every coordinate of the tile exists (no bounds checks)
+        auto block_body = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
             if (BQ) {  // per-bucket scale of this block
                 aq = aq_next;
                 c = c_next;
@@ -231,16 +321,18 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 }
             }
             const long long j0 = (blk << 7) + (lane << 2);
-            const bool in = j0 < a.d;  // d % 4 == 0: all four or none
+            const bool in = FULL || j0 < a.d;  // d % 4 == 0: all four or none
             // WOFF = 0: no worker or coordinate offset (the common case)
             const unsigned long long q =
                 (unsigned long long)(blk << 5) + (unsigned)lane + (WOFF ? a.q0 : 0ull);
             const float* stage = buf + (size_t)s * rows * kTmaTile + warp * 128 + lane * 4;
             unsigned char* codes_blk = a.codes + blk * (16 * BITS);
             // uniform levels accumulate the biased patterns (code + kCodeBias);
-            // exponential levels accumulate the level values as floats (exact:
-            // multiples of the finest level with fewer than 24 bits)
+            // exponential levels accumulate the rounded levels as floats in
+            // units of 2^-126 per finest level (exact: integers below 2^24
+            // times 2^-126, subnormal or not)
             uint32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+            uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;  // an even worker's patterns, held
             float f0 = 0.f, f1 = 0.f, f2 = 0.f, f3 = 0.f;
 #pragma unroll
             for (int w = 0; w < (WT > 0 ? WT : a.W); ++w) {
@@ -264,10 +356,23 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                     const float t3 = quant_uniform_biased_unclamped(v.w, aq, rnd.w);
                     const uint32_t b0 = __float_as_uint(t0), b1 = __float_as_uint(t1);
                     const uint32_t b2 = __float_as_uint(t2), b3 = __float_as_uint(t3);
-                    s0 += b0;
-                    s1 += b1;
-                    s2 += b2;
-                    s3 += b3;
+                    constexpr bool kPair = GQ_PAIR_SUMS && WT > 0 && WT % 2 == 0;
+                    if (kPair && (w & 1) == 0) {
+                        h0 = b0;
+                        h1 = b1;
+                        h2 = b2;
+                        h3 = b3;
+                    } else if (kPair) {
+                        s0 += h0 + b0;
+                        s1 += h1 + b1;
+                        s2 += h2 + b2;
+                        s3 += h3 + b3;
+                    } else {
+                        s0 += b0;
+                        s1 += b1;
+                        s2 += b2;
+                        s3 += b3;
+                    }
                     if (BITS != 0) pk.template store<kCodeBias>(lane, b0, b1, b2, b3, cdst);
                     if (EF) {
                         qv.x = __fsub_rn(t0, 12582912.0f);
@@ -276,22 +381,26 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                         qv.w = __fsub_rn(t3, 12582912.0f);
                     }
                 } else {
-                    const float q0 = quant_exp_level(v.x, aq, a.finest, rnd.x);
-                    const float q1 = quant_exp_level(v.y, aq, a.finest, rnd.y);
-                    const float q2 = quant_exp_level(v.z, aq, a.finest, rnd.z);
-                    const float q3 = quant_exp_level(v.w, aq, a.finest, rnd.w);
+                    const uint32_t y0 = exp_round_bits(v.x, aq, a.exp_shift, rnd.x);
+                    const uint32_t y1 = exp_round_bits(v.y, aq, a.exp_shift, rnd.y);
+                    const uint32_t y2 = exp_round_bits(v.z, aq, a.exp_shift, rnd.z);
+                    const uint32_t y3 = exp_round_bits(v.w, aq, a.exp_shift, rnd.w);
+                    const float q0 = __uint_as_float(y0 & 0xFF800000u);
+                    const float q1 = __uint_as_float(y1 & 0xFF800000u);
+                    const float q2 = __uint_as_float(y2 & 0xFF800000u);
+                    const float q3 = __uint_as_float(y3 & 0xFF800000u);
                     f0 = __fadd_rn(f0, q0);
                     f1 = __fadd_rn(f1, q1);
                     f2 = __fadd_rn(f2, q2);
                     f3 = __fadd_rn(f3, q3);
-                    if (BITS != 0)
-                        pk.store(lane, exp_code_of_level(q0, a.L), exp_code_of_level(q1, a.L),
-                                 exp_code_of_level(q2, a.L), exp_code_of_level(q3, a.L), cdst);
+                    if (BITS != 0)  // y >> 23 < 512: always inside the table
+                        pk.store(lane, code_table[y0 >> 23], code_table[y1 >> 23],
+                                 code_table[y2 >> 23], code_table[y3 >> 23], cdst);
                     if (EF) {  // value in units of the finest level (exact)
-                        qv.x = __fmul_rn(q0, a.inv_finest);
-                        qv.y = __fmul_rn(q1, a.inv_finest);
-                        qv.z = __fmul_rn(q2, a.inv_finest);
-                        qv.w = __fmul_rn(q3, a.inv_finest);
+                        qv.x = __fmul_rn(q0, 0x1p126f);
+                        qv.y = __fmul_rn(q1, 0x1p126f);
+                        qv.z = __fmul_rn(q2, 0x1p126f);
+                        qv.w = __fmul_rn(q3, 0x1p126f);
                     }
                 }
                 if (EF && a.update_e && in) {
@@ -310,21 +419,25 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 s2 -= off;
                 s3 -= off;
             } else {  // level-value sums to integer units of the finest level
-                s0 = (uint32_t)__float2int_rn(__fmul_rn(f0, a.inv_finest));
-                s1 = (uint32_t)__float2int_rn(__fmul_rn(f1, a.inv_finest));
-                s2 = (uint32_t)__float2int_rn(__fmul_rn(f2, a.inv_finest));
-                s3 = (uint32_t)__float2int_rn(__fmul_rn(f3, a.inv_finest));
+                s0 = (uint32_t)float_units_to_int(f0);
+                s1 = (uint32_t)float_units_to_int(f1);
+                s2 = (uint32_t)float_units_to_int(f2);
+                s3 = (uint32_t)float_units_to_int(f3);
             }
-            if (a.sum) store_sum(a.sum, a.wire, j0, a.d, (int)s0, (int)s1, (int)s2, (int)s3);
+            if (a.sum) store_sum<FULL>(a.sum, a.wire, j0, a.d, (int)s0, (int)s1, (int)s2, (int)s3);
             if (a.out) {
                 float4 o;
                 o.x = decode_mean((int)s0, c, a.inv_w, a.w_pow2, W);
                 o.y = decode_mean((int)s1, c, a.inv_w, a.w_pow2, W);
                 o.z = decode_mean((int)s2, c, a.inv_w, a.w_pow2, W);
                 o.w = decode_mean((int)s3, c, a.inv_w, a.w_pow2, W);
-                store_out4(a.out, j0, a.d, o);
+                store_out4<FULL>(a.out, j0, a.d, o);
             }
-        }
+        };
+        if (GQ_TMA_FULL_TILES && (t + 1) * kTmaTile <= a.d)
+            block_body(std::true_type{});
+        else if (blk < nblk)
+            block_body(std::false_type{});
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
         if (++s == stages) {
@@ -336,7 +449,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
 
 size_t tma_smem_bytes(int W, bool ef, int stages) {
     const int rows = ef ? 2 * W : W;
-    return (size_t)stages * rows * kTmaTile * sizeof(float) + 2 * stages * sizeof(unsigned long long);
+    return (size_t)stages * rows * kTmaTile * sizeof(float) + kTmaTailBytes;
 }
 
 template <int LEVELS, int BITS, bool EF, int WT, bool BQ, bool WOFF>
