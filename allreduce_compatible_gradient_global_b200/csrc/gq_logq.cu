@@ -8,9 +8,18 @@
 // Bins: sign + 127 magnitude steps of |q| in [0, 1], stochastic rounding.
 //
 // logq_quantize_kernel: one block per (matrix, worker); pass 1 reduces
-// max |x| over the matrix, pass 2 re-reads it (from L2: a factor is at most a
-// few hundred KB) and writes int8 codes.  logq_decode_kernel: Eq. (6) per
-// code and an fp32 sum over workers in ascending order.
+// max |x| over the matrix, pass 2 re-reads it (from L2, so DRAM sees one read:
+// a factor is at most a few hundred KB) and writes int8 codes.  Where the
+// matrix starts on a 16-byte boundary both passes move 16-byte vectors, four
+// consecutive entries, which are exactly one Philox block, and the codes
+// leave as 4-byte words; otherwise one entry at a time, same arithmetic.
+//
+// logq_decode_kernel: Eq. (6) and an fp32 sum over workers in ascending
+// order.  The inverse map of a magnitude step m, fl(expm1f(fl(fl(m/127) l))/a)
+// with l = log1pf(a), does not depend on the worker or the matrix, so each
+// block tabulates its values once in shared memory with exactly that
+// expression; a code then costs one table read and one multiply by the
+// matrix's max, bit for bit what evaluating Eq. (6) per code gives.
 #include <cfloat>
 
 #include "gq_internal.h"
@@ -32,6 +41,20 @@ __device__ __forceinline__ uint4 philox10_key(uint4 c, uint32_t k0, uint32_t k1)
     return c;
 }
 
+// One code: the magnitude step of |x| / M on the log map, stochastically
+// rounded with the uniform of `word`, and x's sign.
+__device__ __forceinline__ int logq_code(float xv, float M, bool usable, float alpha, float lam,
+                                         uint32_t word) {
+    int k = 0;
+    if (usable) {
+        const float xn = __fdiv_rn(fabsf(xv), M);
+        const float tq = __fdiv_rn(log1pf(__fmul_rn(alpha, xn)), lam);
+        const float y = fminf(__fmul_rn(tq, 127.0f), 127.0f);
+        k = floor_y_plus_u(y, unit_plus_u(word));
+    }
+    return with_sign_of(k, xv);
+}
+
 __global__ void __launch_bounds__(kLogqThreads) logq_quantize_kernel(const __grid_constant__ LogqArgs a) {
     const int mi = blockIdx.x;  // matrix within this launch
     const int w = blockIdx.y;
@@ -40,10 +63,31 @@ __global__ void __launch_bounds__(kLogqThreads) logq_quantize_kernel(const __gri
     const long long base = (long long)w * a.total + a.off[mi];
     const float* x = a.x + base;
     signed char* codes = a.codes + base;
+    // 16-byte vectors when the matrix's first entry and first code allow them
+    const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(codes) & 3u) == 0);
+    const long long n4 = vec ? n >> 2 : 0;  // whole 4-entry groups taken as vectors
 
-    unsigned mx = 0u;
-    for (long long i = threadIdx.x; i < n; i += kLogqThreads)
-        mx = max(mx, __float_as_uint(fabsf(__ldg(x + i))));
+    unsigned mx0 = 0u, mx1 = 0u;
+    {
+        const float4* x4 = reinterpret_cast<const float4*>(x);
+        long long q = threadIdx.x;
+        for (; q + kLogqThreads < n4; q += 2 * kLogqThreads) {  // two vectors in flight
+            const float4 u = __ldg(x4 + q), v = __ldg(x4 + q + kLogqThreads);
+            mx0 = max(mx0, max(max(__float_as_uint(fabsf(u.x)), __float_as_uint(fabsf(u.y))),
+                               max(__float_as_uint(fabsf(u.z)), __float_as_uint(fabsf(u.w)))));
+            mx1 = max(mx1, max(max(__float_as_uint(fabsf(v.x)), __float_as_uint(fabsf(v.y))),
+                               max(__float_as_uint(fabsf(v.z)), __float_as_uint(fabsf(v.w)))));
+        }
+        if (q < n4) {
+            const float4 u = __ldg(x4 + q);
+            mx0 = max(mx0, max(max(__float_as_uint(fabsf(u.x)), __float_as_uint(fabsf(u.y))),
+                               max(__float_as_uint(fabsf(u.z)), __float_as_uint(fabsf(u.w)))));
+        }
+        for (long long i = 4 * n4 + threadIdx.x; i < n; i += kLogqThreads)
+            mx1 = max(mx1, __float_as_uint(fabsf(__ldg(x + i))));
+    }
+    unsigned mx = max(mx0, mx1);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFull, mx, o));
     __shared__ unsigned red[kLogqThreads / 32];
@@ -61,47 +105,84 @@ __global__ void __launch_bounds__(kLogqThreads) logq_quantize_kernel(const __gri
     const float lam = log1pf(alpha);
     const uint32_t k0 = a.seed_lo, k1 = a.seed_hi ^ (0x4C510000u | (uint32_t)m);
     const uint32_t step = a.step_dev ? __ldg(a.step_dev) : a.step;
+    const uint32_t wid = a.worker0 + (uint32_t)w;
 
-    // four consecutive entries per thread share one Philox block
-    for (long long q = threadIdx.x; 4 * q < n; q += kLogqThreads) {
-        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, step, a.worker0 + (uint32_t)w), k0, k1);
+    // entries 4q..4q+3 share Philox block q
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    for (long long q = threadIdx.x; q < n4; q += kLogqThreads) {
+        const float4 v = x4[q];  // an L2 hit: pass 1 just read it
+        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
+        const int c0 = logq_code(v.x, M, usable, alpha, lam, rnd.x);
+        const int c1 = logq_code(v.y, M, usable, alpha, lam, rnd.y);
+        const int c2 = logq_code(v.z, M, usable, alpha, lam, rnd.z);
+        const int c3 = logq_code(v.w, M, usable, alpha, lam, rnd.w);
+        reinterpret_cast<uint32_t*>(codes)[q] =
+            (uint32_t)(c0 & 255) | ((uint32_t)(c1 & 255) << 8) | ((uint32_t)(c2 & 255) << 16) |
+            ((uint32_t)c3 << 24);
+    }
+    // the rest one entry at a time (all of it when the matrix is not aligned)
+    for (long long q = n4 + threadIdx.x; 4 * q < n; q += kLogqThreads) {
+        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
         const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const long long i = 4 * q + t;
-            if (i < n) {
-                const float xv = __ldg(x + i);
-                int k = 0;
-                if (usable) {
-                    const float xn = __fdiv_rn(fabsf(xv), M);
-                    const float tq = __fdiv_rn(log1pf(__fmul_rn(alpha, xn)), lam);
-                    const float y = fminf(__fmul_rn(tq, 127.0f), 127.0f);
-                    k = floor_y_plus_u(y, unit_plus_u(words[t]));
-                }
-                codes[i] = (signed char)with_sign_of(k, xv);
-            }
+            if (i < n)
+                codes[i] = (signed char)logq_code(__ldg(x + i), M, usable, alpha, lam, words[t]);
         }
     }
 }
 
+// The inverse map of magnitude step m (Eq. (6) without the max), m = 0..128
+// (128 only from a caller's code -128, which the quantizer never writes).
+__device__ __forceinline__ float logq_unit_value(int m, float alpha, float lam) {
+    const float z = __fmul_rn(__fdiv_rn((float)m, 127.0f), lam);
+    return __fdiv_rn(expm1f(z), alpha);
+}
+
+__device__ __forceinline__ float logq_decode_one(int k, float M, const float* tab) {
+    const float xm = __fmul_rn(tab[k < 0 ? -k : k], M);
+    return k < 0 ? -xm : xm;
+}
+
 __global__ void __launch_bounds__(kLogqThreads) logq_decode_kernel(const __grid_constant__ LogqArgs a) {
+    __shared__ float tab[129];  // every int8 magnitude, 0..128
+    const float alpha = a.alpha;
+    const float lam = log1pf(alpha);
+    if (threadIdx.x < 129) tab[threadIdx.x] = logq_unit_value((int)threadIdx.x, alpha, lam);
+    __syncthreads();
     const int mi = blockIdx.y;
     const int m = a.m0 + mi;
     const long long n = a.off[mi + 1] - a.off[mi];
-    const float alpha = a.alpha;
-    const float lam = log1pf(alpha);
-    for (long long i = (long long)blockIdx.x * kLogqThreads + threadIdx.x; i < n;
-         i += (long long)gridDim.x * kLogqThreads) {
+    const long long off = a.off[mi];
+    // 4-byte code words and 16-byte outputs when every row's slice allows them
+    const bool vec = ((off & 3) == 0) && ((a.total & 3) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(a.ccodes) & 3u) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(a.out) & 15u) == 0);
+    const long long n4 = vec ? n >> 2 : 0;
+    const long long stride = (long long)gridDim.x * kLogqThreads;
+    for (long long q = (long long)blockIdx.x * kLogqThreads + threadIdx.x; q < n4; q += stride) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int w = 0; w < a.W; ++w) {
+            const uint32_t c = __ldcs(reinterpret_cast<const unsigned int*>(
+                a.ccodes + (long long)w * a.total + off) + q);
+            const float M = __ldg(a.cmaxabs + (long long)w * a.nmats + m);
+            acc.x = __fadd_rn(acc.x, logq_decode_one((int)(signed char)(c & 255), M, tab));
+            acc.y = __fadd_rn(acc.y, logq_decode_one((int)(signed char)((c >> 8) & 255), M, tab));
+            acc.z = __fadd_rn(acc.z, logq_decode_one((int)(signed char)((c >> 16) & 255), M, tab));
+            acc.w = __fadd_rn(acc.w, logq_decode_one((int)(signed char)(c >> 24), M, tab));
+        }
+        __stcs(reinterpret_cast<float4*>(a.out + off) + q, acc);
+    }
+    for (long long i = 4 * n4 + (long long)blockIdx.x * kLogqThreads + threadIdx.x; i < n;
+         i += stride) {
         float acc = 0.f;
         for (int w = 0; w < a.W; ++w) {
-            const int k = a.ccodes[(long long)w * a.total + a.off[mi] + i];
+            const int k = a.ccodes[(long long)w * a.total + off + i];
             const float M = __ldg(a.cmaxabs + (long long)w * a.nmats + m);
-            const int mag = k < 0 ? -k : k;
-            const float z = __fmul_rn(__fdiv_rn((float)mag, 127.0f), lam);
-            const float xm = __fmul_rn(__fdiv_rn(expm1f(z), alpha), M);
-            acc = __fadd_rn(acc, k < 0 ? -xm : xm);
+            acc = __fadd_rn(acc, logq_decode_one(k, M, tab));
         }
-        a.out[a.off[mi] + i] = acc;
+        a.out[off + i] = acc;
     }
 }
 
@@ -114,7 +195,8 @@ cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st) {
 cudaError_t launch_logq_decode(const LogqArgs& a, cudaStream_t st) {
     long long maxn = 0;
     for (int i = 0; i < a.count; ++i) maxn = max(maxn, a.off[i + 1] - a.off[i]);
-    long long bx = (maxn + kLogqThreads - 1) / kLogqThreads;
+    // a thread takes 4 coordinates where the vectors apply, 1 elsewhere
+    long long bx = (maxn / 4 + kLogqThreads - 1) / kLogqThreads;
     if (bx < 1) bx = 1;
     if (bx > 64) bx = 64;
     dim3 grid((unsigned)bx, a.count);
