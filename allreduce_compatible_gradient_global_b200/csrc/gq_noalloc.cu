@@ -10,7 +10,16 @@
 // Host code cannot use the array's name as a device address (on the host it
 // is only a stand-in), so the first call on each device resolves the real
 // address with cudaGetSymbolAddress, with that device current, and caches it.
-// That first call should therefore come before any stream capture.
+// That first call should therefore come before any stream capture.  The
+// cached address belongs to the device's context: after cudaDeviceReset the
+// module is loaded again and the array may move, so this call must not be
+// used across a device reset.
+//
+// The block count per worker row is gq_global_norm's own (the fp32 runs and
+// the fp64 combine order depend on it), so the two calls return bit-identical
+// scales and norms.  It always fits the array: 2 W nb <= 2 * 8 blocks per SM
+// * the SM count, far below kNoallocSlots on any current GPU, and it is
+// clamped to the array in any case.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -49,19 +58,11 @@ int scratch_address(void** out) {
     return GQ_OK;
 }
 
-// Blocks per worker: about 8 resident blocks per SM in all, within the
-// scratch's partial slots.
-int noalloc_blocks_per_worker(int W, long long d) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-            sms = n;
-    }
-    long long nb = ((long long)sms * 8 + W - 1) / W;
-    const long long useful = (d + (long long)gq::kThreads * 16 - 1) / ((long long)gq::kThreads * 16);
-    if (useful < nb) nb = useful;
-    if (nb > kNoallocSlots / (2 * W)) nb = kNoallocSlots / (2 * W);  // two slots per block
+// Blocks per worker: those of gq_global_norm, within the array's partial
+// slots (two per block).
+int noalloc_blocks_per_worker(int W, long long d, int kind, bool has_e) {
+    long long nb = gq::norm_blocks_per_worker(W, d, kind, has_e);
+    if (nb > kNoallocSlots / (2 * W)) nb = kNoallocSlots / (2 * W);
     if (nb < 1) nb = 1;
     return (int)nb;
 }
@@ -93,7 +94,7 @@ extern "C" GQ_API int gq_global_norm_noalloc(const float* g_dev, const float* e_
     a.e = cfg->ef ? e_dev : nullptr;
     a.d = d;
     a.W = W;
-    a.nb = noalloc_blocks_per_worker(W, d);
+    a.nb = noalloc_blocks_per_worker(W, d, cfg->scale_kind, cfg->ef != 0);
     a.kind = cfg->scale_kind;
     a.scale = scale_dev;
     a.norms = norms_dev;

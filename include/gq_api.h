@@ -190,18 +190,23 @@ GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long lo
  * allocator, or a fixed arena that forbids outside allocations), or a hot path
  * that cannot afford cudaMalloc's cost and its implicit device-wide
  * synchronization.  This call computes exactly what gq_global_norm computes
- * (same kernel, same arguments minus the workspace) but keeps its block
- * partials and ticket counter in a fixed device array inside the library:
- * 256 + 8192 * 8 bytes, held by every GPU that loads the library until the
- * process exits.  It allocates nothing and calls no allocating routine.
+ * (same kernel, same block count, bit-identical scale and norms) but keeps
+ * its block partials and ticket counter in a fixed device array inside the
+ * library: 256 + 8192 * 8 bytes, held by every GPU that loads the library
+ * until the process exits.  It allocates nothing and calls no allocating
+ * routine.
  *
- * Limits: W <= 4096, else GQ_ERR_SIZE (nothing is launched).  The first call
- * on each device looks up the array's device address (cudaGetSymbolAddress,
- * with that device current) and caches it, so make that first call before
- * any stream capture.  All calls share the one array: each call clears its
- * counter and flag word on `stream` before launching, and calls that overlap
- * on the GPU (other streams, other threads) race on it.  A NaN or Inf input
- * shows as a non-finite scale_dev[0]; this call has no flag word to read. */
+ * Limits: W <= 4096, else GQ_ERR_SIZE (nothing is launched).  As in
+ * gq_global_norm, above about 8 workers per SM each worker row is reduced by
+ * a single 256-thread block, so very large W runs well below bandwidth.  The
+ * first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it, so make
+ * that first call before any stream capture, and do not use the call across
+ * cudaDeviceReset (the array may move when the module is loaded again).  All
+ * calls share the one array: each call clears its counter and flag word on
+ * `stream` before launching, and calls that overlap on the GPU (other
+ * streams, other threads) race on it.  A NaN or Inf input shows as a
+ * non-finite scale_dev[0]; this call has no flag word to read. */
 GQ_API int gq_global_norm_noalloc(const float* g_dev, const float* e_dev, int W, long long d,
                                   const gq_config* cfg, float* scale_dev, double* norms_dev,
                                   cudaStream_t stream);

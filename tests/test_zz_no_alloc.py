@@ -3,11 +3,20 @@ allocate device memory (another allocator owns the device, or the path cannot
 afford cudaMalloc and its device-wide synchronization).  It keeps its partial
 sums in a fixed array inside the library instead of a caller workspace.
 
-Checked through the C ABI against the ordinary gq_global_norm, on two calls
-in a row (the shared scratch keeps the previous call's contents, so the
-second call shows that each call starts clean).  Tolerance: the one the other
-scale tests use -- 1e-5 relative for the L2 norm, exact for max-abs.  This
-file is collected last, so a run that stops at the first failure has run
+Checked through the C ABI on two calls in a row (the second finds the shared
+scratch as the first left it):
+
+* against the ordinary gq_global_norm bit for bit -- both run the same kernel
+  with the same block count, so the scale and the per-worker norms agree
+  exactly;
+* against the oracle's fp64 norm (the tolerance the other scale tests use:
+  1e-5 relative for L2, exact for max-abs), so a drift of the shared norm
+  kernel away from the oracle fails here too;
+* and that the second call changes neither the device's free memory nor
+  torch's allocated bytes (the first call may load the module and resolve the
+  array's address).
+
+This file is collected last, so a run that stops at the first failure has run
 every other test before it.
 """
 import ctypes
@@ -51,7 +60,7 @@ def call_noalloc(gq, g, e, cfg, scale, norms):
     (1, 4096, "maxabs", True),
     (64, 5000, "l2", False),
 ])
-def test_noalloc_matches_workspace_form(gq, W, d, kind, ef):
+def test_noalloc_matches_workspace_form_and_oracle(gq, oracle, W, d, kind, ef):
     cfg = gq.GQConfig(s=15, bits=5, wire="int8", scale_kind=kind, ef=ef)
     g = synthetic.make_gradients(W, d, "student_t3", seed=W + d, device="cuda", seg=4096,
                                  lo=-4, hi=0)
@@ -60,18 +69,27 @@ def test_noalloc_matches_workspace_form(gq, W, d, kind, ef):
     gq.gq_global_norm(g, e, cfg, ref.scale, ref.norms, ref.ws)
     torch.cuda.synchronize()
     S_ref, n_ref = ref.scale.item(), ref.norms.cpu().numpy()
+    S_ora, n_ora = oracle.global_scale(g.cpu().numpy(), None if e is None else e.cpu().numpy(),
+                                       0 if kind == "l2" else 1)
     for call in range(2):
         scale = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
         norms = torch.full((W,), -1.0, dtype=torch.float64, device="cuda")
+        torch.cuda.synchronize()
+        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         assert call_noalloc(gq, g, e, cfg, scale, norms) == gq.GQ_OK
         torch.cuda.synchronize()
+        if call == 1:  # the first call may load the module; the second allocates nothing
+            assert torch.cuda.mem_get_info()[0] == free0
+            assert torch.cuda.memory_allocated() == alloc0
         S, n = scale.item(), norms.cpu().numpy()
+        assert S == S_ref, (call, S, S_ref)
+        assert np.array_equal(n.view(np.uint64), n_ref.view(np.uint64)), call
         if kind == "l2":
-            assert abs(S - S_ref) <= SCALE_RTOL * S_ref, (call, S, S_ref)
-            assert np.allclose(n, n_ref, rtol=SCALE_RTOL, atol=0), call
+            assert abs(S - float(S_ora)) <= SCALE_RTOL * float(S_ora), (call, S, S_ora)
+            assert np.allclose(n, n_ora, rtol=SCALE_RTOL, atol=0), call
         else:
-            assert S == S_ref, (call, S, S_ref)
-            assert np.array_equal(n, n_ref), call
+            assert S == S_ora, (call, S, S_ora)
+            assert np.array_equal(n, n_ora), call
 
 
 def test_noalloc_rejects_sizes_beyond_its_maximum(gq):
