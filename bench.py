@@ -1,27 +1,39 @@
 """Benchmark of the quantize + aggregate path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-cpu-baseline] [--no-e2e]
+                    [--workload NAME] [--no-cpu-baseline] [--no-e2e] [--no-extras]
 
 One step = one pass of the whole path over one batch of W synthetic worker
-gradients already resident in HBM: gq_global_norm (read 1) then
-gq_quantize_aggregate (read 2: Philox uniforms, stochastic rounding, packed
-codes at wire width, integer sum over workers, decoded mean).  These two calls
-are exactly what gq_step_fused issues; the benchmark makes them separately so
-that, in a second pass of K steps, CUDA events can bracket each kernel.  The
-job's own time comes from K steps with events around the run only.
+gradients resident in HBM: gq_global_norm (read 1) then gq_quantize_aggregate
+(read 2: Philox uniforms, stochastic rounding, packed codes at wire width,
+integer sum over workers, decoded mean, error feedback).  These two calls are
+exactly what gq_step_fused issues; the benchmark makes them separately so that
+CUDA events can bracket each kernel.
+
+The default workload is the largest one-GPU configuration: W = 8 workers of
+d = 2^30 coordinates, per-2^20-segment sigma_k * N(0,1) gradients, uniform
+levels s = 127, 8-bit codes, int16 sums, error feedback.  Every step draws a
+fresh gradient (the step enters the seed) while the error buffers carry over.
+Each step is timed by its own CUDA events around the two kernels; the next
+step's gradient is drawn between the timed spans.  A step moves ~174 GiB of
+algorithmic bytes, so the events cost nothing measurable, and the 32 GiB
+gradient far exceeds L2.  Other workloads (--workload) have fixed gradients:
+K steps back to back with events around the run only, and the per-kernel
+launch times from K further steps with an event around each kernel (an event
+between two kernels drains the GPU at the boundary).
 
 Metric: fp32 gradient GB/s = 4 * W * d bytes / step time (whole job: summed
 over ranks under torchrun, each rank an independent replica, timed as the max
-over ranks).  Prints one JSON line on rank 0.  The line also carries the step
-without materialised codes, the roofline of the dominant kernel, an end-to-end
-figure through host buffers, and the CPU oracle single- and multi-threaded.
+over ranks).  Prints one JSON line on rank 0 with the roofline of the dominant
+kernel, an end-to-end figure through host buffers (gq_step_fused_host), the CPU
+oracle single- and multi-threaded, and, at one GPU, the other workloads under
+"configs" (value, roofline and CPU oracle for each).
 
 Other modes print their own JSON line: --sweep (d = 2^16..2^30, EF off/on,
-eager and graph-replayed), --buckets (per-bucket scales), --lq (the log
-quantizer), --lqsgd (the PowerSGD + LQ step), --nat (natural compression),
---dp (the real exchange under torchrun, eager and graph-replayed, against an
-fp32 all-reduce).
+eager and graph-replayed, oracle beside each row), --buckets (per-bucket
+scales), --lq (the log quantizer), --lqsgd (the PowerSGD + LQ step), --nat
+(natural compression), --dp (the real exchange under torchrun, eager and
+graph-replayed, against an fp32 all-reduce).
 
 --impl reference times the CPU oracle (the plain restatement of the method
 used by the tests) on the host cores, on a bounded sample of the same
@@ -32,7 +44,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -47,7 +58,12 @@ import torch  # noqa: E402
 import synthetic  # noqa: E402
 
 METRIC = "quantize+aggregate fp32-gradient GB/s at 1 B200; % of HBM roofline"
-DEFAULT_WORKLOAD = "resnet50_t3_w8"
+DEFAULT_WORKLOAD = "normal_seg_d2^30_w8_ef"
+# the other configurations, reported under "configs" in the one-GPU line
+EXTRA_WORKLOADS = ("normal_d2^20_w4", "resnet50_t3_w8", "gpt2s_laplace_w8", "gpt2s_laplace_w8_l2")
+# host oracle samples: a prefix of this many coordinates (None: the whole workload)
+CPU_SAMPLE_COORDS = {"normal_seg_d2^30_w8_ef": 1 << 26, "gpt2s_laplace_w8": 1 << 24,
+                     "gpt2s_laplace_w8_l2": 1 << 24}
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "quant_kernel_traffic.json")
@@ -55,14 +71,21 @@ KERNEL_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_quant_tma.c
                   "allreduce_compatible_gradient_global_b200/csrc/gq_kernels.cu",
                   "allreduce_compatible_gradient_global_b200/csrc/gq_device.cuh",
                   "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h"]
+LOGQ_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_logq.cu",
+                "allreduce_compatible_gradient_global_b200/csrc/gq_device.cuh",
+                "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h"]
 
 
-def kernel_source_hash():
+def source_hash(files=KERNEL_SOURCES):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in files:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def kernel_source_hash():
+    return source_hash(KERNEL_SOURCES)
 
 
 def measured_hbm_peak():
@@ -75,9 +98,11 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per launch of the dominant kernel from a committed ncu
-    summary, if it was taken on the current kernel source; else None."""
+def recorded_traffic(workload, d):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None.  A
+    capture of a smaller case of the same recipe (captured_d coordinates) is
+    scaled to d: every byte the kernel moves is proportional to d."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
@@ -86,7 +111,9 @@ def recorded_traffic(workload):
     if rec.get("source_hash") != kernel_source_hash():
         return None
     ent = rec.get("workloads", {}).get(workload)
-    return None if ent is None else float(ent["dram_bytes_per_launch"])
+    if ent is None:
+        return None
+    return float(ent["dram_bytes_per_launch"]) * d / float(ent.get("captured_d", d))
 
 
 # ----------------------------------------------------------------------- clocks
@@ -169,8 +196,16 @@ def workload_config(gq, name):
     return wl, cfg
 
 
+def oracle_kwargs(wl):
+    return dict(levels=0 if wl["levels"] == "uniform" else 1, s=wl.get("s", 15),
+                L=wl.get("L", 8), scale_kind=0 if wl["scale"] == "l2" else 1, bits=wl["bits"],
+                seed=0x5EED)
+
+
 def algorithmic_bytes(gq, cfg, W, d):
-    """(pass-1 bytes, pass-2 bytes) per step: what each kernel must move."""
+    """(pass-1 bytes, pass-2 bytes) per step: what each kernel must move.
+    Pass 1 reads g (and e); pass 2 reads g (and e), writes the packed codes,
+    the integer sum and the mean (and e)."""
     wire = 1 if cfg.wire == "int8" else 2
     p1 = 4 * W * d + (4 * W * d if cfg.ef else 0)
     p2 = (4 * W * d + W * gq.gq_packed_row_bytes(cfg, d) + wire * d + 4 * d
@@ -192,165 +227,242 @@ def job_gbs(bytes_per_rank_step, steps, job_ms, world):
     return world * bytes_per_rank_step * steps / (job_ms * 1e-3) / 1e9
 
 
+def _sync(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def _events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+class Workload:
+    """A workload's gradients and step buffers on the device, and its step."""
+
+    def __init__(self, gq, name, dev, d=None):
+        self.gq, self.name = gq, name
+        self.wl, self.cfg = workload_config(gq, name)
+        self.W, self.d = self.wl["W"], (d or self.wl["d"])
+        self.fresh = bool(self.wl.get("fresh_per_step", False))
+        self.dev = dev
+        self.g = synthetic.workload_gradients(name, device=dev, d=self.d)
+        self.buf = gq.StepBuffers(self.cfg, self.W, self.d, device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.drawn = 0  # the step whose gradient g holds
+
+    def draw(self, i):
+        """The gradient of step i (fresh-per-step workloads only)."""
+        if self.fresh and i != self.drawn:
+            synthetic.workload_gradients(self.name, device=self.dev, step=i, out=self.g,
+                                         d=self.d)
+            self.drawn = i
+
+    def step(self, i, ev=None, codes=True):
+        gq, cfg, buf, st = self.gq, self.cfg, self.buf, self.stream
+        cfg.step = i
+        if ev is not None:
+            ev[0].record(st)
+        gq.gq_global_norm(self.g, buf.e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws,
+                          st)
+        if ev is not None:
+            ev[1].record(st)
+        gq.gq_quantize_aggregate(self.g, buf.e, cfg, buf.scale, buf.codes if codes else None,
+                                 buf.sum, buf.out, buf.ws, st)
+        if ev is not None:
+            ev[2].record(st)
+
+    def check(self, what):
+        if self.gq.gq_get_device_status(self.buf.ws, self.stream) != self.gq.GQ_OK:
+            raise RuntimeError(f"device flag raised in {what} ({self.name})")
+
+    def free(self):
+        del self.g, self.buf
+        torch.cuda.empty_cache()
+
+
+def time_workload(wk, K, warmup, world, flush=None):
+    """Times K steps of a workload.  Returns (job ms over the K steps, per-step
+    norm ms, per-step fused ms, timing note).  Fresh-per-step workloads and
+    those given `flush` (run untimed between steps) are timed step by step;
+    the others run K steps back to back, then K more with per-kernel events."""
+    dev = wk.dev
+    between = None
+    if wk.fresh:
+        def between(i):
+            wk.draw(i)
+    elif flush is not None:
+        def between(i):
+            flush()
+    for i in range(warmup):
+        if between is not None:
+            between(i)
+        wk.step(i)
+    wk.check("warm-up")
+    if between is not None:
+        evs = [_events(3) for _ in range(K)]
+        _sync(world)
+        for i in range(K):
+            between(warmup + i)
+            wk.step(warmup + i, evs[i])
+        _sync(world)
+        spans = [e[0].elapsed_time(e[2]) for e in evs]
+        job_ms = job_time_ms(sum(spans), world, dev)
+        note = ("each step timed by CUDA events around its two kernels; "
+                + ("the next step's fresh gradient is drawn between the timed spans"
+                   if wk.fresh else "L2 flushed between the timed spans"))
+    else:
+        t0, t1 = _events(2)
+        _sync(world)
+        t0.record(wk.stream)
+        for i in range(K):
+            wk.step(warmup + i)
+        t1.record(wk.stream)
+        _sync(world)
+        job_ms = job_time_ms(t0.elapsed_time(t1), world, dev)
+        evs = [_events(3) for _ in range(K)]
+        for i in range(K):
+            wk.step(warmup + K + i, evs[i])
+        torch.cuda.synchronize()
+        note = ("value, ms_per_step: K steps back to back, CUDA events around the whole run "
+                "only; roofline avg_launch_ms: K further steps with events around each kernel")
+    wk.check("timed steps")
+    norm_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    quant_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    return job_ms, norm_ms, quant_ms, note
+
+
+def roofline_of(gq, wk, job_ms, K, norm_ms, quant_ms, with_traffic):
+    W, d, cfg = wk.W, wk.d, wk.cfg
+    p1, p2 = algorithmic_bytes(gq, cfg, W, d)
+    ms_per_step = job_ms / K
+    q_avg = sum(quant_ms) / len(quant_ms)
+    n_avg = sum(norm_ms) / len(norm_ms)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = p2 / (q_avg * 1e-3) / 1e9
+    traffic = recorded_traffic(wk.name, d) if with_traffic else None
+    return {"bound": "hbm", "kernel": "fused pass of gq_quantize_aggregate "
+                                      "(quant_tma_kernel when d % 4 == 0 and the rows fit)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} (hbm_gbs)",
+            "traffic": None if traffic is None else round(traffic),
+            "algorithmic_bytes": p2, "avg_launch_ms": round(q_avg, 5),
+            "norm_kernel": {"achieved": round(p1 / (n_avg * 1e-3) / 1e9, 1),
+                            "frac": round(p1 / (n_avg * 1e-3) / 1e9 / peak, 4),
+                            "algorithmic_bytes": p1, "avg_launch_ms": round(n_avg, 5)},
+            "step": {"achieved": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9, 1),
+                     "frac": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+                     "frac_of_8000": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / 8000, 4)}}
+
+
+def l2_flusher(dev):
+    """Writes a buffer twice the size of L2, evicting whatever the last step left."""
+    junk = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        junk.fill_(1.0)
+    return flush
+
+
 def run_ours(args, rank, world, local_rank):
     import allreduce_compatible_gradient_global_b200 as gq
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl, cfg = workload_config(gq, args.workload)
-    W, d = wl["W"], (args.coords or wl["d"])
-    g = synthetic.workload_gradients(args.workload, device=dev, d=d)
-    buf = gq.StepBuffers(cfg, W, d, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step(i, ev=None, codes=True):
-        cfg.step = i
-        if ev is not None:
-            ev[0].record(stream)
-        gq.gq_global_norm(g, buf.e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws, stream)
-        if ev is not None:
-            ev[1].record(stream)
-        gq.gq_quantize_aggregate(g, buf.e, cfg, buf.scale, buf.codes if codes else None, buf.sum,
-                                 buf.out, buf.ws, stream)
-        if ev is not None:
-            ev[2].record(stream)
-
-    for i in range(args.warmup):
-        step(i)
-        step(i, codes=False)  # the instantiation without codes, timed below too
-    if gq.gq_get_device_status(buf.ws, stream) != gq.GQ_OK:
-        raise RuntimeError("non-finite scale in warm-up")
+    wk = Workload(gq, args.workload, dev, d=args.coords)
+    W, d, cfg = wk.W, wk.d, wk.cfg
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    sampler = ClockSampler(local_rank)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    # The job: K steps with nothing recorded between the kernels (an event
-    # between two kernels drains the GPU at the boundary; three per step cost
-    # ~9 us of a 0.35 ms step).
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(K):
-        step(args.warmup + i)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    elapsed_ms = job_time_ms(t0.elapsed_time(t1), world, dev)
-    # Per-kernel launch times for the roofline: K further steps with an event
-    # before, between and after the two kernels.
-    for i in range(K):
-        step(args.warmup + K + i, evs[i])
-    torch.cuda.synchronize()
-    # The fused pass without materialised codes (the sum-based exchange needs
-    # none): K more steps, events around the run only.
-    n0 = torch.cuda.Event(enable_timing=True)
-    n1 = torch.cuda.Event(enable_timing=True)
-    n0.record(stream)
-    for i in range(K):
-        step(args.warmup + 2 * K + i, codes=False)
-    n1.record(stream)
-    torch.cuda.synchronize()
-    sampler.stop()
-    if world > 1:
-        torch.distributed.barrier()
-    nc_ms = job_time_ms(n0.elapsed_time(n1), world, dev)
-    norm_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    quant_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    ms_per_step = elapsed_ms / K
     grad_bytes = 4 * W * d
-    value = job_gbs(grad_bytes, K, elapsed_ms, world)
-
-    # roofline of the dominant kernel (pass 2)
+    flush = l2_flusher(dev) if grad_bytes < 2 * L2_BYTES else None
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    job_ms, norm_ms, quant_ms, note = time_workload(wk, K, args.warmup, world, flush)
+    # the fused pass without materialised codes (the sum-based exchange needs none)
+    Knc = K if not wk.fresh else min(K, 5)
+    n0, n1 = _events(2)
+    _sync(world)
+    n0.record(wk.stream)
+    for i in range(Knc):
+        wk.step(args.warmup + 2 * K + i, codes=False)
+    n1.record(wk.stream)
+    _sync(world)
+    sampler.stop()
+    nc_ms = job_time_ms(n0.elapsed_time(n1), world, dev)
+    ms_per_step = job_ms / K
+    value = job_gbs(grad_bytes, K, job_ms, world)
+    roofline = roofline_of(gq, wk, job_ms, K, norm_ms, quant_ms, with_traffic=not args.coords)
     p1, p2 = algorithmic_bytes(gq, cfg, W, d)
-    q_avg = sum(quant_ms) / K
-    n_avg = sum(norm_ms) / K
-    peak, peak_kind = measured_hbm_peak()
-    achieved = p2 / (q_avg * 1e-3) / 1e9
-    traffic = None if args.coords else recorded_traffic(args.workload)
-    roofline = {"bound": "hbm", "kernel": "fused pass of gq_quantize_aggregate "
-                                          "(quant_tma_kernel when d % 4 == 0 and the rows fit)",
-                "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} (hbm_gbs)",
-                "traffic": traffic, "algorithmic_bytes": p2,
-                "avg_launch_ms": round(q_avg, 5),
-                "norm_kernel": {"achieved": round(p1 / (n_avg * 1e-3) / 1e9, 1),
-                                "frac": round(p1 / (n_avg * 1e-3) / 1e9 / peak, 4),
-                                "algorithmic_bytes": p1, "avg_launch_ms": round(n_avg, 5)},
-                "step": {"achieved": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9, 1),
-                         "frac": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
-                         "frac_of_8000": round((p1 + p2) / (ms_per_step * 1e-3) / 1e9 / 8000, 4)}}
-
+    peak = roofline["peak"]
     p2_nc = p2 - W * gq.gq_packed_row_bytes(cfg, d)
-    without_codes = {"value": round(job_gbs(grad_bytes, K, nc_ms, world), 2), "unit": "GB/s",
-                     "ms_per_step": round(nc_ms / K, 5), "algorithmic_bytes": p1 + p2_nc,
-                     "step_frac": round((p1 + p2_nc) / (nc_ms / K * 1e-3) / 1e9 / peak, 4)}
-
-    e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(gq, args, cfg, g, buf, stream, world, dev)
+    without_codes = {"value": round(job_gbs(grad_bytes, Knc, nc_ms, world), 2), "unit": "GB/s",
+                     "ms_per_step": round(nc_ms / Knc, 5), "steps": Knc,
+                     "algorithmic_bytes": p1 + p2_nc,
+                     "step_frac": round((p1 + p2_nc) / (nc_ms / Knc * 1e-3) / 1e9 / peak, 4)}
+    e2e = None if args.no_e2e else run_e2e(gq, args, wk, world, dev)
+    data = {"normal_seg_d2^30_w8_ef": "synthetic (seeded per-2^20-segment sigma_k*N(0,1) "
+                                      "gradients, a fresh draw every step)",
+            "resnet50_t3_w8": "synthetic (seeded per-segment Student-t(3) gradients, "
+                              "ResNet-50-sized)"}.get(args.workload, "synthetic")
     result = dict(
         metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=K,
         warmup=args.warmup, ms_per_step=round(ms_per_step, 5), higher_is_better=True,
-        scaling="weak", vs_baseline=None, dtype="f32",
-        data="synthetic (seeded per-segment Student-t(3) gradients, ResNet-50-sized)"
-        if args.workload == DEFAULT_WORKLOAD else "synthetic",
+        scaling="weak", vs_baseline=None, dtype="f32", data=data,
         config={"workload": args.workload, "W": W, "d": d, "levels": cfg.levels, "s": cfg.s,
                 "L": cfg.L, "bits": cfg.bits, "wire": cfg.wire, "scale": cfg.scale_kind,
-                "ef": cfg.ef, "parallelism": f"replicas x{world}",
-                "truncated_to_coords": args.coords,
-                "l2": f"inputs exceed L2: {grad_bytes / 1e6:.1f} MB of gradient per read "
-                      f"vs {L2_BYTES / 1e6:.0f} MB L2"},
+                "ef": cfg.ef, "fresh_gradient_per_step": wk.fresh,
+                "parallelism": f"replicas x{world}", "truncated_to_coords": args.coords,
+                "l2": (f"inputs exceed L2: {grad_bytes / 1e6:.1f} MB of gradient per read vs "
+                       f"{L2_BYTES / 1e6:.0f} MB L2") if flush is None else
+                      "L2 flushed between timed steps (a 2x-L2 buffer written)"},
         roofline=roofline, gpu_launches=2 * K, clocks=sampler.summary(), e2e=e2e,
-        timing="value, ms_per_step: K steps, CUDA events around the whole run only; "
-               "roofline avg_launch_ms: K further steps with CUDA events around each kernel",
-        fused_without_codes=without_codes)
-    del g, buf
-    torch.cuda.empty_cache()
+        timing=note, fused_without_codes=without_codes)
+    wk.free()
     return result
 
 
-def run_e2e(gq, args, cfg, g, buf, stream, world, dev):
+def run_e2e(gq, args, wk, world, dev):
     """Same metric through gq_step_fused_host: every step copies its gradients
     host->device from pinned memory, runs both kernels and reads the decoded
-    mean and the scale back.  Consecutive steps alternate between two buffer
-    sets on two streams, as a training loop that double-buffers its gradient
-    uploads would, so one step's upload overlaps the previous step's compute
-    and read-back."""
-    W, d = g.shape
-    g_host = g.cpu().pin_memory()
-    streams = [stream, torch.cuda.Stream(device=dev)]
+    mean and the scale back.  When two buffer sets fit the device, steps
+    alternate between them on two streams (as a training loop that
+    double-buffers its uploads would: one step's upload overlaps the previous
+    step's compute and read-back); otherwise one set, one stream, and the
+    upload lands in the workload's own gradient buffer."""
+    W, d, cfg, g = wk.W, wk.d, wk.cfg, wk.g
+    g_host = torch.empty((W, d), dtype=torch.float32, pin_memory=True)
+    g_host.copy_(g)
+    set_bytes = 4 * W * d * (2 if cfg.ef else 1) + W * gq.gq_packed_row_bytes(cfg, d) + 8 * d
+    free_b, _ = torch.cuda.mem_get_info(dev)
+    two = free_b > 1.2 * (set_bytes + 4 * W * d) and 4 * W * d < (8 << 30)
+    streams = [wk.stream] + ([torch.cuda.Stream(device=dev)] if two else [])
     sets = []
-    for k in range(2):
-        b = buf if k == 0 else gq.StepBuffers(cfg, W, d, device=dev)
-        sets.append(dict(buf=b, g_dev=torch.empty_like(g),
-                         out_host=torch.empty(d, dtype=torch.float32).pin_memory(),
-                         scale_host=torch.empty(1, dtype=torch.float32).pin_memory()))
-    K = args.steps
+    for k in range(len(streams)):
+        b = wk.buf if k == 0 else gq.StepBuffers(cfg, W, d, device=dev)
+        sets.append(dict(buf=b, g_dev=g if not two else torch.empty_like(g),
+                         out_host=torch.empty(d, dtype=torch.float32, pin_memory=True),
+                         scale_host=torch.empty(1, dtype=torch.float32, pin_memory=True)))
+    K = args.steps if two else max(1, min(args.steps, 3))
 
     def one(i):
-        sset, st = sets[i % 2], streams[i % 2]
+        n = len(sets)
+        sset, st = sets[i % n], streams[i % n]
         b = sset["buf"]
         cfg.step = 1000 + i
         gq.gq_step_fused_host(g_host, sset["g_dev"], b.e, cfg, b.scale, b.codes, b.sum, b.out,
                               sset["out_host"], sset["scale_host"], b.ws, st)
 
-    for i in range(min(args.warmup, 4)):
+    for i in range(min(args.warmup, 4) if two else 1):
         one(i)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
+    _sync(world)
+    t0, t1 = _events(2)
     t0.record(streams[0])
-    streams[1].wait_event(t0)
+    for s2 in streams[1:]:
+        s2.wait_event(t0)
     for i in range(K):
         one(i)
-    done = torch.cuda.Event()
-    done.record(streams[1])
-    streams[0].wait_event(done)
+    for s2 in streams[1:]:
+        done = torch.cuda.Event()
+        done.record(s2)
+        streams[0].wait_event(done)
     t1.record(streams[0])
     torch.cuda.synchronize()
     ms = job_time_ms(t0.elapsed_time(t1), world, dev)
@@ -360,39 +472,68 @@ def run_e2e(gq, args, cfg, g, buf, stream, world, dev):
             raise RuntimeError("device flag raised in the end-to-end run")
     del g_host, sets
     return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
-            "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4),
-            "api": "gq_step_fused_host, two streams alternating buffer sets"}
+            "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4), "steps": K,
+            "api": ("gq_step_fused_host, two streams alternating buffer sets" if two else
+                    "gq_step_fused_host, one buffer set on one stream (two sets do not fit)")}
 
 
-def cpu_baseline(args, sample_coords=None):
-    """The oracle as it stands (single-threaded C) on a sample of the workload."""
-    import oracle
-    wl = synthetic.WORKLOADS[args.workload]
+def host_threads():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else \
+        (os.cpu_count() or 1)
+
+
+_CPU_SAMPLE = {}
+
+
+def cpu_sample(name, sample_coords):
+    """The host sample of a workload (drawn once, shared by both CPU figures)."""
+    wl = synthetic.WORKLOADS[name]
     W, d = wl["W"], wl["d"]
     n = d if sample_coords is None else min(d, sample_coords)
-    g = synthetic.workload_gradients(args.workload, device="cpu", d=n).numpy()
-    kw = dict(levels=0 if wl["levels"] == "uniform" else 1, s=wl.get("s", 15), L=wl.get("L", 8),
-              scale_kind=0 if wl["scale"] == "l2" else 1, bits=wl["bits"], seed=0x5EED)
+    key = (name, n)
+    if key not in _CPU_SAMPLE:
+        _CPU_SAMPLE.clear()
+        g = synthetic.workload_gradients(name, device="cpu", d=n).numpy()
+        e = np.zeros_like(g) if wl["ef"] else None
+        _CPU_SAMPLE[key] = (g, e)
+    g, e = _CPU_SAMPLE[key]
+    return wl, W, d, n, g, e
+
+
+def _sample_words(name, W, d, n, dt, extra=""):
+    whole = n == d
+    txt = (f"one oracle step (scale, codes, pack, sum, decode{', error feedback' if extra else ''})"
+           f" on W={W} x {n} coordinates of the {name} recipe")
+    if whole:
+        return txt + f" (the full workload), {dt:.1f} s"
+    return (txt + f" (a prefix; the per-coordinate cost does not depend on d, so the GB/s "
+                  f"figure is extrapolated to the full d={d}), {dt:.1f} s")
+
+
+def cpu_baseline(name, sample_coords=None):
+    """The oracle as it stands (single-threaded C) on a sample of the workload."""
+    import oracle
+    wl, W, d, n, g, e = cpu_sample(name, sample_coords)
+    kw = oracle_kwargs(wl)
     oracle.lib()
     t = time.perf_counter()
-    oracle.step(g, **kw)
+    oracle.step(g, e, ef=wl["ef"], **kw)
     dt = time.perf_counter() - t
     return {"value": round(4 * W * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"one oracle step (scale, codes, pack, sum, decode) on W={W} x "
-                      f"{n} coordinates of the {args.workload} recipe "
-                      f"({'the full workload' if n == d else 'a prefix'}), {dt:.1f} s"}
+            "kind": "oracle", "extrapolated": n != d,
+            "sample": _sample_words(name, W, d, n, dt, "ef" if wl["ef"] else "")}
 
 
-def oracle_step_threaded(g, threads, *, levels, s, L, scale_kind, bits, seed, step=0):
+def oracle_step_threaded(g, threads, e=None, *, levels, s, L, scale_kind, bits, seed, step=0):
     """The oracle's step on `threads` host threads, for the threaded CPU figure.
     The oracle's scale is per worker (an fp64 sum in ascending coordinate order
     within a row, or the row's max |v|), so the rows run in parallel and S is
     the max of their scales.  With S fixed, every code depends only on its own
     coordinate (the uniforms are counter-based), so coordinate chunks of whole
     128-coordinate packing blocks are quantized at their own indices, packed,
-    summed and decoded independently.  The oracle's C routines release the GIL
-    while they run.  Returns S, the packed rows, the integer sums and the mean."""
+    summed, decoded and (with e) error-fed independently.  The oracle's C
+    routines release the GIL while they run.  Returns S, the packed rows, the
+    integer sums, the mean and the new error rows (None without e)."""
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     W, d = g.shape
@@ -401,67 +542,190 @@ def oracle_step_threaded(g, threads, *, levels, s, L, scale_kind, bits, seed, st
     bounds = [(c0, min(d, c0 + step_c)) for c0 in range(0, d, step_c)]
 
     def row_scale(w):
-        return oracle.global_scale(g[w:w + 1], None, scale_kind)[0]
+        return oracle.global_scale(g[w:w + 1], None if e is None else e[w:w + 1], scale_kind)[0]
 
     with ThreadPoolExecutor(max_workers=threads) as pool:
         S = np.float32(max(pool.map(row_scale, range(W))))
 
         def chunk(b):
             c0, c1 = b
-            codes = oracle.quantize(g[:, c0:c1], None, levels=levels, s=s, L=L, seed=seed,
-                                    step=step, S=S, js=np.arange(c0, c1, dtype=np.int64))
+            gs = g[:, c0:c1]
+            es = None if e is None else e[:, c0:c1]
+            codes = oracle.quantize(gs, es, levels=levels, s=s, L=L, seed=seed, step=step, S=S,
+                                    js=np.arange(c0, c1, dtype=np.int64))
             packed = oracle.pack(codes, bits) if bits else None
             total = oracle.aggregate(codes, levels=levels, L=L)
-            return packed, total, oracle.decode_mean(total, W, levels=levels, s=s, L=L, S=S)
+            mean = oracle.decode_mean(total, W, levels=levels, s=s, L=L, S=S)
+            e_new = None if e is None else oracle.error_feedback(gs, es, codes, levels=levels,
+                                                                 s=s, L=L, S=S)
+            return packed, total, mean, e_new
 
         parts = list(pool.map(chunk, bounds))
     packed = np.concatenate([x[0] for x in parts], axis=1) if bits else None
+    e_new = None if e is None else np.concatenate([x[3] for x in parts], axis=1)
     return dict(S=S, packed=packed, sum=np.concatenate([x[1] for x in parts]),
-                out=np.concatenate([x[2] for x in parts]))
+                out=np.concatenate([x[2] for x in parts]), e=e_new)
 
 
-def cpu_baseline_threads(args):
+def cpu_baseline_threads(name, sample_coords=None):
     """The same oracle step run coordinate-parallel over every host core the
     process may use (oracle_step_threaded): a second, fairer CPU figure."""
     import oracle
-    wl = synthetic.WORKLOADS[args.workload]
-    W, d = wl["W"], wl["d"]
-    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else \
-        (os.cpu_count() or 1)
-    g = synthetic.workload_gradients(args.workload, device="cpu").numpy()
+    wl, W, d, n, g, e = cpu_sample(name, sample_coords)
+    kw = oracle_kwargs(wl)
+    threads = host_threads()
     oracle.lib()
     t = time.perf_counter()
-    oracle_step_threaded(g, threads, levels=0 if wl["levels"] == "uniform" else 1,
-                         s=wl.get("s", 15), L=wl.get("L", 8),
-                         scale_kind=0 if wl["scale"] == "l2" else 1, bits=wl["bits"],
-                         seed=0x5EED)
+    oracle_step_threaded(g, threads, e, **kw)
     dt = time.perf_counter() - t
-    return {"value": round(4 * W * d / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": f"oracle x{threads} threads",
-            "sample": f"one oracle step on W={W} x {d} coordinates of the {args.workload} "
-                      f"recipe (the full workload), rows then coordinate chunks over "
-                      f"{threads} threads, {dt:.1f} s"}
+    return {"value": round(4 * W * n / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": f"oracle x{threads} threads", "extrapolated": n != d,
+            "sample": _sample_words(name, W, d, n, dt, "ef" if wl["ef"] else "")
+            + f"; rows then coordinate chunks over {threads} threads"}
 
 
+# ------------------------------------------------------- the other configurations
+def measure_config(gq, name, K, warmup, dev, with_cpu):
+    """value, roofline and CPU oracle of one fixed-gradient workload (one GPU)."""
+    wk = Workload(gq, name, dev)
+    flush = l2_flusher(dev) if 4 * wk.W * wk.d < 2 * L2_BYTES else None
+    job_ms, norm_ms, quant_ms, note = time_workload(wk, K, warmup, 1, flush)
+    roof = roofline_of(gq, wk, job_ms, K, norm_ms, quant_ms, with_traffic=True)
+    cfg = wk.cfg
+    res = {"value": round(job_gbs(4 * wk.W * wk.d, K, job_ms, 1), 2), "unit": "GB/s",
+           "ms_per_step": round(job_ms / K, 5), "steps": K, "W": wk.W, "d": wk.d,
+           "levels": cfg.levels, "s": cfg.s, "L": cfg.L, "bits": cfg.bits, "wire": cfg.wire,
+           "scale": cfg.scale_kind, "ef": cfg.ef, "roofline": roof, "timing": note,
+           "gpu_launches": 2 * K}
+    wk.free()
+    if with_cpu:
+        res["cpu_baseline"] = cpu_baseline(name, CPU_SAMPLE_COORDS.get(name))
+    return res
+
+
+def lq_bytes(W, n, nmats):
+    """Algorithmic bytes of the log quantizer on W workers x n factor entries
+    (nmats matrices per worker): the quantize pass reads the factors once and
+    writes int8 codes and the per-matrix max; the decode-sum reads the codes
+    and the max and writes the fp32 sum."""
+    q = 4 * W * n + W * n + 4 * W * nmats
+    dsum = W * n + 4 * W * nmats + 4 * n
+    return q, dsum
+
+
+def measure_lq(gq, r, K, dev, with_cpu):
+    """The log quantizer on W = 8 workers x 24 factor pairs of 4096 x r:
+    quantize + decode-sum per step, each timed by events, L2 flushed between
+    steps (the factors fit in L2)."""
+    W = synthetic.LQ_WORKLOAD["W"]
+    alpha = synthetic.LQ_WORKLOAD["alpha"]
+    x, sizes = synthetic.lq_factors(r, W=W, device=dev)
+    n = x.shape[1]
+    nm = len(sizes)
+    R = [4096] * nm
+    C = [r] * nm
+    cfg = gq.GQConfig(levels="log", alpha=alpha, seed=1)
+    mx = torch.empty((W, nm), dtype=torch.float32, device=dev)
+    codes = torch.empty((W, n), dtype=torch.int8, device=dev)
+    out = torch.empty(n, dtype=torch.float32, device=dev)
+    ws = torch.empty(gq.gq_workspace_bytes(gq.GQConfig(), W, 1), dtype=torch.uint8, device=dev)
+    gq.gq_workspace_init(ws)
+    flush = l2_flusher(dev)
+    st = torch.cuda.current_stream()
+    evs = [_events(3) for _ in range(K + 3)]
+    for i in range(K + 3):
+        flush()
+        cfg.step = i
+        evs[i][0].record(st)
+        gq.gq_logq_quantize(x, R, C, cfg, mx, codes, ws, st)
+        evs[i][1].record(st)
+        gq.gq_logq_decode_sum(codes, mx, R, C, cfg, out, st)
+        evs[i][2].record(st)
+    torch.cuda.synchronize()
+    if gq.gq_get_device_status(ws, st) != gq.GQ_OK:
+        raise RuntimeError("device flag raised in the log-quantizer run")
+    qm = sum(e[0].elapsed_time(e[1]) for e in evs[3:]) / K
+    dm = sum(e[1].elapsed_time(e[2]) for e in evs[3:]) / K
+    step_ms = qm + dm
+    qb, db = lq_bytes(W, n, nm)
+    peak, peak_kind = measured_hbm_peak()
+    res = {"value": round(4 * W * n / (step_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "ms_per_step": round(step_ms, 5), "steps": K, "rank": r, "W": W,
+           "elements_per_worker": n, "matrices_per_worker": nm,
+           "roofline": {"bound": "hbm", "kernel": "logq_quantize_kernel",
+                        "achieved": round(qb / (qm * 1e-3) / 1e9, 1), "peak": peak,
+                        "unit": "GB/s", "frac": round(qb / (qm * 1e-3) / 1e9 / peak, 4),
+                        "peak_source": f"{peak_kind} (hbm_gbs)", "traffic": None,
+                        "algorithmic_bytes": qb, "avg_launch_ms": round(qm, 5),
+                        "decode_sum_kernel": {
+                            "achieved": round(db / (dm * 1e-3) / 1e9, 1),
+                            "frac": round(db / (dm * 1e-3) / 1e9 / peak, 4),
+                            "algorithmic_bytes": db, "avg_launch_ms": round(dm, 5)},
+                        "step": {"achieved": round((qb + db) / (step_ms * 1e-3) / 1e9, 1),
+                                 "frac": round((qb + db) / (step_ms * 1e-3) / 1e9 / peak, 4)}},
+           "timing": "each step's two kernels timed by CUDA events; L2 flushed between steps",
+           "code_bytes_per_worker": n, "fp32_bytes_per_worker": 4 * n}
+    if with_cpu:
+        res["cpu_baseline"] = cpu_baseline_lq(x.cpu().numpy(), sizes, alpha)
+    del x, mx, codes, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline_lq(x, sizes, alpha):
+    import oracle
+    W, n = x.shape
+    oracle.lib()
+    t = time.perf_counter()
+    mx, codes = oracle.logq_quantize(x, sizes, alpha=alpha, seed=1, step=0)
+    oracle.logq_decode_sum(codes, mx, sizes, alpha=alpha)
+    dt = time.perf_counter() - t
+    return {"value": round(4 * W * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "extrapolated": False,
+            "sample": f"one oracle log-quantize + decode-sum of all W={W} x {n} factor "
+                      f"entries (the full workload), {dt:.2f} s"}
+
+
+def run_extras(args, dev):
+    import allreduce_compatible_gradient_global_b200 as gq
+    K = max(10, min(args.steps, 50))
+    out = {}
+    for name in EXTRA_WORKLOADS:
+        out[name] = measure_config(gq, name, K, args.warmup, dev, not args.no_cpu_baseline)
+    for r in synthetic.LQ_WORKLOAD["ranks"]:
+        out[f"lq_r{r}_w8"] = measure_lq(gq, r, K, dev, not args.no_cpu_baseline)
+    return out
+
+
+# --------------------------------------------------------------- reference arm
 def run_reference(args):
-    """Reference arm: the CPU oracle, each step a bounded sample."""
+    """Reference arm: the CPU oracle, each step a bounded sample of the
+    workload (a prefix of reference_coords coordinates, a fresh draw every step
+    when the workload has one, error buffers carried over)."""
     import oracle
     wl = synthetic.WORKLOADS[args.workload]
     W, d = wl["W"], wl["d"]
     n = min(d, args.reference_coords)
+    fresh = bool(wl.get("fresh_per_step", False))
+    kw = oracle_kwargs(wl)
     g = synthetic.workload_gradients(args.workload, device="cpu", d=n).numpy()
-    kw = dict(levels=0 if wl["levels"] == "uniform" else 1, s=wl.get("s", 15), L=wl.get("L", 8),
-              scale_kind=0 if wl["scale"] == "l2" else 1, bits=wl["bits"], seed=0x5EED)
+    e = np.zeros_like(g) if wl["ef"] else None
     oracle.lib()
-    for i in range(args.warmup):
-        oracle.step(g, step=i, **kw)
-    t = time.perf_counter()
-    for i in range(args.steps):
-        oracle.step(g, step=args.warmup + i, **kw)
-    dt = time.perf_counter() - t
+    dt = 0.0
+    for i in range(args.warmup + args.steps):
+        if fresh and i > 0:
+            g = synthetic.workload_gradients(args.workload, device="cpu", d=n, step=i).numpy()
+        t = time.perf_counter()
+        res = oracle.step(g, e, step=i, ef=wl["ef"], **kw)
+        if i >= args.warmup:
+            dt += time.perf_counter() - t
+        if wl["ef"]:
+            e = res["e"]
     value = 4 * W * n * args.steps / dt / 1e9
     sample = (f"each step: one oracle step on W={W} x {n} coordinates (a prefix of the "
-              f"{args.workload} recipe, d={d})")
+              f"{args.workload} recipe, d={d}"
+              + (", a fresh draw every step, error buffers carried over" if fresh else "")
+              + "; the prefix's draw is untimed)")
     return dict(metric=METRIC, value=round(value, 4), unit="GB/s", n_gpus=args.gpus,
                 steps=args.steps, warmup=args.warmup, ms_per_step=round(dt / args.steps * 1e3, 3),
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f32",
@@ -471,6 +735,24 @@ def run_reference(args):
                               "kind": "oracle", "sample": sample},
                 e2e={"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                      "d2h_bytes_per_step": 0})
+
+
+# ------------------------------------------------------------------ other modes
+SWEEP_ORACLE_COORDS = 1 << 20
+
+
+def sweep_oracle(g, ef):
+    """The oracle's step on a prefix of a sweep row's gradient (CPU, one thread)."""
+    import oracle
+    W, d = g.shape
+    n = min(d, SWEEP_ORACLE_COORDS)
+    gh = g[:, :n].cpu().numpy()
+    eh = np.zeros_like(gh) if ef else None
+    oracle.lib()
+    t = time.perf_counter()
+    oracle.step(gh, eh, levels=0, s=15, scale_kind=0, seed=0x5EED, ef=ef, bits=5)
+    dt = time.perf_counter() - t
+    return {"value": round(4 * W * n / dt / 1e9, 4), "unit": "GB/s", "coords": n}
 
 
 def time_step_pair(gq, g, e, cfg, buf, K, warmup, stream):
@@ -564,7 +846,8 @@ def run_sweep(args):
             n_ms, q_ms, step_ms = time_step_pair(gq, g, buf.e, cfg, buf, K, 5, stream)
             graph_ms = time_step_graph(gq, g, cfg, W, d, K)
             p1, p2 = algorithmic_bytes(gq, cfg, W, d)
-            rows.append({"d": d, "log2_d": lg, "ef": ef, "steps": K,
+            ora = None if args.no_cpu_baseline else sweep_oracle(g, ef)
+            rows.append({"d": d, "log2_d": lg, "ef": ef, "steps": K, "oracle": ora,
                          "step_ms": round(step_ms, 5), "norm_ms": round(n_ms, 5),
                          "quant_ms": round(q_ms, 5),
                          "grad_gbs": round(4 * W * d / (step_ms * 1e-3) / 1e9, 1),
@@ -576,6 +859,11 @@ def run_sweep(args):
             torch.cuda.empty_cache()
     return {"metric": METRIC, "mode": "sweep", "unit": "GB/s", "peak": peak,
             "peak_source": peak_kind, "W": W, "config": "uniform s=15, 5-bit, int8 sum, L2",
+            "oracle": None if args.no_cpu_baseline else
+            {"kind": "oracle", "cores": 1,
+             "sample": f"each row: one oracle step on a prefix of min(d, {SWEEP_ORACLE_COORDS}) "
+                       "coordinates of the row's gradient (all 8 workers), single-threaded; "
+                       "GB/s of fp32 gradient"},
             "sweep": rows}
 
 
@@ -872,46 +1160,15 @@ def run_nat(args):
 
 def run_lq(args):
     """The LQ-SGD log quantizer: quantize + decode-sum of 24 factor pairs of
-    4096 x r per worker, W = 8, r in {1, 4, 7}."""
+    4096 x r per worker, W = 8, r in {1, 4, 7}, with the roofline of both
+    kernels and the oracle on the same factors."""
     import allreduce_compatible_gradient_global_b200 as gq
     torch.cuda.set_device(0)
-    stream = torch.cuda.current_stream()
-    W = synthetic.LQ_WORKLOAD["W"]
-    rows = []
-    for r in synthetic.LQ_WORKLOAD["ranks"]:
-        x, sizes = synthetic.lq_factors(r, W=W, device="cuda")
-        n = x.shape[1]
-        R = [4096] * len(sizes)
-        C = [r] * len(sizes)
-        cfg = gq.GQConfig(levels="log", alpha=synthetic.LQ_WORKLOAD["alpha"], seed=1)
-        mx = torch.empty((W, len(sizes)), dtype=torch.float32, device="cuda")
-        codes = torch.empty((W, n), dtype=torch.int8, device="cuda")
-        out = torch.empty(n, dtype=torch.float32, device="cuda")
-        ws = torch.empty(gq.gq_workspace_bytes(gq.GQConfig(), W, 1), dtype=torch.uint8,
-                         device="cuda")
-        gq.gq_workspace_init(ws)
-        K = 200
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K + 5)]
-        for i in range(K + 5):
-            cfg.step = i
-            evs[i][0].record(stream)
-            gq.gq_logq_quantize(x, R, C, cfg, mx, codes, ws, stream)
-            evs[i][1].record(stream)
-            gq.gq_logq_decode_sum(codes, mx, R, C, cfg, out, stream)
-            evs[i][2].record(stream)
-        torch.cuda.synchronize()
-        qm = statistics.median(e[0].elapsed_time(e[1]) for e in evs[5:])
-        dm = statistics.median(e[1].elapsed_time(e[2]) for e in evs[5:])
-        # algorithmic bytes: two reads of the factors + int8 codes; codes + fp32 out
-        qb = 8 * W * n + W * n
-        db = W * n + 4 * n
-        rows.append({"rank": r, "elements_per_worker": n, "quantize_ms": round(qm, 5),
-                     "decode_sum_ms": round(dm, 5),
-                     "quantize_gbs": round(qb / (qm * 1e-3) / 1e9, 1),
-                     "decode_sum_gbs": round(db / (dm * 1e-3) / 1e9, 1),
-                     "code_bytes_per_worker": n, "fp32_bytes_per_worker": 4 * n})
-    return {"metric": "LQ-SGD log quantizer: factor GB/s", "mode": "lq", "unit": "GB/s",
-            "W": W, "rows": rows}
+    dev = torch.device("cuda", 0)
+    rows = [measure_lq(gq, r, max(10, args.steps), dev, not args.no_cpu_baseline)
+            for r in synthetic.LQ_WORKLOAD["ranks"]]
+    return {"metric": "LQ-SGD log quantizer: fp32 factor GB/s", "mode": "lq", "unit": "GB/s",
+            "W": synthetic.LQ_WORKLOAD["W"], "rows": rows}
 
 
 def _free_port():
@@ -924,12 +1181,14 @@ def _free_port():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations (the \"configs\" key of the line)")
     ap.add_argument("--reference-coords", type=int, default=1 << 21)
     ap.add_argument("--coords", type=int, default=None,
                     help="truncate the workload to this many coordinates (a smaller case "
@@ -997,10 +1256,13 @@ def main():
     try:
         result = run_ours(args, rank, world, local_rank)
         if rank == 0:
-            result["cpu_baseline"] = None if (args.no_cpu_baseline or world > 1) \
-                else cpu_baseline(args)
-            result["cpu_baseline_threads"] = None if (args.no_cpu_baseline or world > 1) \
-                else cpu_baseline_threads(args)
+            cpu = not (args.no_cpu_baseline or world > 1)
+            sample = None if args.coords else CPU_SAMPLE_COORDS.get(args.workload)
+            result["cpu_baseline"] = cpu_baseline(args.workload, sample) if cpu else None
+            result["cpu_baseline_threads"] = \
+                cpu_baseline_threads(args.workload, sample) if cpu else None
+            if world == 1 and not args.no_extras and not args.coords:
+                result["configs"] = run_extras(args, torch.device("cuda", local_rank))
             print(json.dumps(result), flush=True)
     finally:
         if world > 1:

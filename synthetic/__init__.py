@@ -36,10 +36,15 @@ WORKLOADS = {
     "gpt2s_laplace_w8": dict(W=8, d=124_439_808, recipe="laplace", seg=1 << 16,
                              lo=-5.0, hi=-2.0, levels="exp", L=8, bits=5,
                              wire="int16", scale="maxabs", ef=False, seed_index=2),
+    # the same gradients with the L2 global scale (the second scale variant)
+    "gpt2s_laplace_w8_l2": dict(W=8, d=124_439_808, recipe="laplace", seg=1 << 16,
+                                lo=-5.0, hi=-2.0, levels="exp", L=8, bits=5,
+                                wire="int16", scale="l2", ef=False, seed_index=2),
+    # a fresh draw every step (the step enters the seed), error feedback carried over
     "normal_seg_d2^30_w8_ef": dict(W=8, d=1 << 30, recipe="normal_seg", seg=1 << 20,
                                    lo=-4.0, hi=0.0, levels="uniform", s=127, bits=8,
                                    wire="int16", scale="l2", ef=True, steps=5,
-                                   seed_index=3),
+                                   fresh_per_step=True, seed_index=3),
 }
 
 # LQ-SGD factor workload: per worker, `pairs` factor pairs P (n x r), Q (m x r).
