@@ -63,14 +63,12 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 #ifndef GQ_EXP_BYTE_TABLE
 #define GQ_EXP_BYTE_TABLE 1
 #endif
-// 1: whole tiles take a copy of the block body without bounds checks.
+// 1: whole tiles take a copy of the block body without bounds checks (3-5%
+// faster on the GPT-2-sized and 8 x 2^26 workloads, even elsewhere).  Not with
+// error feedback: that pass is bound by HBM, measured no gain, and the second
+// copy of its body would spill within two blocks' registers.
 #ifndef GQ_TMA_FULL_TILES
-#define GQ_TMA_FULL_TILES 0
-#endif
-// 1: with the worker count fixed at compile time, uniform-level patterns of
-// two workers enter the sums in one three-input add.
-#ifndef GQ_PAIR_SUMS
-#define GQ_PAIR_SUMS 0
+#define GQ_TMA_FULL_TILES 1
 #endif
 
 constexpr int kExpTableSize = 512;  // indexed by the top nine bits of a rounded level
@@ -332,7 +330,6 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
             // units of 2^-126 per finest level (exact: integers below 2^24
             // times 2^-126, subnormal or not)
             uint32_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-            uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;  // an even worker's patterns, held
             float f0 = 0.f, f1 = 0.f, f2 = 0.f, f3 = 0.f;
 #pragma unroll
             for (int w = 0; w < (WT > 0 ? WT : a.W); ++w) {
@@ -356,23 +353,10 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                     const float t3 = quant_uniform_biased_unclamped(v.w, aq, rnd.w);
                     const uint32_t b0 = __float_as_uint(t0), b1 = __float_as_uint(t1);
                     const uint32_t b2 = __float_as_uint(t2), b3 = __float_as_uint(t3);
-                    constexpr bool kPair = GQ_PAIR_SUMS && WT > 0 && WT % 2 == 0;
-                    if (kPair && (w & 1) == 0) {
-                        h0 = b0;
-                        h1 = b1;
-                        h2 = b2;
-                        h3 = b3;
-                    } else if (kPair) {
-                        s0 += h0 + b0;
-                        s1 += h1 + b1;
-                        s2 += h2 + b2;
-                        s3 += h3 + b3;
-                    } else {
-                        s0 += b0;
-                        s1 += b1;
-                        s2 += b2;
-                        s3 += b3;
-                    }
+                    s0 += b0;
+                    s1 += b1;
+                    s2 += b2;
+                    s3 += b3;
                     if (BITS != 0) pk.template store<kCodeBias>(lane, b0, b1, b2, b3, cdst);
                     if (EF) {
                         qv.x = __fsub_rn(t0, 12582912.0f);
@@ -434,7 +418,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 store_out4<FULL>(a.out, j0, a.d, o);
             }
         };
-        if (GQ_TMA_FULL_TILES && (t + 1) * kTmaTile <= a.d)
+        if (GQ_TMA_FULL_TILES && !EF && (t + 1) * kTmaTile <= a.d)
             block_body(std::true_type{});
         else if (blk < nblk)
             block_body(std::false_type{});
