@@ -21,12 +21,43 @@
 // expression; a code then costs one table read and one multiply by the
 // matrix's max, bit for bit what evaluating Eq. (6) per code gives.
 #include <cfloat>
+#include <type_traits>
 
 #include "gq_internal.h"
 
 namespace gq {
 
 constexpr int kLogqThreads = 512;
+
+// 1: the two divisions of the log map (by the matrix's max and by log1p(a))
+// as a product with the divisor's reciprocal plus one fused correction;
+// 0: IEEE division.
+#ifndef GQ_LOGQ_FMA_DIV
+#define GQ_LOGQ_FMA_DIV 1
+#endif
+
+// a / b for 0 <= a <= b, given rb = RN(1/b) and lo = fma_div_floor(b):
+// q0 = RN(a rb) is within an ulp of a/b, the remainder r = a - q0 b is exact
+// in one fused multiply-add, and RN(q0 + r rb) is the correctly rounded
+// quotient (Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Develop. 34(1), 1990) -- provided
+// neither the reciprocal, the remainder nor the correction underflows.
+// Dividends below lo (a quotient or a dividend under 2^-100, or any dividend
+// of a divisor from 2^125 up, whose reciprocal is subnormal) therefore take
+// IEEE division.  Measured equal to IEEE division on 1.7e10 sampled quotients
+// in that domain over 255 divisors from 2^-110 to 2^110, edge mantissas and
+// log1p(10) among them; outside it the correction alone missed on 0.6% of
+// samples, and for the divisor FLT_MAX on 7 in 6.7e7.
+__device__ __forceinline__ float fma_div_floor(float b) {
+    return b < 0x1p125f ? 0x1p-100f * fmaxf(1.0f, b) : __int_as_float(0x7F800000);  // +inf
+}
+
+__device__ __forceinline__ float div_by_reciprocal(float a, float b, float rb, float lo) {
+    if (a < lo) return __fdiv_rn(a, b);
+    const float q0 = __fmul_rn(a, rb);
+    const float r = __fmaf_rn(-q0, b, a);
+    return __fmaf_rn(r, rb, q0);
+}
 
 __device__ __forceinline__ uint4 philox10_key(uint4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
@@ -42,20 +73,28 @@ __device__ __forceinline__ uint4 philox10_key(uint4 c, uint32_t k0, uint32_t k1)
 }
 
 // One code: the magnitude step of |x| / M on the log map, stochastically
-// rounded with the uniform of `word`, and x's sign.
+// rounded with the uniform of `word`, and x's sign.  FAST: the divisions use
+// the reciprocals rM, rlam (and IEEE division below loM, lolam).
+template <bool FAST>
 __device__ __forceinline__ int logq_code(float xv, float M, bool usable, float alpha, float lam,
+                                         float rM, float rlam, float loM, float lolam,
                                          uint32_t word) {
     int k = 0;
     if (usable) {
-        const float xn = __fdiv_rn(fabsf(xv), M);
-        const float tq = __fdiv_rn(log1pf(__fmul_rn(alpha, xn)), lam);
+        const float ax = fabsf(xv);
+        const float xn = FAST ? div_by_reciprocal(ax, M, rM, loM) : __fdiv_rn(ax, M);
+        const float lg = log1pf(__fmul_rn(alpha, xn));
+        const float tq = FAST ? div_by_reciprocal(lg, lam, rlam, lolam) : __fdiv_rn(lg, lam);
         const float y = fminf(__fmul_rn(tq, 127.0f), 127.0f);
         k = floor_y_plus_u(y, unit_plus_u(word));
     }
     return with_sign_of(k, xv);
 }
 
-__global__ void __launch_bounds__(kLogqThreads) logq_quantize_kernel(const __grid_constant__ LogqArgs a) {
+// Three 512-thread blocks per SM (40 registers): 384 (worker, matrix) blocks
+// of the LQ-SGD workload then run in one wave.
+__global__ void __launch_bounds__(kLogqThreads, 3)
+    logq_quantize_kernel(const __grid_constant__ LogqArgs a) {
     const int mi = blockIdx.x;  // matrix within this launch
     const int w = blockIdx.y;
     const int m = a.m0 + mi;
@@ -106,31 +145,48 @@ __global__ void __launch_bounds__(kLogqThreads) logq_quantize_kernel(const __gri
     const uint32_t k0 = a.seed_lo, k1 = a.seed_hi ^ (0x4C510000u | (uint32_t)m);
     const uint32_t step = a.step_dev ? __ldg(a.step_dev) : a.step;
     const uint32_t wid = a.worker0 + (uint32_t)w;
+    const float rM = __frcp_rn(M), rlam = __frcp_rn(lam);
+    const float loM = fma_div_floor(M), lolam = fma_div_floor(lam);
 
-    // entries 4q..4q+3 share Philox block q
-    const float4* x4 = reinterpret_cast<const float4*>(x);
-    for (long long q = threadIdx.x; q < n4; q += kLogqThreads) {
-        const float4 v = x4[q];  // an L2 hit: pass 1 just read it
-        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
-        const int c0 = logq_code(v.x, M, usable, alpha, lam, rnd.x);
-        const int c1 = logq_code(v.y, M, usable, alpha, lam, rnd.y);
-        const int c2 = logq_code(v.z, M, usable, alpha, lam, rnd.z);
-        const int c3 = logq_code(v.w, M, usable, alpha, lam, rnd.w);
-        reinterpret_cast<uint32_t*>(codes)[q] =
-            (uint32_t)(c0 & 255) | ((uint32_t)(c1 & 255) << 8) | ((uint32_t)(c2 & 255) << 16) |
-            ((uint32_t)c3 << 24);
-    }
-    // the rest one entry at a time (all of it when the matrix is not aligned)
-    for (long long q = n4 + threadIdx.x; 4 * q < n; q += kLogqThreads) {
-        const uint4 rnd = philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
-        const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const long long i = 4 * q + t;
-            if (i < n)
-                codes[i] = (signed char)logq_code(__ldg(x + i), M, usable, alpha, lam, words[t]);
+    auto quantize_pass = [&](auto fast_tag) {
+        constexpr bool FAST = decltype(fast_tag)::value;
+        // entries 4q..4q+3 share Philox block q
+        const float4* x4 = reinterpret_cast<const float4*>(x);
+        for (long long q = threadIdx.x; q < n4; q += kLogqThreads) {
+            const float4 v = x4[q];  // an L2 hit: pass 1 just read it
+            const uint4 rnd =
+                philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
+            const int c0 =
+                logq_code<FAST>(v.x, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.x);
+            const int c1 =
+                logq_code<FAST>(v.y, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.y);
+            const int c2 =
+                logq_code<FAST>(v.z, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.z);
+            const int c3 =
+                logq_code<FAST>(v.w, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.w);
+            reinterpret_cast<uint32_t*>(codes)[q] = (uint32_t)(c0 & 255) |
+                                                   ((uint32_t)(c1 & 255) << 8) |
+                                                   ((uint32_t)(c2 & 255) << 16) |
+                                                   ((uint32_t)c3 << 24);
         }
-    }
+        // the rest one entry at a time (all of it when the matrix is not aligned)
+        for (long long q = n4 + threadIdx.x; 4 * q < n; q += kLogqThreads) {
+            const uint4 rnd =
+                philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
+            const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const long long i = 4 * q + t;
+                if (i < n)
+                    codes[i] = (signed char)logq_code<FAST>(__ldg(x + i), M, usable, alpha, lam,
+                                                            rM, rlam, loM, lolam, words[t]);
+            }
+        }
+    };
+    if (GQ_LOGQ_FMA_DIV)
+        quantize_pass(std::true_type{});
+    else
+        quantize_pass(std::false_type{});
 }
 
 // The inverse map of magnitude step m (Eq. (6) without the max), m = 0..128
@@ -195,7 +251,9 @@ cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st) {
 cudaError_t launch_logq_decode(const LogqArgs& a, cudaStream_t st) {
     long long maxn = 0;
     for (int i = 0; i < a.count; ++i) maxn = max(maxn, a.off[i + 1] - a.off[i]);
-    // a thread takes 4 coordinates where the vectors apply, 1 elsewhere
+    // a thread takes 4 coordinates where the vectors apply, 1 elsewhere (two
+    // groups per thread, so that the grid fits one wave, measured slower:
+    // 16.4 against 13.3 us at rank 7)
     long long bx = (maxn / 4 + kLogqThreads - 1) / kLogqThreads;
     if (bx < 1) bx = 1;
     if (bx > 64) bx = 64;

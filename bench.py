@@ -59,6 +59,8 @@ import synthetic  # noqa: E402
 
 METRIC = "quantize+aggregate fp32-gradient GB/s at 1 B200; % of HBM roofline"
 DEFAULT_WORKLOAD = "normal_seg_d2^30_w8_ef"
+# the workload of the extension modes (--buckets, --nat, --dp) unless --workload says otherwise
+MODE_WORKLOAD = "resnet50_t3_w8"
 # the other configurations, reported under "configs" in the one-GPU line
 EXTRA_WORKLOADS = ("normal_d2^20_w4", "resnet50_t3_w8", "gpt2s_laplace_w8", "gpt2s_laplace_w8_l2")
 # host oracle samples: a prefix of this many coordinates (None: the whole workload)
@@ -74,6 +76,11 @@ KERNEL_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_quant_tma.c
 LOGQ_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_logq.cu",
                 "allreduce_compatible_gradient_global_b200/csrc/gq_device.cuh",
                 "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h"]
+LOGQ_COUNTS_FILE = os.path.join(ROOT, "profiles", "logq_kernel_counts.json")
+# Issue peak of the log quantizer's roofline: every SM's four schedulers issue
+# one warp instruction (32 thread instructions) per clock at the maximum SM clock.
+SM_COUNT_B200 = 148
+ISSUE_PER_SM_PER_CLK = 4 * 32
 
 
 def source_hash(files=KERNEL_SOURCES):
@@ -603,6 +610,31 @@ def measure_config(gq, name, K, warmup, dev, with_cpu):
     return res
 
 
+def recorded_logq_counts(rank):
+    """Thread instructions per launch of the two log-quantizer kernels at this
+    rank (ncu, committed), if taken on the current sources; else None."""
+    try:
+        with open(LOGQ_COUNTS_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_hash") != source_hash(LOGQ_SOURCES):
+        return None
+    return rec.get("ranks", {}).get(str(rank))
+
+
+def issue_peak_ginst():
+    """G thread instructions per second the SMs can issue at their maximum clock."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f)["sm_max_mhz"])
+    except (OSError, KeyError, ValueError):
+        mhz = 1965.0
+    sms = torch.cuda.get_device_properties(0).multi_processor_count \
+        if torch.cuda.is_available() else SM_COUNT_B200
+    return sms * ISSUE_PER_SM_PER_CLK * mhz * 1e-3
+
+
 def lq_bytes(W, n, nmats):
     """Algorithmic bytes of the log quantizer on W workers x n factor entries
     (nmats matrices per worker): the quantize pass reads the factors once and
@@ -649,20 +681,36 @@ def measure_lq(gq, r, K, dev, with_cpu):
     step_ms = qm + dm
     qb, db = lq_bytes(W, n, nm)
     peak, peak_kind = measured_hbm_peak()
+    # The quantize kernel is bound by instruction issue (a log1p, two divisions
+    # and a quarter of a Philox call per entry), not by HBM: its roofline is
+    # thread instructions executed (ncu, committed) per second against the
+    # issue peak; the HBM figures stand beside it.
+    counts = recorded_logq_counts(r)
+    ipeak = issue_peak_ginst()
+    hbm = {"achieved": round(qb / (qm * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+           "frac": round(qb / (qm * 1e-3) / 1e9 / peak, 4),
+           "peak_source": f"{peak_kind} (hbm_gbs)", "algorithmic_bytes": qb}
+    if counts is not None:
+        qi = float(counts["quantize_thread_inst"])
+        roof = {"bound": "alu", "kernel": "logq_quantize_kernel",
+                "achieved": round(qi / (qm * 1e-3) / 1e9, 1), "peak": round(ipeak, 1),
+                "unit": "G thread-instr/s", "frac": round(qi / (qm * 1e-3) / 1e9 / ipeak, 4),
+                "peak_source": "derived: SMs x 4 schedulers x 32 lanes x max SM clock",
+                "instructions": int(qi), "instructions_per_entry": round(qi / (W * n), 2),
+                "traffic": counts.get("quantize_dram_bytes"), "hbm": hbm}
+    else:
+        roof = dict(hbm, bound="hbm", kernel="logq_quantize_kernel", traffic=None,
+                    note="no instruction count recorded for the current log-quantizer source")
+    roof.update({"avg_launch_ms": round(qm, 5),
+                 "decode_sum_kernel": {
+                     "achieved": round(db / (dm * 1e-3) / 1e9, 1),
+                     "frac": round(db / (dm * 1e-3) / 1e9 / peak, 4),
+                     "algorithmic_bytes": db, "avg_launch_ms": round(dm, 5)},
+                 "step_hbm": {"achieved": round((qb + db) / (step_ms * 1e-3) / 1e9, 1),
+                              "frac": round((qb + db) / (step_ms * 1e-3) / 1e9 / peak, 4)}})
     res = {"value": round(4 * W * n / (step_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
            "ms_per_step": round(step_ms, 5), "steps": K, "rank": r, "W": W,
-           "elements_per_worker": n, "matrices_per_worker": nm,
-           "roofline": {"bound": "hbm", "kernel": "logq_quantize_kernel",
-                        "achieved": round(qb / (qm * 1e-3) / 1e9, 1), "peak": peak,
-                        "unit": "GB/s", "frac": round(qb / (qm * 1e-3) / 1e9 / peak, 4),
-                        "peak_source": f"{peak_kind} (hbm_gbs)", "traffic": None,
-                        "algorithmic_bytes": qb, "avg_launch_ms": round(qm, 5),
-                        "decode_sum_kernel": {
-                            "achieved": round(db / (dm * 1e-3) / 1e9, 1),
-                            "frac": round(db / (dm * 1e-3) / 1e9 / peak, 4),
-                            "algorithmic_bytes": db, "avg_launch_ms": round(dm, 5)},
-                        "step": {"achieved": round((qb + db) / (step_ms * 1e-3) / 1e9, 1),
-                                 "frac": round((qb + db) / (step_ms * 1e-3) / 1e9 / peak, 4)}},
+           "elements_per_worker": n, "matrices_per_worker": nm, "roofline": roof,
            "timing": "each step's two kernels timed by CUDA events; L2 flushed between steps",
            "code_bytes_per_worker": n, "fp32_bytes_per_worker": 4 * n}
     if with_cpu:
@@ -1184,7 +1232,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(synthetic.WORKLOADS),
+                    help=f"default: {DEFAULT_WORKLOAD} for the bench line and the reference "
+                         f"arm, {MODE_WORKLOAD} for --buckets, --nat and --dp")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
@@ -1216,6 +1266,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload is None:
+        args.workload = MODE_WORKLOAD if (args.buckets or args.nat or args.dp) \
+            else DEFAULT_WORKLOAD
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
