@@ -435,6 +435,15 @@ def run_e2e(gq, args, wk, world, dev):
     step's compute and read-back); otherwise one set, one stream, and the
     upload lands in the workload's own gradient buffer."""
     W, d, cfg, g = wk.W, wk.d, wk.cfg, wk.g
+    # every rank on this host pins its gradient and mean: refuse (and say why)
+    # rather than exhaust the host's memory when the ranks together cannot
+    need = (4 * W * d + 8 * d) * int(os.environ.get("LOCAL_WORLD_SIZE", world))
+    avail = host_available_bytes()
+    if avail is not None and need > 0.8 * avail:
+        return {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
+                "d2h_bytes_per_step": 4 * d + 4,
+                "skipped": f"pinned host buffers for the ranks on this host ({need / 2**30:.0f} "
+                           f"GiB) exceed 80% of its available memory ({avail / 2**30:.0f} GiB)"}
     g_host = torch.empty((W, d), dtype=torch.float32, pin_memory=True)
     g_host.copy_(g)
     set_bytes = 4 * W * d * (2 if cfg.ef else 1) + W * gq.gq_packed_row_bytes(cfg, d) + 8 * d
@@ -482,6 +491,22 @@ def run_e2e(gq, args, wk, world, dev):
             "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4), "steps": K,
             "api": ("gq_step_fused_host, two streams alternating buffer sets" if two else
                     "gq_step_fused_host, one buffer set on one stream (two sets do not fit)")}
+
+
+def host_available_bytes():
+    """Available host memory (bytes), or None if it cannot be read."""
+    try:
+        import psutil
+        return int(psutil.virtual_memory().available)
+    except Exception:
+        try:
+            with open("/proc/meminfo") as f:
+                for line in f:
+                    if line.startswith("MemAvailable:"):
+                        return int(line.split()[1]) * 1024
+        except OSError:
+            return None
+    return None
 
 
 def host_threads():
