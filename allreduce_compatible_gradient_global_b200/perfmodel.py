@@ -71,7 +71,8 @@ class Machine:
     link: float = 770e9
     allreduce_alpha: float = 15e-6
     launch: float = 4e-6
-    pass2_efficiency: float = 0.76  # measured fraction of hbm the fused pass reaches
+    pass2_efficiency: float = 0.81  # measured fraction of hbm the fused pass reaches
+    # (5-bit codes, int8 sums, no error feedback, on the ResNet-50-sized workload)
 
 
 def dp_step_seconds(d, ranks, bits=8, sum_bytes=1, m=Machine(), compressed=True, chunks=1):
