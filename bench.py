@@ -427,14 +427,20 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_e2e(gq, args, wk, world, dev):
-    """Same metric through gq_step_fused_host: every step copies its gradients
-    host->device from pinned memory, runs both kernels and reads the decoded
-    mean and the scale back.  When two buffer sets fit the device, steps
-    alternate between them on two streams (as a training loop that
-    double-buffers its uploads would: one step's upload overlaps the previous
-    step's compute and read-back); otherwise one set, one stream, and the
-    upload lands in the workload's own gradient buffer."""
-    W, d, cfg, g = wk.W, wk.d, wk.cfg, wk.g
+    """The same metric end to end: every step uploads its gradients from pinned
+    host memory, runs both kernels and reads the decoded mean and the scale back
+    into pinned host memory; host <-> device copies inside the timed region.
+
+    Where a second gradient buffer fits the device, the steps are pipelined as a
+    training loop would pipeline them: step i+1's upload (a copy stream, into the
+    other gradient buffer) overlaps step i's kernels (gq_global_norm +
+    gq_quantize_aggregate on the compute stream) and its read-back (a third
+    stream).  The error rows, codes, sum and mean are the workload's one buffer
+    set, so error feedback runs exactly as in consecutive steps; events order
+    each buffer's writer after its last reader.  Otherwise gq_step_fused_host
+    runs each step on one stream, the upload landing in the workload's own
+    gradient buffer."""
+    W, d, cfg, g, buf = wk.W, wk.d, wk.cfg, wk.g, wk.buf
     # every rank on this host pins its gradient and mean: refuse (and say why)
     # rather than exhaust the host's memory when the ranks together cannot
     need = (4 * W * d + 8 * d) * int(os.environ.get("LOCAL_WORLD_SIZE", world))
@@ -446,51 +452,77 @@ def run_e2e(gq, args, wk, world, dev):
                            f"GiB) exceed 80% of its available memory ({avail / 2**30:.0f} GiB)"}
     g_host = torch.empty((W, d), dtype=torch.float32, pin_memory=True)
     g_host.copy_(g)
-    set_bytes = 4 * W * d * (2 if cfg.ef else 1) + W * gq.gq_packed_row_bytes(cfg, d) + 8 * d
+    out_host = torch.empty(d, dtype=torch.float32, pin_memory=True)
+    scale_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
     free_b, _ = torch.cuda.mem_get_info(dev)
-    two = free_b > 1.2 * (set_bytes + 4 * W * d) and 4 * W * d < (8 << 30)
-    streams = [wk.stream] + ([torch.cuda.Stream(device=dev)] if two else [])
-    sets = []
-    for k in range(len(streams)):
-        b = wk.buf if k == 0 else gq.StepBuffers(cfg, W, d, device=dev)
-        sets.append(dict(buf=b, g_dev=g if not two else torch.empty_like(g),
-                         out_host=torch.empty(d, dtype=torch.float32, pin_memory=True),
-                         scale_host=torch.empty(1, dtype=torch.float32, pin_memory=True)))
-    K = args.steps if two else max(1, min(args.steps, 3))
+    pipelined = free_b > 4 * W * d + (2 << 30)
+    K = max(1, min(args.steps, 8))
+    if pipelined:
+        gbufs = [g, torch.empty_like(g)]
+        s_in, s_comp, s_out = torch.cuda.Stream(device=dev), wk.stream, torch.cuda.Stream(
+            device=dev)
+        nsteps = 2 + K
+        h2d = [torch.cuda.Event() for _ in range(nsteps)]
+        comp = [torch.cuda.Event() for _ in range(nsteps)]
+        d2h = [torch.cuda.Event() for _ in range(nsteps)]
 
-    def one(i):
-        n = len(sets)
-        sset, st = sets[i % n], streams[i % n]
-        b = sset["buf"]
-        cfg.step = 1000 + i
-        gq.gq_step_fused_host(g_host, sset["g_dev"], b.e, cfg, b.scale, b.codes, b.sum, b.out,
-                              sset["out_host"], sset["scale_host"], b.ws, st)
+        def one(i):
+            gb = gbufs[i % 2]
+            if i >= 2:
+                s_in.wait_event(comp[i - 2])  # step i-2's kernels were this buffer's readers
+            with torch.cuda.stream(s_in):
+                gb.copy_(g_host, non_blocking=True)
+            h2d[i].record(s_in)
+            s_comp.wait_event(h2d[i])
+            if i >= 1:
+                s_comp.wait_event(d2h[i - 1])  # the mean and scale have been read back
+            cfg.step = 1000 + i
+            gq.gq_global_norm(gb, buf.e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws,
+                              s_comp)
+            gq.gq_quantize_aggregate(gb, buf.e, cfg, buf.scale, buf.codes, buf.sum, buf.out,
+                                     buf.ws, s_comp)
+            comp[i].record(s_comp)
+            s_out.wait_event(comp[i])
+            with torch.cuda.stream(s_out):
+                out_host.copy_(buf.out, non_blocking=True)
+                scale_host.copy_(buf.scale, non_blocking=True)
+            d2h[i].record(s_out)
 
-    for i in range(min(args.warmup, 4) if two else 1):
-        one(i)
-    _sync(world)
-    t0, t1 = _events(2)
-    t0.record(streams[0])
-    for s2 in streams[1:]:
-        s2.wait_event(t0)
-    for i in range(K):
-        one(i)
-    for s2 in streams[1:]:
-        done = torch.cuda.Event()
-        done.record(s2)
-        streams[0].wait_event(done)
-    t1.record(streams[0])
-    torch.cuda.synchronize()
+        for i in range(2):
+            one(i)
+        _sync(world)
+        t0, t1 = _events(2)
+        t0.record(s_in)
+        for i in range(2, 2 + K):
+            one(i)
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        api = ("pipelined: gradient upload on a copy stream into two alternating device "
+               "buffers, gq_global_norm + gq_quantize_aggregate on the compute stream, mean "
+               "and scale read back on a third stream")
+    else:
+        def one(i):
+            cfg.step = 1000 + i
+            gq.gq_step_fused_host(g_host, g, buf.e, cfg, buf.scale, buf.codes, buf.sum, buf.out,
+                                  out_host, scale_host, buf.ws, wk.stream)
+
+        one(0)
+        _sync(world)
+        t0, t1 = _events(2)
+        t0.record(wk.stream)
+        for i in range(1, 1 + K):
+            one(i)
+        t1.record(wk.stream)
+        torch.cuda.synchronize()
+        api = "gq_step_fused_host, one stream (a second gradient buffer does not fit)"
     ms = job_time_ms(t0.elapsed_time(t1), world, dev)
     val = job_gbs(4 * W * d, K, ms, world)
-    for sset in sets:
-        if gq.gq_get_device_status(sset["buf"].ws, streams[0]) != gq.GQ_OK:
-            raise RuntimeError("device flag raised in the end-to-end run")
-    del g_host, sets
+    if gq.gq_get_device_status(buf.ws, wk.stream) != gq.GQ_OK:
+        raise RuntimeError("device flag raised in the end-to-end run")
+    del g_host
     return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
             "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4), "steps": K,
-            "api": ("gq_step_fused_host, two streams alternating buffer sets" if two else
-                    "gq_step_fused_host, one buffer set on one stream (two sets do not fit)")}
+            "api": api}
 
 
 def host_available_bytes():
@@ -1335,7 +1367,8 @@ def main():
         result = run_ours(args, rank, world, local_rank)
         if rank == 0:
             cpu = not (args.no_cpu_baseline or world > 1)
-            sample = None if args.coords else CPU_SAMPLE_COORDS.get(args.workload)
+            # a truncated run (--coords) times the oracle on the same truncation
+            sample = args.coords or CPU_SAMPLE_COORDS.get(args.workload)
             result["cpu_baseline"] = cpu_baseline(args.workload, sample) if cpu else None
             result["cpu_baseline_threads"] = \
                 cpu_baseline_threads(args.workload, sample) if cpu else None
