@@ -444,12 +444,13 @@ def run_e2e(gq, args, wk, world, dev):
     # every rank on this host pins its gradient and mean: refuse (and say why)
     # rather than exhaust the host's memory when the ranks together cannot
     need = (4 * W * d + 8 * d) * int(os.environ.get("LOCAL_WORLD_SIZE", world))
-    avail = host_available_bytes()
-    if avail is not None and need > 0.8 * avail:
+    fits, avail = host_buffers_fit(need, world, dev)
+    if not fits:
         return {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
                 "d2h_bytes_per_step": 4 * d + 4,
                 "skipped": f"pinned host buffers for the ranks on this host ({need / 2**30:.0f} "
-                           f"GiB) exceed 80% of its available memory ({avail / 2**30:.0f} GiB)"}
+                           f"GiB) exceed 80% of its available memory"
+                           + ("" if avail is None else f" ({avail / 2**30:.0f} GiB on this rank)")}
     g_host = torch.empty((W, d), dtype=torch.float32, pin_memory=True)
     g_host.copy_(g)
     out_host = torch.empty(d, dtype=torch.float32, pin_memory=True)
@@ -523,6 +524,23 @@ def run_e2e(gq, args, wk, world, dev):
     return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
             "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4), "steps": K,
             "api": api}
+
+
+def host_buffers_fit(need, world, device):
+    """Whether `need` bytes of pinned host buffers (every local rank's) fit in 80%
+    of the host's available memory, decided once for all ranks: each measures
+    after a barrier (before any rank pins) and the answer is the MIN over ranks,
+    so every rank takes the same collective steps afterwards.  Returns
+    (fits, this rank's available bytes or None)."""
+    if world > 1:
+        torch.distributed.barrier()
+    avail = host_available_bytes()
+    fits = avail is None or need <= 0.8 * avail
+    if world > 1:
+        flag = torch.tensor([1 if fits else 0], dtype=torch.int32, device=device)
+        torch.distributed.all_reduce(flag, op=torch.distributed.ReduceOp.MIN)
+        fits = bool(flag.item())
+    return fits, avail
 
 
 def host_available_bytes():

@@ -56,6 +56,40 @@ def test_job_time_is_max_over_ranks_and_value_sums_ranks():
         assert abs(v - 2 * 32000 * 10 / 5e-3 / 1e9) < 1e-12
 
 
+def _fit_main(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    import bench
+    # rank 1 sees less free host memory (another rank pinned first): the ranks
+    # must still agree, or one would skip the collectives the other enters
+    avail = [100 << 30, 40 << 30][rank]
+    bench.host_available_bytes = lambda: avail
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        fits_big, _ = bench.host_buffers_fit(60 << 30, world, "cpu")
+        fits_small, _ = bench.host_buffers_fit(10 << 30, world, "cpu")
+        q.put((rank, fits_big, fits_small))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_host_buffer_decision_is_the_same_on_every_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_fit_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    # 60 GiB fits rank 0's 80 GiB budget but not rank 1's 32 GiB: both skip;
+    # 10 GiB fits both
+    assert got == [(0, False, True), (1, False, True)]
+
+
 def test_single_rank_needs_no_process_group():
     sys.path.insert(0, ROOT)
     import bench
