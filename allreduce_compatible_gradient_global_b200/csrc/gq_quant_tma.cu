@@ -58,26 +58,20 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 #define GQ_TMA_SPECIALIZE_W8 1
 #endif
 
-// 1: exponential-level codes in a byte table at a fixed shared address (the
-// top nine bits index it directly); 0: a 32-bit table after the ring.
-#ifndef GQ_EXP_BYTE_TABLE
-#define GQ_EXP_BYTE_TABLE 1
-#endif
-// 1: whole tiles take a copy of the block body without bounds checks (3-5%
-// faster on the GPT-2-sized and 8 x 2^26 workloads, even elsewhere).  Not with
-// error feedback: that pass is bound by HBM, measured no gain, and the second
-// copy of its body would spill within two blocks' registers.
-#ifndef GQ_TMA_FULL_TILES
-#define GQ_TMA_FULL_TILES 1
-#endif
-
-constexpr int kExpTableSize = 512;  // indexed by the top nine bits of a rounded level
-// Shared memory after the ring: 2 * stages mbarriers, a tile number per stage
-// (at most kMaxStages), then the exponential-level code table.
+// Whole tiles (all but a ragged last one) take a copy of the block body
+// without coordinate checks: 3-5% faster on the GPT-2-sized and 8 x 2^26
+// workloads, even elsewhere.  Not with error feedback: that pass is bound by
+// HBM, measured no gain, and the second copy of its body would spill within
+// two blocks' registers.
+// The exponential-level code table: signed bytes at a fixed shared address, so
+// the top nine bits of a rounded level index it with no scaling (1.05 ms
+// against 1.12 ms for 32-bit entries after the ring, GPT-2-sized workload).
+constexpr int kExpTableSize = 512;
+// Dynamic shared memory after the ring: 2 * stages mbarriers and a tile number
+// per stage, room for at most kMaxStages.
 constexpr int kMaxStages = 8;
-constexpr size_t kTmaTailBytes = 2 * kMaxStages * sizeof(unsigned long long) +
-                                 kMaxStages * sizeof(long long) +
-                                 (GQ_EXP_BYTE_TABLE ? 0 : kExpTableSize * sizeof(int));
+constexpr size_t kTmaTailBytes =
+    2 * kMaxStages * sizeof(unsigned long long) + kMaxStages * sizeof(long long);
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -184,11 +178,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     unsigned long long* bars = reinterpret_cast<unsigned long long*>(
         smem + (size_t)stages * rows * kTmaTile * sizeof(float));
     long long* tile_of = reinterpret_cast<long long*>(bars + 2 * kMaxStages);
-#if GQ_EXP_BYTE_TABLE
     __shared__ signed char code_table[kExpTableSize];
-#else
-    int* code_table = reinterpret_cast<int*>(tile_of + kMaxStages);
-#endif
     const uint32_t full0 = smem_addr(bars);
     const uint32_t empty0 = smem_addr(bars + stages);
 
@@ -418,7 +408,7 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 store_out4<FULL>(a.out, j0, a.d, o);
             }
         };
-        if (GQ_TMA_FULL_TILES && !EF && (t + 1) * kTmaTile <= a.d)
+        if (!EF && (t + 1) * kTmaTile <= a.d)
             block_body(std::true_type{});
         else if (blk < nblk)
             block_body(std::false_type{});
