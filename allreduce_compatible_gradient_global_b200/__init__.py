@@ -102,6 +102,7 @@ def _load():
         "gq_workspace_init": ([P, ctypes.c_size_t, P], I),
         "gq_get_device_status": ([P, P], I),
         "gq_selftest_wait_timeout": ([P, ctypes.c_uint, P], I),
+        "gq_selftest_fma_div": ([P, ctypes.c_float, P, LL, P], I),
         "gq_global_norm": ([P, P, I, LL, CP, P, P, P, P], I),
         "gq_global_norm_noalloc": ([P, P, I, LL, CP, P, P, P], I),
         "gq_quantize_pack": ([P, P, I, LL, CP, P, P, P, P], I),
@@ -231,6 +232,15 @@ def gq_selftest_wait_timeout(ws, limit_ms=50, stream=None):
     _check(lib().gq_selftest_wait_timeout(_ptr(ws), int(limit_ms), _stream(stream)),
            "gq_selftest_wait_timeout")
     return lib().gq_get_device_status(_ptr(ws), _stream(stream))
+
+
+def gq_selftest_fma_div(a, b, out, stream=None):
+    """out = a / b as the log quantizer divides (see gq_api.h); a, out: float32
+    CUDA tensors of one shape, b a positive finite float."""
+    _need(a, torch.float32, tuple(a.shape), "a")
+    _need(out, torch.float32, tuple(a.shape), "out")
+    _check(lib().gq_selftest_fma_div(_ptr(a), float(b), _ptr(out), a.numel(), _stream(stream)),
+           "gq_selftest_fma_div")
 
 
 def gq_advance_step(step_dev, by=1, stream=None):

@@ -15,6 +15,12 @@
 #include "gq_psgd.h"
 #include "gq_nat.h"
 
+namespace gq {
+// The log map's division as the quantize kernel computes it (gq_logq.cu).
+cudaError_t launch_fma_div_selftest(const float* a, float b, float* out, long long n, int sms,
+                                    cudaStream_t st);
+}  // namespace gq
+
 using namespace gq;
 
 namespace {
@@ -298,6 +304,15 @@ GQ_API int gq_selftest_wait_timeout(void* ws_dev, unsigned int limit_ms, cudaStr
     return cuda_status(launch_wait_timeout_selftest(header_of(ws_dev),
                                                     (unsigned long long)limit_ms * 1000000ull,
                                                     stream));
+}
+
+GQ_API int gq_selftest_fma_div(const float* a_dev, float b, float* out_dev, long long n,
+                               cudaStream_t stream) {
+    if (n < 0 || (n > 0 && (!a_dev || !out_dev)) || !(b > 0.f) || !(b <= 3.4028235e38f))
+        return GQ_ERR_ARG;
+    if (!aligned4(a_dev) || !aligned4(out_dev)) return GQ_ERR_ALIGN;
+    if (n == 0) return GQ_OK;
+    return cuda_status(launch_fma_div_selftest(a_dev, b, out_dev, n, sm_count(), stream));
 }
 
 GQ_API int gq_global_norm(const float* g_dev, const float* e_dev, int W, long long d,

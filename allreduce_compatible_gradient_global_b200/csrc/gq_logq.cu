@@ -21,20 +21,12 @@
 // expression; a code then costs one table read and one multiply by the
 // matrix's max, bit for bit what evaluating Eq. (6) per code gives.
 #include <cfloat>
-#include <type_traits>
 
 #include "gq_internal.h"
 
 namespace gq {
 
 constexpr int kLogqThreads = 512;
-
-// 1: the two divisions of the log map (by the matrix's max and by log1p(a))
-// as a product with the divisor's reciprocal plus one fused correction;
-// 0: IEEE division.
-#ifndef GQ_LOGQ_FMA_DIV
-#define GQ_LOGQ_FMA_DIV 1
-#endif
 
 // a / b for 0 <= a <= b, given rb = RN(1/b) and lo = fma_div_floor(b):
 // q0 = RN(a rb) is within an ulp of a/b, the remainder r = a - q0 b is exact
@@ -73,18 +65,17 @@ __device__ __forceinline__ uint4 philox10_key(uint4 c, uint32_t k0, uint32_t k1)
 }
 
 // One code: the magnitude step of |x| / M on the log map, stochastically
-// rounded with the uniform of `word`, and x's sign.  FAST: the divisions use
-// the reciprocals rM, rlam (and IEEE division below loM, lolam).
-template <bool FAST>
+// rounded with the uniform of `word`, and x's sign.  Both divisions of the map
+// (by the matrix's max and by log1p(a)) use the divisors' reciprocals rM,
+// rlam and floors loM, lolam (div_by_reciprocal).
 __device__ __forceinline__ int logq_code(float xv, float M, bool usable, float alpha, float lam,
                                          float rM, float rlam, float loM, float lolam,
                                          uint32_t word) {
     int k = 0;
     if (usable) {
-        const float ax = fabsf(xv);
-        const float xn = FAST ? div_by_reciprocal(ax, M, rM, loM) : __fdiv_rn(ax, M);
+        const float xn = div_by_reciprocal(fabsf(xv), M, rM, loM);
         const float lg = log1pf(__fmul_rn(alpha, xn));
-        const float tq = FAST ? div_by_reciprocal(lg, lam, rlam, lolam) : __fdiv_rn(lg, lam);
+        const float tq = div_by_reciprocal(lg, lam, rlam, lolam);
         const float y = fminf(__fmul_rn(tq, 127.0f), 127.0f);
         k = floor_y_plus_u(y, unit_plus_u(word));
     }
@@ -148,45 +139,34 @@ __global__ void __launch_bounds__(kLogqThreads, 3)
     const float rM = __frcp_rn(M), rlam = __frcp_rn(lam);
     const float loM = fma_div_floor(M), lolam = fma_div_floor(lam);
 
-    auto quantize_pass = [&](auto fast_tag) {
-        constexpr bool FAST = decltype(fast_tag)::value;
-        // entries 4q..4q+3 share Philox block q
-        const float4* x4 = reinterpret_cast<const float4*>(x);
-        for (long long q = threadIdx.x; q < n4; q += kLogqThreads) {
-            const float4 v = x4[q];  // an L2 hit: pass 1 just read it
-            const uint4 rnd =
-                philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
-            const int c0 =
-                logq_code<FAST>(v.x, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.x);
-            const int c1 =
-                logq_code<FAST>(v.y, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.y);
-            const int c2 =
-                logq_code<FAST>(v.z, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.z);
-            const int c3 =
-                logq_code<FAST>(v.w, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.w);
-            reinterpret_cast<uint32_t*>(codes)[q] = (uint32_t)(c0 & 255) |
-                                                   ((uint32_t)(c1 & 255) << 8) |
-                                                   ((uint32_t)(c2 & 255) << 16) |
-                                                   ((uint32_t)c3 << 24);
-        }
-        // the rest one entry at a time (all of it when the matrix is not aligned)
-        for (long long q = n4 + threadIdx.x; 4 * q < n; q += kLogqThreads) {
-            const uint4 rnd =
-                philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
-            const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+    // entries 4q..4q+3 share Philox block q
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    for (long long q = threadIdx.x; q < n4; q += kLogqThreads) {
+        const float4 v = x4[q];  // an L2 hit: pass 1 just read it
+        const uint4 rnd =
+            philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
+        const int c0 = logq_code(v.x, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.x);
+        const int c1 = logq_code(v.y, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.y);
+        const int c2 = logq_code(v.z, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.z);
+        const int c3 = logq_code(v.w, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.w);
+        reinterpret_cast<uint32_t*>(codes)[q] = (uint32_t)(c0 & 255) |
+                                               ((uint32_t)(c1 & 255) << 8) |
+                                               ((uint32_t)(c2 & 255) << 16) |
+                                               ((uint32_t)c3 << 24);
+    }
+    // the rest one entry at a time (all of it when the matrix is not aligned)
+    for (long long q = n4 + threadIdx.x; 4 * q < n; q += kLogqThreads) {
+        const uint4 rnd =
+            philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
+        const uint32_t words[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const long long i = 4 * q + t;
-                if (i < n)
-                    codes[i] = (signed char)logq_code<FAST>(__ldg(x + i), M, usable, alpha, lam,
-                                                            rM, rlam, loM, lolam, words[t]);
-            }
+        for (int t = 0; t < 4; ++t) {
+            const long long i = 4 * q + t;
+            if (i < n)
+                codes[i] = (signed char)logq_code(__ldg(x + i), M, usable, alpha, lam, rM,
+                                                  rlam, loM, lolam, words[t]);
         }
-    };
-    if (GQ_LOGQ_FMA_DIV)
-        quantize_pass(std::true_type{});
-    else
-        quantize_pass(std::false_type{});
+    }
 }
 
 // The inverse map of magnitude step m (Eq. (6) without the max), m = 0..128
@@ -201,7 +181,8 @@ __device__ __forceinline__ float logq_decode_one(int k, float M, const float* ta
     return k < 0 ? -xm : xm;
 }
 
-__global__ void __launch_bounds__(kLogqThreads) logq_decode_kernel(const __grid_constant__ LogqArgs a) {
+__global__ void __launch_bounds__(kLogqThreads)
+    logq_decode_kernel(const __grid_constant__ LogqArgs a) {
     __shared__ float tab[129];  // every int8 magnitude, 0..128
     const float alpha = a.alpha;
     const float lam = log1pf(alpha);
@@ -240,6 +221,24 @@ __global__ void __launch_bounds__(kLogqThreads) logq_decode_kernel(const __grid_
         }
         a.out[off + i] = acc;
     }
+}
+
+// Self-test of the log map's division: out[i] = a[i] / b as the quantize
+// kernel computes it (div_by_reciprocal with b's reciprocal and floor).
+__global__ void fma_div_selftest_kernel(const float* a, float b, float* out, long long n) {
+    const float rb = __frcp_rn(b), lo = fma_div_floor(b);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x)
+        out[i] = div_by_reciprocal(a[i], b, rb, lo);
+}
+
+cudaError_t launch_fma_div_selftest(const float* a, float b, float* out, long long n, int sms,
+                                    cudaStream_t st) {
+    long long blocks = (n + 255) / 256;
+    if (blocks > (long long)sms * 8) blocks = (long long)sms * 8;
+    if (blocks < 1) blocks = 1;
+    fma_div_selftest_kernel<<<(unsigned)blocks, 256, 0, st>>>(a, b, out, n);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_logq_quantize(const LogqArgs& a, cudaStream_t st) {

@@ -167,6 +167,17 @@ GQ_API int gq_get_device_status(void* ws_dev, cudaStream_t stream);
  * faults and the context stays usable. */
 GQ_API int gq_selftest_wait_timeout(void* ws_dev, unsigned int limit_ms, cudaStream_t stream);
 
+/* Self-test of the log quantizer's division (no counterpart in the pages):
+ * out_dev[i] = a_dev[i] / b for i < n (device arrays, caller-owned, 4-byte
+ * aligned), computed exactly as gq_logq_quantize divides an entry by its
+ * matrix's max and a log by log1p(alpha): the product with b's reciprocal plus
+ * one fused correction (Markstein's method) where the dividend is at least
+ * 2^-100 max(1, b) and b < 2^125, IEEE division elsewhere.  Tests compare it
+ * with IEEE division bit for bit.  b must be positive and finite (else
+ * GQ_ERR_ARG); dividends are meant to lie in [0, b]. */
+GQ_API int gq_selftest_fma_div(const float* a_dev, float b, float* out_dev, long long n,
+                               cudaStream_t stream);
+
 /* Step 1 -- global scale.  g_dev, e_dev (NULL unless cfg->ef): [W][d] fp32.
  * v = fl(g + e).  L2: per-worker sum of squares with fp32 squares, fp32
  * partial sums of at most 16 terms and fp64 accumulation, combined in a

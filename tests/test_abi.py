@@ -46,6 +46,14 @@ def test_library_exports_every_declared_symbol(gq):
         assert getattr(lib, n) is not None
 
 
+def test_division_selftest_checks_its_arguments_on_the_host(gq):
+    lib = gq.lib()
+    for b in (0.0, -1.0, float("inf"), float("nan")):
+        assert lib.gq_selftest_fma_div(None, b, None, 0, None) == gq.GQ_ERR_ARG
+    assert lib.gq_selftest_fma_div(None, 2.0, None, 0, None) == gq.GQ_OK  # nothing to do
+    assert lib.gq_selftest_fma_div(None, 2.0, None, 5, None) == gq.GQ_ERR_ARG
+
+
 def test_version_and_status_strings(gq):
     assert gq.gq_version() >= 100
     for st in (0, -1, -2, -3, -4, -5, -6, -7):
