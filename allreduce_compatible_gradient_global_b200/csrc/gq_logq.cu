@@ -28,24 +28,26 @@ namespace gq {
 
 constexpr int kLogqThreads = 512;
 
-// a / b for 0 <= a <= b, given rb = RN(1/b) and lo = fma_div_floor(b):
-// q0 = RN(a rb) is within an ulp of a/b, the remainder r = a - q0 b is exact
-// in one fused multiply-add, and RN(q0 + r rb) is the correctly rounded
-// quotient (Markstein, "Computation of elementary functions on the IBM RISC
-// System/6000 processor", IBM J. Res. Develop. 34(1), 1990) -- provided
-// neither the reciprocal, the remainder nor the correction underflows.
-// Dividends below lo (a quotient or a dividend under 2^-100, or any dividend
-// of a divisor from 2^125 up, whose reciprocal is subnormal) therefore take
-// IEEE division.  Measured equal to IEEE division on 1.7e10 sampled quotients
-// in that domain over 255 divisors from 2^-110 to 2^110, edge mantissas and
-// log1p(10) among them; outside it the correction alone missed on 0.6% of
-// samples, and for the divisor FLT_MAX on 7 in 6.7e7.
-__device__ __forceinline__ float fma_div_floor(float b) {
-    return b < 0x1p125f ? 0x1p-100f * fmaxf(1.0f, b) : __int_as_float(0x7F800000);  // +inf
-}
+// a / b for 0 <= a <= b, given rb = RN(1/b): q0 = RN(a rb) is within an ulp
+// of a/b, the remainder r = a - q0 b is exact in one fused multiply-add, and
+// RN(q0 + r rb) is the correctly rounded quotient (Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Develop. 34(1), 1990) -- provided neither the reciprocal, the remainder nor
+// the correction underflows or overflows.  The domain: a divisor in
+// [2^-125, 2^125) (a normal, finite reciprocal; fma_div_ok) and a dividend
+// that is 0 (exact either way) or at least lo = 2^-100 max(1, b)
+// (fma_div_floor); everything else takes IEEE division.  Measured equal to
+// IEEE division on 1.7e10 sampled quotients in that domain over 255 divisors
+// from 2^-110 to 2^110, edge mantissas and log1p(10) among them; outside it
+// the correction alone missed on 0.6% of samples, and for the divisor
+// FLT_MAX on 7 in 6.7e7.
+__device__ __forceinline__ bool fma_div_ok(float b) { return b >= 0x1p-125f && b < 0x1p125f; }
 
-__device__ __forceinline__ float div_by_reciprocal(float a, float b, float rb, float lo) {
-    if (a < lo) return __fdiv_rn(a, b);
+__device__ __forceinline__ float fma_div_floor(float b) { return 0x1p-100f * fmaxf(1.0f, b); }
+
+__device__ __forceinline__ float div_by_reciprocal(float a, float b, float rb, float lo,
+                                                   bool ok) {
+    if (!ok || (a < lo && a != 0.f)) return __fdiv_rn(a, b);
     const float q0 = __fmul_rn(a, rb);
     const float r = __fmaf_rn(-q0, b, a);
     return __fmaf_rn(r, rb, q0);
@@ -64,18 +66,82 @@ __device__ __forceinline__ uint4 philox10_key(uint4 c, uint32_t k0, uint32_t k1)
     return c;
 }
 
+// The corrected quotient without the domain check, for callers that checked it.
+__device__ __forceinline__ float div_by_reciprocal_in_domain(float a, float b, float rb) {
+    const float q0 = __fmul_rn(a, rb);
+    const float r = __fmaf_rn(-q0, b, a);
+    return __fmaf_rn(r, rb, q0);
+}
+
+// Magnitude step of y = 127 t on the log map, rounded with the uniform of
+// `word`, and the sign of v.
+__device__ __forceinline__ int logq_round(float tq, float v, uint32_t word) {
+    const float y = fminf(__fmul_rn(tq, 127.0f), 127.0f);
+    return with_sign_of(floor_y_plus_u(y, unit_plus_u(word)), v);
+}
+
+// Whether four non-negative dividends all lie in the corrected quotient's
+// domain: each is 0 (exact either way) or at least lo.  On the bit patterns
+// minus one, compared unsigned, 0 wraps to the largest value and the order of
+// the rest is the order of the floats.
+__device__ __forceinline__ bool in_domain4(float a0, float a1, float a2, float a3, float lo) {
+    const uint32_t m = min(min(__float_as_uint(a0) - 1u, __float_as_uint(a1) - 1u),
+                           min(__float_as_uint(a2) - 1u, __float_as_uint(a3) - 1u));
+    return m >= __float_as_uint(lo) - 1u;
+}
+
+// Four codes from one Philox block.  Each division takes the corrected
+// quotient when all four dividends lie in its domain, IEEE division for all
+// four otherwise: the same quotients either way, with one domain check per
+// four entries instead of one per entry.
+__device__ __forceinline__ uint32_t logq_codes4(float4 v, float M, float alpha, float lam,
+                                                float rM, float rlam, float loM, float lolam,
+                                                bool okM, bool oklam, uint4 rnd) {
+    const float a0 = fabsf(v.x), a1 = fabsf(v.y), a2 = fabsf(v.z), a3 = fabsf(v.w);
+    float x0, x1, x2, x3;
+    if (okM && in_domain4(a0, a1, a2, a3, loM)) {
+        x0 = div_by_reciprocal_in_domain(a0, M, rM);
+        x1 = div_by_reciprocal_in_domain(a1, M, rM);
+        x2 = div_by_reciprocal_in_domain(a2, M, rM);
+        x3 = div_by_reciprocal_in_domain(a3, M, rM);
+    } else {
+        x0 = __fdiv_rn(a0, M);
+        x1 = __fdiv_rn(a1, M);
+        x2 = __fdiv_rn(a2, M);
+        x3 = __fdiv_rn(a3, M);
+    }
+    const float l0 = log1pf(__fmul_rn(alpha, x0)), l1 = log1pf(__fmul_rn(alpha, x1));
+    const float l2 = log1pf(__fmul_rn(alpha, x2)), l3 = log1pf(__fmul_rn(alpha, x3));
+    float t0, t1, t2, t3;
+    if (oklam && in_domain4(l0, l1, l2, l3, lolam)) {
+        t0 = div_by_reciprocal_in_domain(l0, lam, rlam);
+        t1 = div_by_reciprocal_in_domain(l1, lam, rlam);
+        t2 = div_by_reciprocal_in_domain(l2, lam, rlam);
+        t3 = div_by_reciprocal_in_domain(l3, lam, rlam);
+    } else {
+        t0 = __fdiv_rn(l0, lam);
+        t1 = __fdiv_rn(l1, lam);
+        t2 = __fdiv_rn(l2, lam);
+        t3 = __fdiv_rn(l3, lam);
+    }
+    const int c0 = logq_round(t0, v.x, rnd.x), c1 = logq_round(t1, v.y, rnd.y);
+    const int c2 = logq_round(t2, v.z, rnd.z), c3 = logq_round(t3, v.w, rnd.w);
+    return (uint32_t)(c0 & 255) | ((uint32_t)(c1 & 255) << 8) | ((uint32_t)(c2 & 255) << 16) |
+           ((uint32_t)c3 << 24);
+}
+
 // One code: the magnitude step of |x| / M on the log map, stochastically
 // rounded with the uniform of `word`, and x's sign.  Both divisions of the map
 // (by the matrix's max and by log1p(a)) use the divisors' reciprocals rM,
 // rlam and floors loM, lolam (div_by_reciprocal).
 __device__ __forceinline__ int logq_code(float xv, float M, bool usable, float alpha, float lam,
-                                         float rM, float rlam, float loM, float lolam,
-                                         uint32_t word) {
+                                         float rM, float rlam, float loM, float lolam, bool okM,
+                                         bool oklam, uint32_t word) {
     int k = 0;
     if (usable) {
-        const float xn = div_by_reciprocal(fabsf(xv), M, rM, loM);
+        const float xn = div_by_reciprocal(fabsf(xv), M, rM, loM, okM);
         const float lg = log1pf(__fmul_rn(alpha, xn));
-        const float tq = div_by_reciprocal(lg, lam, rlam, lolam);
+        const float tq = div_by_reciprocal(lg, lam, rlam, lolam, oklam);
         const float y = fminf(__fmul_rn(tq, 127.0f), 127.0f);
         k = floor_y_plus_u(y, unit_plus_u(word));
     }
@@ -138,6 +204,7 @@ __global__ void __launch_bounds__(kLogqThreads, 3)
     const uint32_t wid = a.worker0 + (uint32_t)w;
     const float rM = __frcp_rn(M), rlam = __frcp_rn(lam);
     const float loM = fma_div_floor(M), lolam = fma_div_floor(lam);
+    const bool okM = fma_div_ok(M), oklam = fma_div_ok(lam);
 
     // entries 4q..4q+3 share Philox block q
     const float4* x4 = reinterpret_cast<const float4*>(x);
@@ -145,14 +212,8 @@ __global__ void __launch_bounds__(kLogqThreads, 3)
         const float4 v = x4[q];  // an L2 hit: pass 1 just read it
         const uint4 rnd =
             philox10_key(philox_counter((unsigned long long)q, step, wid), k0, k1);
-        const int c0 = logq_code(v.x, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.x);
-        const int c1 = logq_code(v.y, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.y);
-        const int c2 = logq_code(v.z, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.z);
-        const int c3 = logq_code(v.w, M, usable, alpha, lam, rM, rlam, loM, lolam, rnd.w);
-        reinterpret_cast<uint32_t*>(codes)[q] = (uint32_t)(c0 & 255) |
-                                               ((uint32_t)(c1 & 255) << 8) |
-                                               ((uint32_t)(c2 & 255) << 16) |
-                                               ((uint32_t)c3 << 24);
+        reinterpret_cast<uint32_t*>(codes)[q] =
+            usable ? logq_codes4(v, M, alpha, lam, rM, rlam, loM, lolam, okM, oklam, rnd) : 0u;
     }
     // the rest one entry at a time (all of it when the matrix is not aligned)
     for (long long q = n4 + threadIdx.x; 4 * q < n; q += kLogqThreads) {
@@ -164,7 +225,7 @@ __global__ void __launch_bounds__(kLogqThreads, 3)
             const long long i = 4 * q + t;
             if (i < n)
                 codes[i] = (signed char)logq_code(__ldg(x + i), M, usable, alpha, lam, rM,
-                                                  rlam, loM, lolam, words[t]);
+                                                  rlam, loM, lolam, okM, oklam, words[t]);
         }
     }
 }
@@ -227,9 +288,10 @@ __global__ void __launch_bounds__(kLogqThreads)
 // kernel computes it (div_by_reciprocal with b's reciprocal and floor).
 __global__ void fma_div_selftest_kernel(const float* a, float b, float* out, long long n) {
     const float rb = __frcp_rn(b), lo = fma_div_floor(b);
+    const bool ok = fma_div_ok(b);
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x)
-        out[i] = div_by_reciprocal(a[i], b, rb, lo);
+        out[i] = div_by_reciprocal(a[i], b, rb, lo, ok);
 }
 
 cudaError_t launch_fma_div_selftest(const float* a, float b, float* out, long long n, int sms,

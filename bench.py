@@ -501,6 +501,14 @@ def run_e2e(gq, args, wk, world, dev):
         api = ("pipelined: gradient upload on a copy stream into two alternating device "
                "buffers, gq_global_norm + gq_quantize_aggregate on the compute stream, mean "
                "and scale read back on a third stream")
+        # the bound: the same upload alone, over the host link
+        u0, u1 = _events(2)
+        u0.record(s_in)
+        with torch.cuda.stream(s_in):
+            gbufs[1].copy_(g_host, non_blocking=True)
+        u1.record(s_in)
+        torch.cuda.synchronize()
+        link_gbs = 4 * W * d / (u0.elapsed_time(u1) * 1e-3) / 1e9
     else:
         def one(i):
             cfg.step = 1000 + i
@@ -516,14 +524,19 @@ def run_e2e(gq, args, wk, world, dev):
         t1.record(wk.stream)
         torch.cuda.synchronize()
         api = "gq_step_fused_host, one stream (a second gradient buffer does not fit)"
+        link_gbs = None
     ms = job_time_ms(t0.elapsed_time(t1), world, dev)
     val = job_gbs(4 * W * d, K, ms, world)
     if gq.gq_get_device_status(buf.ws, wk.stream) != gq.GQ_OK:
         raise RuntimeError("device flag raised in the end-to-end run")
     del g_host
-    return {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
-            "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4), "steps": K,
-            "api": api}
+    out = {"value": round(val, 3), "unit": "GB/s", "h2d_bytes_per_step": 4 * W * d,
+           "d2h_bytes_per_step": 4 * d + 4, "ms_per_step": round(ms / K, 4), "steps": K,
+           "api": api}
+    if link_gbs is not None:  # this rank's upload alone; the value is the whole job's
+        out["host_link_upload_gbs"] = round(link_gbs, 2)
+        out["frac_of_host_link"] = round(val / world / link_gbs, 4)
+    return out
 
 
 def host_buffers_fit(need, world, device):

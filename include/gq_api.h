@@ -171,10 +171,10 @@ GQ_API int gq_selftest_wait_timeout(void* ws_dev, unsigned int limit_ms, cudaStr
  * out_dev[i] = a_dev[i] / b for i < n (device arrays, caller-owned, 4-byte
  * aligned), computed exactly as gq_logq_quantize divides an entry by its
  * matrix's max and a log by log1p(alpha): the product with b's reciprocal plus
- * one fused correction (Markstein's method) where the dividend is at least
- * 2^-100 max(1, b) and b < 2^125, IEEE division elsewhere.  Tests compare it
- * with IEEE division bit for bit.  b must be positive and finite (else
- * GQ_ERR_ARG); dividends are meant to lie in [0, b]. */
+ * one fused correction (Markstein's method) where 2^-125 <= b < 2^125 and the
+ * dividend is 0 or at least 2^-100 max(1, b), IEEE division elsewhere.  Tests
+ * compare it with IEEE division bit for bit.  b must be positive and finite
+ * (else GQ_ERR_ARG); dividends are meant to lie in [0, b]. */
 GQ_API int gq_selftest_fma_div(const float* a_dev, float b, float* out_dev, long long n,
                                cudaStream_t stream);
 

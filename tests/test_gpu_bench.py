@@ -42,6 +42,7 @@ def test_bench_line_fields(workload, coords):
     assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-3
     e2e = line["e2e"]
     assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] == 4 * 8 * coords
+    assert e2e["api"].startswith("pipelined") and 0 < e2e["frac_of_host_link"] < 1.2
     cpu = line["cpu_baseline"]
     assert cpu["kind"] == "oracle" and cpu["cores"] == 1 and cpu["value"] > 0
 
