@@ -132,6 +132,8 @@ def test_split_pipeline_equals_fused(gq, oracle, W, d, kw):
     (4, 4097, dict(s=15, bits=5, wire="int8")),
     (8, 20000, dict(levels="exp", L=8, bits=5, wire="int16", scale_kind="maxabs")),
     (16, 5003, dict(s=127, bits=8, wire="f16")),
+    (3, 10001, dict(levels="exp", L=5, bits=4, wire="int8", scale_kind="l2")),  # generic W
+    (4, 12345, dict(levels="exp", L=13, bits=5, wire="int16", scale_kind="l2")),
 ])
 def test_error_feedback_steps_match_oracle(gq, oracle, W, d, kw, split):
     cfg = gq.GQConfig(**{"ef": True, "seed": 77, **kw})
@@ -145,6 +147,39 @@ def test_error_feedback_steps_match_oracle(gq, oracle, W, d, kw, split):
         ref = check_against_oracle(oracle, cfg, g.cpu().numpy(), e_ref, r)
         e_gpu = torch.from_numpy(r["e"]).cuda()
         e_ref = ref["e"]
+
+
+@pytest.mark.parametrize("ef", [False, True])
+@pytest.mark.parametrize("W,d,kw", [
+    (8, 1 << 20, dict(s=127, bits=8, wire="int16")),       # whole tiles, unrolled W
+    (8, 30001, dict(s=127, bits=8, wire="int16")),         # ragged tail
+    (3, 10001, dict(s=7, bits=4, wire="int8")),            # generic W
+    (8, 40001, dict(levels="exp", L=8, bits=5, wire="int16", scale_kind="maxabs")),
+    (5, 7001, dict(levels="exp", L=6, bits=4, wire="int16", scale_kind="l2")),
+])
+def test_fused_pass_without_codes_matches_oracle(gq, oracle, W, d, kw, ef):
+    """With no code buffer the fused pass writes only the sums, the means and
+    the error-feedback buffer; those match the oracle bit for bit."""
+    cfg = gq.GQConfig(**{"ef": ef, "seed": 4242, "step": 3, **kw})
+    g = synthetic.make_gradients(W, d, "normal_seg", seed=d + W, device="cuda", seg=777,
+                                 lo=-4, hi=0)
+    e0 = (0.01 * synthetic.make_gradients(W, d, "normal", seed=d + 1, device="cuda")
+          if ef else None)
+    buf = gq.StepBuffers(cfg, W, d, codes=False, ef=False)
+    e_dev = e0.clone() if ef else None
+    gq.gq_global_norm(g, e_dev, cfg, buf.scale, buf.norms, buf.ws)
+    gq.gq_quantize_aggregate(g, e_dev, cfg, buf.scale, None, buf.sum, buf.out, buf.ws)
+    assert gq.gq_get_device_status(buf.ws) == gq.GQ_OK
+    torch.cuda.synchronize()
+    S = np.float32(buf.scale.item())
+    sk = oracle.SCALE_L2 if cfg.scale_kind == "l2" else oracle.SCALE_MAXABS
+    e_host = e0.cpu().numpy() if ef else None
+    ref = oracle.step(g.cpu().numpy(), e_host, scale_kind=sk, seed=cfg.seed, step=cfg.step,
+                      ef=ef, bits=cfg.bits, S=S, **oracle_kw(cfg))
+    assert np.array_equal(buf.sum.cpu().numpy().astype(np.int32), ref["sum"]), "integer sums differ"
+    assert np.array_equal(buf.out.cpu().numpy().view(np.uint32), ref["out"].view(np.uint32))
+    if ef:
+        assert np.array_equal(e_dev.cpu().numpy().view(np.uint32), ref["e"].view(np.uint32))
 
 
 def test_zero_input_and_empty(gq, oracle):
