@@ -135,6 +135,7 @@ class ClockSampler:
 
     def __init__(self, device_index):
         self.samples = []
+        self.times = []        # time.perf_counter() of each sample
         self.reasons = 0
         self.max_mhz = None
         self._stop = threading.Event()
@@ -172,6 +173,7 @@ class ClockSampler:
                 mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
                 self.samples.append(mhz)
+                self.times.append(time.perf_counter())
                 self.reasons |= int(rs)
             except Exception:
                 pass
@@ -186,6 +188,12 @@ class ClockSampler:
         if self._thread is not None:
             self._stop.set()
             self._thread.join()
+
+    def median_between(self, t0, t1):
+        """Median SM clock of the samples taken in [t0, t1] (perf_counter
+        seconds), or None if none fell there."""
+        m = [c for t, c in zip(self.times, self.samples) if t0 <= t <= t1]
+        return statistics.median(m) if m else None
 
     def summary(self):
         if self.nvml is None:
@@ -971,6 +979,8 @@ def run_sweep(args):
     peak, peak_kind = measured_hbm_peak()
     rows = []
     W = 8
+    sampler = ClockSampler(0)   # sm_mhz of a row: median clock over its timed steps
+    sampler.start()
     for ef in (False, True):
         for lg in range(16, 31, 2):
             d = 1 << lg
@@ -979,7 +989,11 @@ def run_sweep(args):
             g = synthetic.make_gradients(W, d, "normal", seed=lg, device="cuda")
             buf = gq.StepBuffers(cfg, W, d)
             K = max(20, min(400, int(2e9 // (4 * W * d))))
+            sampler.samples.clear()
+            sampler.times.clear()
+            t_row = time.perf_counter()
             n_ms, q_ms, step_ms = time_step_pair(gq, g, buf.e, cfg, buf, K, 5, stream)
+            row_mhz = sampler.median_between(t_row, time.perf_counter())
             graph_ms = time_step_graph(gq, g, cfg, W, d, K)
             p1, p2 = algorithmic_bytes(gq, cfg, W, d)
             ora = None if args.no_cpu_baseline else sweep_oracle(g, ef)
@@ -990,9 +1004,11 @@ def run_sweep(args):
                          "step_frac": round((p1 + p2) / (step_ms * 1e-3) / 1e9 / peak, 4),
                          "quant_frac": round(p2 / (q_ms * 1e-3) / 1e9 / peak, 4),
                          "graph_step_ms": round(graph_ms, 5),
-                         "graph_grad_gbs": round(4 * W * d / (graph_ms * 1e-3) / 1e9, 1)})
+                         "graph_grad_gbs": round(4 * W * d / (graph_ms * 1e-3) / 1e9, 1),
+                         "sm_mhz": row_mhz})
             del g, buf
             torch.cuda.empty_cache()
+    sampler.stop()
     return {"metric": METRIC, "mode": "sweep", "unit": "GB/s", "peak": peak,
             "peak_source": peak_kind, "W": W, "config": "uniform s=15, 5-bit, int8 sum, L2",
             "oracle": None if args.no_cpu_baseline else
@@ -1001,6 +1017,78 @@ def run_sweep(args):
                        "coordinates of the row's gradient (all 8 workers), single-threaded; "
                        "GB/s of fp32 gradient"},
             "sweep": rows}
+
+
+def time_launch_series(gq, sampler, d, n, idle_s):
+    """n fused passes (W = 8, uniform s = 15, 5-bit codes, int8 sums, L2 scale,
+    no error feedback) launched back to back after idle_s seconds of idle GPU:
+    per launch its fraction of the copy figure and the median SM clock while it
+    ran (the launch's device interval placed on the host clock from the series'
+    first event)."""
+    W = 8
+    cfg = gq.GQConfig(levels="uniform", s=15, bits=5, wire="int8", scale_kind="l2", seed=0x5EED)
+    g = synthetic.make_gradients(W, d, "normal", seed=3, device="cuda")
+    buf = gq.StepBuffers(cfg, W, d)
+    gq.gq_global_norm(g, None, cfg, buf.scale, buf.norms, buf.ws)
+    for i in range(3):
+        gq.gq_quantize_aggregate(g, None, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws)
+    torch.cuda.synchronize()
+    time.sleep(idle_s)
+    ev = _events(n + 1)
+    stream = torch.cuda.current_stream()
+    t0 = time.perf_counter()
+    ev[0].record(stream)
+    for i in range(n):
+        cfg.step = 3 + i
+        gq.gq_quantize_aggregate(g, None, cfg, buf.scale, buf.codes, buf.sum, buf.out, buf.ws)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if gq.gq_get_device_status(buf.ws) != gq.GQ_OK:
+        raise RuntimeError("device flag raised in the launch series")
+    _, p2 = algorithmic_bytes(gq, cfg, W, d)
+    peak, _ = measured_hbm_peak()
+    launches = []
+    for i in range(n):
+        a = ev[0].elapsed_time(ev[i]) * 1e-3
+        ms = ev[i].elapsed_time(ev[i + 1])
+        launches.append((p2 / (ms * 1e-3) / 1e9 / peak,
+                         sampler.median_between(t0 + a, t0 + a + ms * 1e-3)))
+    del g, buf
+    torch.cuda.empty_cache()
+    return launches
+
+
+def run_power(args):
+    """The fused pass without error feedback is bound by instruction issue, so
+    its speed follows the SM clock, which the 1 kW power cap lowers under
+    sustained load.  The same launch at d = 2^26 is timed as a short burst and
+    as a sustained series, and at d = 2^30 as a series: per segment the median
+    fraction of the copy figure and the median SM clock, and the fraction
+    scaled to the maximum clock."""
+    import allreduce_compatible_gradient_global_b200 as gq
+    torch.cuda.set_device(0)
+    sampler = ClockSampler(0)
+    sampler.start()
+    series = [(1 << 26, 20), (1 << 26, 600), (1 << 30, 40)]
+    rows = []
+    try:
+        for d, n in series:
+            launches = time_launch_series(gq, sampler, d, n, 1.0)
+            for name, part in (("first 5", launches[:5]), ("first 20", launches[:20]),
+                               ("last 20", launches[-20:])):
+                fr = statistics.median(f for f, _ in part)
+                mhz = [m for _, m in part if m is not None]
+                mhz = statistics.median(mhz) if mhz else None
+                rows.append({"d": d, "launches": n, "segment": name, "frac": round(fr, 4),
+                             "sm_mhz": mhz,
+                             "frac_at_max_clock": (round(fr * sampler.max_mhz / mhz, 4)
+                                                   if mhz and sampler.max_mhz else None)})
+    finally:
+        sampler.stop()
+    return {"metric": "fused pass fraction of the measured copy figure against the SM clock",
+            "mode": "power", "unit": "fraction", "config": "W=8, uniform s=15, 5-bit codes, "
+            "int8 sums, L2 scale, no error feedback; 1 s idle before each series",
+            "clocks": sampler.summary(), "rows": rows}
 
 
 def run_buckets(args):
@@ -1337,6 +1425,9 @@ def main():
                     help="one JSON line timing natural compression (quantize + decode-sum)")
     ap.add_argument("--lq", action="store_true",
                     help="one JSON line with the LQ-SGD log-quantizer timings")
+    ap.add_argument("--power", action="store_true",
+                    help="one JSON line: the fused pass as a burst and sustained, with the "
+                         "SM clock of each segment")
     ap.add_argument("--buckets", action="store_true",
                     help="one JSON line comparing the global scale with per-bucket scales")
     ap.add_argument("--dp", action="store_true",
@@ -1366,10 +1457,11 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
-    if args.sweep or args.lq or args.buckets or args.lqsgd or args.nat:
+    if args.sweep or args.lq or args.buckets or args.lqsgd or args.nat or args.power:
         if rank == 0:
             fn = (run_sweep if args.sweep else run_lq if args.lq else
-                  run_buckets if args.buckets else run_nat if args.nat else run_lqsgd)
+                  run_buckets if args.buckets else run_nat if args.nat else
+                  run_power if args.power else run_lqsgd)
             print(json.dumps(fn(args)), flush=True)
         return
 

@@ -56,3 +56,11 @@ def test_lq_mode_reports_its_issue_roofline():
         assert roof["bound"] == "alu", roof.get("note")
         assert 0 < roof["frac"] < 1.0
         assert roof["decode_sum_kernel"]["avg_launch_ms"] > 0
+
+
+def test_power_mode_reports_clocks_per_segment():
+    line = run_bench("--power")
+    assert line["mode"] == "power" and len(line["rows"]) == 9
+    for r in line["rows"]:
+        assert 0 < r["frac"] < 2 and r["sm_mhz"] and r["sm_mhz"] > 0
+        assert r["frac_at_max_clock"] >= r["frac"] - 1e-9
