@@ -1395,13 +1395,6 @@ def run_lq(args):
             "W": synthetic.LQ_WORKLOAD["W"], "rows": rows}
 
 
-def _free_port():
-    import socket
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1471,11 +1464,15 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     if args.dp:
+        store_dir = None
         if world == 1:
             import datetime
+            import tempfile
             torch.cuda.set_device(local_rank)
+            # a one-rank group: its rendezvous is a file store (no TCP port)
+            store_dir = tempfile.mkdtemp(prefix="gq_bench_")
             torch.distributed.init_process_group(
-                "nccl", rank=0, world_size=1, init_method="tcp://127.0.0.1:%d" % _free_port(),
+                "nccl", rank=0, world_size=1, init_method="file://" + store_dir + "/store",
                 timeout=datetime.timedelta(seconds=120),
                 device_id=torch.device("cuda", local_rank))
         try:
@@ -1485,6 +1482,9 @@ def main():
         finally:
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
+            if store_dir is not None:
+                import shutil
+                shutil.rmtree(store_dir, ignore_errors=True)
         return
     try:
         result = run_ours(args, rank, world, local_rank)

@@ -9,7 +9,6 @@ single-process step on all W rows, bit for bit (the oracle's per-worker norms do
 not depend on how rows are grouped).
 """
 import os
-import socket
 
 import numpy as np
 import pytest
@@ -57,10 +56,10 @@ class OracleOps:
         return 0
 
 
-def _free_port():
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
+def _store(tmp_path):
+    """The rendezvous of a test's group: a file store in the test's own
+    directory, so no TCP port can collide with another process's."""
+    return "file://" + str(tmp_path / "store")
 
 
 CASES = {
@@ -72,10 +71,9 @@ CASES = {
 }
 
 
-def _rank_main(rank, world, port, case, w_local, d, outdir, chunks=1):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+def _rank_main(rank, world, store, case, w_local, d, outdir, chunks=1):
     import datetime
-    dist.init_process_group("gloo", rank=rank, world_size=world,
+    dist.init_process_group("gloo", init_method=store, rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
         import oracle
@@ -107,7 +105,7 @@ def test_two_ranks_equal_the_single_process_step(oracle, tmp_path, case, w_local
     """chunks > 1: chunk k + 1 is quantized while chunk k is all-reduced; each
     chunk draws the uniforms of its own coordinates (coord0)."""
     world, d = 2, 700
-    mp.start_processes(_rank_main, args=(world, _free_port(), case, w_local, d, str(tmp_path),
+    mp.start_processes(_rank_main, args=(world, _store(tmp_path), case, w_local, d, str(tmp_path),
                                          chunks),
                        nprocs=world, join=True, start_method="spawn")
     import allreduce_compatible_gradient_global_b200 as gq
@@ -157,12 +155,11 @@ def test_worker0_offsets_the_uniform_streams(oracle):
     assert not np.array_equal(full[0:2], part)
 
 
-def test_int16_wire_is_refused():
+def test_int16_wire_is_refused(tmp_path):
     """NCCL cannot reduce 16-bit integers: the exchange refuses int16 sums up front."""
     import allreduce_compatible_gradient_global_b200 as gq
     from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("gloo", rank=0, world_size=1)
+    dist.init_process_group("gloo", init_method=_store(tmp_path), rank=0, world_size=1)
     try:
         with pytest.raises(ValueError):
             DataParallelStep(gq.GQConfig(s=127, bits=8, wire="int16"), 100, device="cpu")
@@ -170,9 +167,8 @@ def test_int16_wire_is_refused():
         dist.destroy_process_group()
 
 
-def _gather_main(rank, world, port, outdir):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+def _gather_main(rank, world, store, outdir):
+    dist.init_process_group("gloo", init_method=store, rank=rank, world_size=world)
     try:
         import oracle
         from allreduce_compatible_gradient_global_b200.dp import gather_rows
@@ -197,7 +193,7 @@ def test_gathered_log_codes_decode_like_one_process(oracle, tmp_path):
     the codes and max-abs values are all-gathered rank-major, and every rank's
     decoded sum equals the single-process decode of all workers, bit for bit."""
     world = 2
-    mp.start_processes(_gather_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+    mp.start_processes(_gather_main, args=(world, _store(tmp_path), str(tmp_path)), nprocs=world,
                        join=True, start_method="spawn")
     sizes = np.array([300, 120], np.int64)
     x = synthetic.make_gradients(4, int(sizes.sum()), "normal", seed=4).numpy()
@@ -225,9 +221,8 @@ class OracleNatOps:
         return 0
 
 
-def _nat_main(rank, world, port, outdir, w_local, n, sharded):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+def _nat_main(rank, world, store, outdir, w_local, n, sharded):
+    dist.init_process_group("gloo", init_method=store, rank=rank, world_size=world)
     try:
         import oracle
         from allreduce_compatible_gradient_global_b200.dp import DataParallelNatStep
@@ -250,7 +245,8 @@ def test_natural_exchange_sums_like_one_process(oracle, tmp_path, world, w_local
     rank the codes of its column shard, which it decodes and sums, and the fp32
     shard sums are all-gathered.  Either way every rank's sum equals the
     single-process sum of all workers, bit for bit."""
-    mp.start_processes(_nat_main, args=(world, _free_port(), str(tmp_path), w_local, n, sharded),
+    mp.start_processes(_nat_main,
+                       args=(world, _store(tmp_path), str(tmp_path), w_local, n, sharded),
                        nprocs=world, join=True, start_method="spawn")
     W = world * w_local
     x = synthetic.make_gradients(W, n, "student_t3", seed=6, seg=50, lo=-20, hi=3).numpy()
@@ -261,11 +257,10 @@ def test_natural_exchange_sums_like_one_process(oracle, tmp_path, world, w_local
             assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (t, r)
 
 
-def test_sharded_natural_exchange_needs_one_worker_per_rank():
+def test_sharded_natural_exchange_needs_one_worker_per_rank(tmp_path):
     """The column shards are slices of one code row: more rows per rank are refused."""
     from allreduce_compatible_gradient_global_b200.dp import DataParallelNatStep
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("gloo", rank=0, world_size=1)
+    dist.init_process_group("gloo", init_method=_store(tmp_path), rank=0, world_size=1)
     try:
         with pytest.raises(ValueError):
             DataParallelNatStep(100, w_local=2, device="cpu", sharded=True)

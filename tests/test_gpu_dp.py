@@ -11,8 +11,6 @@ more ranks need two or more GPUs; their host-side orchestration is covered by
 tests/test_dp_exchange.py with gloo on CPU.
 """
 import datetime
-import os
-import socket
 
 import numpy as np
 import pytest
@@ -25,10 +23,13 @@ from psgd_checks import check_step, host
 pytestmark = pytest.mark.gpu
 
 
-def _free_port():
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
+def _init_single_rank(tmp_path):
+    """A one-rank NCCL group whose rendezvous is a file store: no TCP port
+    that another process on the box could already hold."""
+    store = dist.FileStore(str(tmp_path / "store"), 1)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
 
 
 @pytest.fixture(scope="module")
@@ -62,12 +63,9 @@ def check_against_oracle(oracle, cfg, g, e_before, step, scale, out, e_after):
                                          scale_kind="maxabs"), True),
                                    (dict(levels="exp", L=8, bits=5, wire="f16"), False),
                                    (dict(s=127, bits=8, wire="f16"), True)])
-def test_nccl_single_rank_matches_oracle_and_fused_step(gq, oracle, kw, ef):
+def test_nccl_single_rank_matches_oracle_and_fused_step(gq, oracle, kw, ef, tmp_path):
     from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("nccl", rank=0, world_size=1,
-                            timeout=datetime.timedelta(seconds=60),
-                            device_id=torch.device("cuda", 0))
+    _init_single_rank(tmp_path)
     try:
         W, d = 4, 100_003
         cfg = gq.GQConfig(seed=7, ef=ef, **kw)
@@ -97,17 +95,14 @@ def test_nccl_single_rank_matches_oracle_and_fused_step(gq, oracle, kw, ef):
 
 
 @pytest.mark.parametrize("r", [1, 5])
-def test_nccl_single_rank_lqsgd_matches_oracle_and_whole_step(gq, oracle, r):
+def test_nccl_single_rank_lqsgd_matches_oracle_and_whole_step(gq, oracle, r, tmp_path):
     """The LQ-SGD exchange (all-gather of the factor codes) on one NCCL rank
     holding all W workers: every stage against the oracle (oracle/psgd.py and
     the C log quantizer) on the exchange's own inputs to that stage, and the
     result equal to gq_lqsgd_step bit for bit, state included."""
     from oracle import psgd
     from allreduce_compatible_gradient_global_b200.dp import DataParallelLqsgdStep
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("nccl", rank=0, world_size=1,
-                            timeout=datetime.timedelta(seconds=60),
-                            device_id=torch.device("cuda", 0))
+    _init_single_rank(tmp_path)
     try:
         W = 4
         sh = gq.PsgdShapes([256, 100], [128, 64], r)
@@ -146,16 +141,13 @@ def test_nccl_single_rank_lqsgd_matches_oracle_and_whole_step(gq, oracle, r):
 
 @pytest.mark.parametrize("chunks,kw", [(4, dict(s=15, bits=5, wire="int8", ef=True)),
                                        (3, dict(levels="exp", L=8, bits=5, wire="f16"))])
-def test_nccl_chunked_exchange_matches_oracle_and_unchunked(gq, oracle, chunks, kw):
+def test_nccl_chunked_exchange_matches_oracle_and_unchunked(gq, oracle, chunks, kw, tmp_path):
     """Chunk k + 1 is quantized while chunk k is all-reduced (NCCL, async);
     with each chunk drawing the uniforms of its own coordinates the mean and
     the error buffer equal the oracle's step on the whole row and are
     bit-identical to the unchunked exchange."""
     from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("nccl", rank=0, world_size=1,
-                            timeout=datetime.timedelta(seconds=60),
-                            device_id=torch.device("cuda", 0))
+    _init_single_rank(tmp_path)
     try:
         d = 1_000_003 - 3  # a multiple of 4, not of 128
         cfg = gq.GQConfig(seed=5, **kw)
@@ -184,16 +176,14 @@ def test_nccl_chunked_exchange_matches_oracle_and_unchunked(gq, oracle, chunks, 
                                                (3, 1, dict(s=15, bits=5, wire="int8", ef=True)),
                                                (4, 1, dict(levels="exp", L=8, bits=5,
                                                            wire="f16"))])
-def test_nccl_graph_replay_matches_oracle_and_eager_exchange(gq, oracle, chunks, w_local, kw):
+def test_nccl_graph_replay_matches_oracle_and_eager_exchange(gq, oracle, chunks, w_local, kw,
+                                                           tmp_path):
     """The exchange captured once in a CUDA graph (kernels, NCCL all-reduces and,
     chunked, their overlap) and replayed with new gradients written in place
     equals the oracle's step and the eager exchange step for step, error
     buffers included; the graph advances the device step word itself."""
     from allreduce_compatible_gradient_global_b200.dp import DataParallelStep
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("nccl", rank=0, world_size=1,
-                            timeout=datetime.timedelta(seconds=60),
-                            device_id=torch.device("cuda", 0))
+    _init_single_rank(tmp_path)
     graphed = None
     try:
         d = 100_003
@@ -226,15 +216,12 @@ def test_nccl_graph_replay_matches_oracle_and_eager_exchange(gq, oracle, chunks,
 
 
 @pytest.mark.parametrize("W,sharded", [(4, False), (1, True)])
-def test_nccl_single_rank_natural_exchange_matches_the_oracle(gq, oracle, W, sharded):
+def test_nccl_single_rank_natural_exchange_matches_the_oracle(gq, oracle, W, sharded, tmp_path):
     """DataParallelNatStep on one NCCL rank (all W workers gathered, or one
     worker through the all-to-all of the sharded form): the codes and the
     decoded sum equal the oracle's, bit for bit."""
     from allreduce_compatible_gradient_global_b200.dp import DataParallelNatStep
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("nccl", rank=0, world_size=1,
-                            timeout=datetime.timedelta(seconds=60),
-                            device_id=torch.device("cuda", 0))
+    _init_single_rank(tmp_path)
     try:
         n = 50_001
         x = synthetic.make_gradients(W, n, "student_t3", seed=8, device="cuda", seg=100, lo=-25,
