@@ -43,6 +43,55 @@ __device__ __forceinline__ uint4 philox_counter(unsigned long long q, uint32_t s
     return make_uint4((uint32_t)q, step, worker, (uint32_t)(q >> 32));
 }
 
+// philox10 on the counter (lo32 q, step, worker, hi32 q) with its first two
+// rounds split by what they depend on.  Round 0 multiplies lo32 q (one product
+// per coordinate block) and the worker word (one per worker and step).  Round
+// 1 multiplies the word that came from the worker product and the step (one
+// per worker) and the word that came from q (one per block).  Two XORs per
+// (worker, block) join the halves.
+struct PhiloxWorkerPart {
+    uint32_t bx;  // round-1 word x before the block half: lo(worker*M1) ^ k2
+    uint32_t hz;  // round-1 word z before the block half: hi(A*M0) ^ k3
+    uint32_t lw;  // round-1 word w: lo(A*M0), A = hi(worker*M1) ^ step ^ k0
+};
+struct PhiloxBlockPart {
+    uint32_t hx;  // hi(X*M1), X = hi(lo32q*M0) ^ hi32q ^ k1
+    uint32_t lx;  // round-1 word y: lo(X*M1)
+    uint32_t y;   // lo(lo32q*M0), joined into round-1 word z
+};
+
+__device__ __forceinline__ PhiloxWorkerPart philox_worker_part(uint32_t step, uint32_t worker,
+                                                               const RoundKeys& rk) {
+    const unsigned long long p1 = (unsigned long long)worker * 0xCD9E8D57ull;
+    const uint32_t A = (uint32_t)(p1 >> 32) ^ step ^ rk.k[0];
+    const unsigned long long p0 = (unsigned long long)A * 0xD2511F53ull;
+    return PhiloxWorkerPart{(uint32_t)p1 ^ rk.k[2], (uint32_t)(p0 >> 32) ^ rk.k[3], (uint32_t)p0};
+}
+
+__device__ __forceinline__ PhiloxBlockPart philox_block_part(unsigned long long q,
+                                                             const RoundKeys& rk) {
+    const unsigned long long p0 = (unsigned long long)(uint32_t)q * 0xD2511F53ull;
+    const uint32_t X = (uint32_t)(p0 >> 32) ^ (uint32_t)(q >> 32) ^ rk.k[1];
+    const unsigned long long p1 = (unsigned long long)X * 0xCD9E8D57ull;
+    return PhiloxBlockPart{(uint32_t)(p1 >> 32), (uint32_t)p1, (uint32_t)p0};
+}
+
+// philox10(philox_counter(q, step, worker), rk) from the two halves.
+__device__ __forceinline__ uint4 philox10_split(const PhiloxBlockPart& b,
+                                                const PhiloxWorkerPart& w,
+                                                const RoundKeys& rk) {
+    uint4 c = make_uint4(b.hx ^ w.bx, b.lx, b.y ^ w.hz, w.lw);
+#pragma unroll
+    for (int r = 2; r < 10; ++r) {
+        const unsigned long long p0 = (unsigned long long)c.x * 0xD2511F53ull;
+        const unsigned long long p1 = (unsigned long long)c.z * 0xCD9E8D57ull;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        c = make_uint4(hi1 ^ c.y ^ rk.k[2 * r], lo1, hi0 ^ c.w ^ rk.k[2 * r + 1], lo0);
+    }
+    return c;
+}
+
 // ---------------------------------------------------------------------------
 // Stochastic rounding.  A magnitude y >= 0 becomes floor(y + u) with
 // u = f * 2^-23, f the top 23 bits of a Philox word: that is floor(y) + 1

@@ -28,6 +28,14 @@
 // rounded level as a float (+-2^(idx-127), or +-0), and the top nine bits
 // (sign, exponent) index a 512-entry table of signed codes in shared memory.
 //
+// Philox: with W known at compile time (W = 8), the workers' halves of the
+// first two rounds (philox10_split) are computed once per block into shared
+// memory, and each coordinate block's half is shared by the W workers.  On
+// the uniform pass the executed instructions barely change (20.94 per element
+// against 20.71: one more 16-byte shared load per worker and block), but the
+// FMA-heavy pipe, which carries the multiplies, is busy 58.8% of cycles
+// instead of 60.9%, and the pass runs 0.9-1.4% faster (codes bit-identical).
+//
 // Tile order: each block's producer claims the next tile from a counter in
 // the workspace header, so every block works inside the same narrow window of
 // the rows however unevenly the blocks progress (measured on W = 8 rows of
@@ -196,6 +204,16 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     if (LEVELS != 0 && BITS != 0)
         for (int h = threadIdx.x; h < kExpTableSize; h += kTmaThreads)
             code_table[h] = exp_table_entry(h, a.L);  // |code| <= 15
+    // The unrolled kernel's workers' halves of Philox's first two rounds, once
+    // per block (philox10_split); each coordinate block's half is shared by
+    // all WT workers.
+    __shared__ uint4 worker_part[WT > 0 ? WT : 1];
+    if (WT > 0 && threadIdx.x < WT) {
+        const uint32_t st = a.step_dev ? __ldg(a.step_dev) : a.step;
+        const uint32_t wid = WOFF ? a.worker0 + threadIdx.x : threadIdx.x;
+        const PhiloxWorkerPart p = philox_worker_part(st, wid, a.rk);
+        worker_part[threadIdx.x] = make_uint4(p.bx, p.hz, p.lw, 0u);
+    }
     __syncthreads();
 
     if (warp == kTmaComputeWarps) {
@@ -315,6 +333,8 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 (unsigned long long)(blk << 5) + (unsigned)lane + (WOFF ? a.q0 : 0ull);
             const float* stage = buf + (size_t)s * rows * kTmaTile + warp * 128 + lane * 4;
             unsigned char* codes_blk = a.codes + blk * (16 * BITS);
+            const PhiloxBlockPart bpart =
+                WT > 0 ? philox_block_part(q, a.rk) : PhiloxBlockPart{0u, 0u, 0u};
             // uniform levels accumulate the biased patterns (code + kCodeBias);
             // exponential levels accumulate the rounded levels as floats in
             // units of 2^-126 per finest level (exact: integers below 2^24
@@ -333,7 +353,13 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 }
                 // WOFF = 0: the worker word is the loop constant w (the common case)
                 const uint32_t wid = WOFF ? a.worker0 + (uint32_t)w : (uint32_t)w;
-                const uint4 rnd = philox10(philox_counter(q, step, wid), a.rk);
+                uint4 rnd;
+                if (WT > 0) {
+                    const uint4 wp = worker_part[WT > 0 ? w : 0];
+                    rnd = philox10_split(bpart, PhiloxWorkerPart{wp.x, wp.y, wp.z}, a.rk);
+                } else {
+                    rnd = philox10(philox_counter(q, step, wid), a.rk);
+                }
                 unsigned char* cdst = codes_blk + (long long)w * row_bytes;
                 float4 qv;  // the values Q(v) in units of c, as floats
                 if (LEVELS == 0) {
