@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libgq.so")
 
 SOURCES = ["gq_api.cu", "gq_kernels.cu", "gq_quant_tma.cu", "gq_bucket.cu", "gq_psgd.cu", "gq_logq.cu", "gq_noalloc.cu", "gq_nat.cu"]
-HEADERS = ["gq_device.cuh", "gq_internal.h", "gq_psgd.h", "gq_nat.h"]
+HEADERS = ["gq_device.cuh", "gq_internal.h", "gq_pdl.cuh", "gq_psgd.h", "gq_nat.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -15,6 +15,7 @@
 #include <cfloat>
 
 #include "gq_internal.h"
+#include "gq_pdl.cuh"
 
 namespace gq {
 
@@ -117,6 +118,10 @@ __device__ __forceinline__ T ld_norm(const T* p) {
 
 template <int KIND, bool HAS_E, bool VEC>
 __global__ void __launch_bounds__(kThreads, 8) norm_kernel(const __grid_constant__ NormArgs a) {
+    // the rows may come from the previous kernel in the stream; the fused pass
+    // that follows may be scheduled as soon as every block is running
+    pdl_wait();
+    pdl_launch_dependents();
     const int w = blockIdx.y;
     const int b = blockIdx.x;
     const float* gw = a.g + (long long)w * a.d;
@@ -277,7 +282,9 @@ int norm_resident_blocks(int kind, bool has_e, bool vec) {
 cudaError_t launch_norm(const NormArgs& a, bool vec, cudaStream_t st) {
     dim3 grid(a.nb, a.W);
     const bool he = a.e != nullptr;
-#define GQ_NORM(K, E, V) norm_kernel<K, E, V><<<grid, kThreads, 0, st>>>(a)
+    const bool pdl = pdl_allowed(st);
+#define GQ_NORM(K, E, V) \
+    return launch_with_pdl(norm_kernel<K, E, V>, grid, dim3(kThreads), 0, st, pdl, a)
     if (a.kind == 0) {
         if (he) { if (vec) GQ_NORM(0, true, true); else GQ_NORM(0, true, false); }
         else    { if (vec) GQ_NORM(0, false, true); else GQ_NORM(0, false, false); }

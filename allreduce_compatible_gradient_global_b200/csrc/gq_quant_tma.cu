@@ -48,6 +48,7 @@
 #include <type_traits>
 
 #include "gq_internal.h"
+#include "gq_pdl.cuh"
 
 namespace gq {
 
@@ -204,6 +205,10 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
     if (LEVELS != 0 && BITS != 0)
         for (int h = threadIdx.x; h < kExpTableSize; h += kTmaThreads)
             code_table[h] = exp_table_entry(h, a.L);  // |code| <= 15
+    // everything above touched shared memory only: now wait for the previous
+    // kernel in the stream (the norm pass) and let the next one be scheduled
+    pdl_wait();
+    pdl_launch_dependents();
     // The unrolled kernel's workers' halves of Philox's first two rounds, once
     // per block (philox10_split); each coordinate block's half is shared by
     // all WT workers.
@@ -459,8 +464,8 @@ static cudaError_t launch_tma_inst(const QuantArgs& a, int stages, int grid, cud
     static int limits[64] = {};
     cudaError_t e = ensure_dynamic_smem((const void*)kern, smem, limits);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTmaThreads, smem, st>>>(a, stages);
-    return cudaGetLastError();
+    return launch_with_pdl(kern, dim3(grid), dim3(kTmaThreads), smem, st, pdl_allowed(st), a,
+                           stages);
 }
 
 template <int LEVELS, int BITS, bool EF>

@@ -72,7 +72,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "quant_kernel_traffic.json")
 KERNEL_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_quant_tma.cu",
                   "allreduce_compatible_gradient_global_b200/csrc/gq_kernels.cu",
                   "allreduce_compatible_gradient_global_b200/csrc/gq_device.cuh",
-                  "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h"]
+                  "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h",
+                  "allreduce_compatible_gradient_global_b200/csrc/gq_pdl.cuh"]
 LOGQ_SOURCES = ["allreduce_compatible_gradient_global_b200/csrc/gq_logq.cu",
                 "allreduce_compatible_gradient_global_b200/csrc/gq_device.cuh",
                 "allreduce_compatible_gradient_global_b200/csrc/gq_internal.h"]
