@@ -275,18 +275,21 @@ class Workload:
             self.drawn = i
 
     def step(self, i, ev=None, codes=True):
+        """One step.  ev: two events (around the step) or three (around each
+        kernel too; an event between the kernels keeps the fused pass from
+        being scheduled before the norm pass ends)."""
         gq, cfg, buf, st = self.gq, self.cfg, self.buf, self.stream
         cfg.step = i
         if ev is not None:
             ev[0].record(st)
         gq.gq_global_norm(self.g, buf.e if cfg.ef else None, cfg, buf.scale, buf.norms, buf.ws,
                           st)
-        if ev is not None:
+        if ev is not None and len(ev) == 3:
             ev[1].record(st)
         gq.gq_quantize_aggregate(self.g, buf.e, cfg, buf.scale, buf.codes if codes else None,
                                  buf.sum, buf.out, buf.ws, st)
         if ev is not None:
-            ev[2].record(st)
+            ev[-1].record(st)
 
     def check(self, what):
         if self.gq.gq_get_device_status(self.buf.ws, self.stream) != self.gq.GQ_OK:
@@ -316,17 +319,23 @@ def time_workload(wk, K, warmup, world, flush=None):
         wk.step(i)
     wk.check("warm-up")
     if between is not None:
-        evs = [_events(3) for _ in range(K)]
+        spans_ev = [_events(2) for _ in range(K)]
         _sync(world)
         for i in range(K):
             between(warmup + i)
-            wk.step(warmup + i, evs[i])
+            wk.step(warmup + i, spans_ev[i])
         _sync(world)
-        spans = [e[0].elapsed_time(e[2]) for e in evs]
+        spans = [e[0].elapsed_time(e[1]) for e in spans_ev]
         job_ms = job_time_ms(sum(spans), world, dev)
-        note = ("each step timed by CUDA events around its two kernels; "
+        evs = [_events(3) for _ in range(K)]
+        for i in range(K):
+            between(warmup + K + i)
+            wk.step(warmup + K + i, evs[i])
+        torch.cuda.synchronize()
+        note = ("value, ms_per_step: each step timed by CUDA events around its two kernels; "
                 + ("the next step's fresh gradient is drawn between the timed spans"
-                   if wk.fresh else "L2 flushed between the timed spans"))
+                   if wk.fresh else "L2 flushed between the timed spans")
+                + "; roofline avg_launch_ms: K further steps with events around each kernel")
     else:
         t0, t1 = _events(2)
         _sync(world)
