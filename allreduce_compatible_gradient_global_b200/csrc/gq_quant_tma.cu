@@ -36,14 +36,17 @@
 // FMA-heavy pipe, which carries the multiplies, is busy 58.8% of cycles
 // instead of 60.9%, and the pass runs 0.9-1.4% faster (codes bit-identical).
 //
-// Tile order: each block's producer claims the next tile from a counter in
-// the workspace header, so every block works inside the same narrow window of
-// the rows however unevenly the blocks progress (measured on W = 8 rows of
-// 2^26 to 2^30 coordinates: 3-4% faster than block b taking tiles b, b + grid,
-// b + 2 grid, ...).  The last producer to finish puts the counter back to zero,
-// so two launches must not share a workspace at the same time.  The
-// per-bucket instantiation keeps the static order: it prefetches the next
-// block's scale a tile ahead.
+// Tile order: block b starts with tile b, then its producer claims each next
+// tile from a counter in the workspace header (tiles grid, grid + 1, ...), so
+// every block works inside the same narrow window of the rows however unevenly
+// the blocks progress (measured on W = 8 rows of 2^26 to 2^30 coordinates: 3-4%
+// faster than block b taking tiles b, b + grid, b + 2 grid, ...).  Taking the
+// first tile without a claim keeps the claim's round trip out of the first
+// copy (8 x 2^16 coordinates, one tile per block: 14.4 us per step against
+// 15.3 us; no change at 8 x 25.6 M).  The last producer to finish puts the
+// counter back to zero, so two launches must not share a workspace at the
+// same time.  The per-bucket instantiation keeps the static order: it
+// prefetches the next block's scale a tile ahead.
 #include <cfloat>
 #include <type_traits>
 
@@ -229,7 +232,10 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
             uint32_t round = 0;
             long long issued = 0;
             bool ok = true;
-            long long t = kDynamic ? (long long)atomicAdd(&a.hdr->tile_next, 1u) : blockIdx.x;
+            // the first tile is the block's own (the grid never exceeds the tile
+            // count), so the first copy waits for no claim; later tiles are
+            // claimed beyond the first wave
+            long long t = blockIdx.x;
             for (;; ++issued) {
                 if (!kDynamic && t >= ntiles) break;
                 if (round > 0 && !mbar_wait_bounded(empty0 + 8 * s, (round - 1) & 1u, a.hdr)) {
@@ -244,7 +250,8 @@ __global__ void __launch_bounds__(kTmaThreads, GQ_TMA_MIN_BLOCKS)
                 const long long j0 = t * kTmaTile;
                 // claim the next tile now, so the atomic's round trip overlaps this one
                 const long long t_next =
-                    kDynamic ? (long long)atomicAdd(&a.hdr->tile_next, 1u) : t + gridDim.x;
+                    kDynamic ? (long long)gridDim.x + atomicAdd(&a.hdr->tile_next, 1u)
+                             : t + gridDim.x;
                 tile_of[s] = t;
                 const long long n = a.d - j0 < kTmaTile ? a.d - j0 : kTmaTile;
                 const uint32_t bytes = (uint32_t)(n * sizeof(float));
