@@ -20,6 +20,7 @@ This file is collected last, so a run that stops at the first failure has run
 every other test before it.
 """
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -75,12 +76,20 @@ def test_noalloc_matches_workspace_form_and_oracle(gq, oracle, W, d, kind, ef):
         scale = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
         norms = torch.full((W,), -1.0, dtype=torch.float64, device="cuda")
         torch.cuda.synchronize()
-        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
-        assert call_noalloc(gq, g, e, cfg, scale, norms) == gq.GQ_OK
-        torch.cuda.synchronize()
+        # no collection of unrelated garbage (tensors of earlier tests) may free
+        # memory between the two readings
+        gc.collect()
+        gc.disable()
+        try:
+            free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+            assert call_noalloc(gq, g, e, cfg, scale, norms) == gq.GQ_OK
+            torch.cuda.synchronize()
+            free1, alloc1 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+        finally:
+            gc.enable()
         if call == 1:  # the first call may load the module; the second allocates nothing
-            assert torch.cuda.mem_get_info()[0] == free0
-            assert torch.cuda.memory_allocated() == alloc0
+            assert free1 == free0
+            assert alloc1 == alloc0
         S, n = scale.item(), norms.cpu().numpy()
         assert S == S_ref, (call, S, S_ref)
         assert np.array_equal(n.view(np.uint64), n_ref.view(np.uint64)), call
